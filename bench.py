@@ -1,0 +1,463 @@
+"""Benchmark of one Medusa verification step (heads + top-k, tree build, tree
+attention, posterior, KV compaction) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-graph]
+
+A step is one ``medusa_step`` call over one batch of synthetic inputs already
+resident in HBM (the Vicuna-7B-shaped batch-1 workload by default).  Each
+rank runs its own replica (sequences are independent, so the path shards
+with no exchange: weak scaling).  Rank 0 prints one JSON line.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload (rank 0 only) and prints the same metric.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+REPO = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, REPO)
+
+METRIC = "Medusa step µs (heads+tree-attn+posterior) at 7B shape; % of HBM roofline"
+NOMINAL_HBM_GBS = 8000.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default=None)
+    p.add_argument("--no-graph", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(REPO, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+def subseeds(name):
+    path = os.path.join(REPO, "tests", "golden", "subseeds.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        if name in d:
+            return d[name]["sub_h"], d[name]["sub_logits"]
+    return 0, 0
+
+
+def workload_config(w, graph=None):
+    cfg = {"workload": w.name, "B": w.B, "d": w.d, "V": w.V, "K": w.K, "topk": w.topk, "T": w.T,
+           "layers": w.layers, "H": w.H, "hd": w.hd,
+           "L": int(w.prefix) if w.prefix is not None else list(w.prefix_range),
+           "mode": w.modes[0], "metric_bytes": w.metric_bytes(),
+           "l2": "inputs larger than L2 (%.2f GB read per step vs 126 MB L2); no flush" % (w.metric_bytes() / 1e9)}
+    if graph is not None:
+        cfg["graph"] = graph
+    return cfg
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# oracle on a bounded sample (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+
+class OracleSample:
+    """The fp64 oracle on one bounded sample of a step, extrapolated to a full step.
+
+    Heads, top-k, candidate assembly and the posterior run in full; tree
+    attention and KV compaction run on ``n_slices`` (layer, sequence, head)
+    slices spread over the cache and are scaled by total/sampled slices.
+    """
+
+    def __init__(self, w, n_slices=8):
+        import numpy as np
+        import oracle.medusa_oracle as O
+        from synth import inputs as I
+        self.np, self.O, self.I, self.w = np, O, I, w
+        sub_h, sub_l = subseeds(w.name)
+        self.tr = O.tree_tables(O.ranksum_choices(w.K, w.topk, w.n_nodes), w.K, w.topk)
+        self.h = I.values(I.hidden(w, sub_h))
+        self.b1 = I.values(I.b1(w))
+        self.W1 = [I.values(I.w1(w, k)) for k in range(w.K)]
+        self.Wo = [I.values(I.wout(w, k)) for k in range(w.K)]
+        self.root = I.root_tokens(w)
+        self.lens = w.prefix_lens()
+        total = w.layers * w.B * w.H
+        rng = np.random.default_rng(0)
+        picks = sorted(set([0, total - 1] + list(rng.choice(total, size=min(total, n_slices) - 2, replace=False))))
+        self.slices = []
+        for s in picks:
+            e, lb = s % w.H, s // w.H
+            l, b = lb // w.B, lb % w.B
+            n = int(self.lens[b]) + w.T
+            self.slices.append((l, b, e, I.q_slice(w, l, b, e), I.values(I.kv_slice(w, "k", l, b, e, n)),
+                                I.values(I.kv_slice(w, "v", l, b, e, n))))
+        self.scale_slices = total / len(self.slices)
+        self.sub_l = sub_l
+        self.logits = None
+        self.cores = 1
+        self.desc = (f"heads, top-k, tree and posterior in full; attention and KV compaction on "
+                     f"{len(self.slices)} of {total} (layer, seq, head) slices, scaled x{self.scale_slices:.0f}; "
+                     f"fp64, 1 BLAS thread")
+
+    def step_seconds(self):
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(1):
+            return self._step_seconds()
+
+    def _step_seconds(self):
+        np, O, w = self.np, self.O, self.w
+        t0 = time.perf_counter()
+        zs = [O.medusa_head_one(self.h, self.W1[k], self.b1[k], self.Wo[k])[1] for k in range(w.K)]
+        z = np.stack(zs, 1)
+        ids, _ = O.topk_desc(z, w.topk)
+        toks, cand, _ = O.build_tree(self.tr, self.root, ids, self.lens)
+        t_full = time.perf_counter() - t0
+        if self.logits is None:      # input synthesis, not timed
+            self.logits = self.I.base_logits(w, toks, self.tr["parent"], self.sub_l)
+        t1 = time.perf_counter()
+        post = O.evaluate_posterior(self.tr, self.logits, cand, w.modes[0], w.temperature, w.eps, w.alpha)
+        t_full += time.perf_counter() - t1
+        t2 = time.perf_counter()
+        for (l, b, e, q, k, v) in self.slices:
+            O.tree_attention_slice(self.tr, q, k, v, int(self.lens[b]), O.attention_scale(w.hd))
+            a = int(post["accept_len"][b])
+            L = int(self.lens[b])
+            rows = [L + int(self.tr["retrieve"][post["best_path"][b], j]) for j in range(a + 1)]
+            k2, v2 = k.copy(), v.copy()
+            k2[L:L + a + 1] = k[rows]
+            v2[L:L + a + 1] = v[rows]
+        t_sample = time.perf_counter() - t2
+        return t_full + t_sample * self.scale_slices
+
+
+def run_reference(a, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    samp = OracleSample(w)
+    for _ in range(a.warmup):
+        samp.step_seconds()
+    times = [samp.step_seconds() for _ in range(a.steps)]
+    us = statistics.median(times) * 1e6
+    line = {"metric": METRIC, "impl": "reference", "value": us, "unit": "us", "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w),
+            "cpu_baseline": {"value": us, "unit": "us", "cores": samp.cores, "kind": "oracle", "sample": samp.desc},
+            "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+
+def run_ours(a, w):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev_index = torch.cuda.current_device()
+
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("medusa_b200_build",
+                                                  os.path.join(REPO, "speculative_decoding_heads_b200", "_build.py"))
+    bmod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bmod)
+    if rank == 0 or world == 1:
+        bmod.build_all()
+    if world > 1:
+        dist.barrier()
+    import speculative_decoding_heads_b200 as mb
+    from synth import device, workloads as W
+
+    sub_h, sub_l = subseeds(w.name)
+    choices = mb.medusa_tree_choices_ranksum(w.K, w.topk, w.n_nodes)
+    tree = mb.Tree(choices, w.K, w.topk)
+    t = device.materialise(w, sub_h=sub_h, sub_logits=sub_l, with_head_logits=False)
+    device.tree_outputs(t, w.B, tree.T, tree.P, tree.D)
+    mode = mb.MEDUSA_TYPICAL if w.modes[0] == "typical" else mb.MEDUSA_GREEDY
+    args = mb.make_step_args(tree, t, mode, w.temperature, w.eps, w.alpha)
+    ws = mb.workspace(mb.medusa_step_workspace_size(args))
+    # Plant head/base agreement once the tree tokens are known (input synthesis).
+    hws = mb.workspace(mb.medusa_heads_workspace_size(w.B, w.d, w.V, w.K, w.topk))
+    mb.medusa_heads_topk(t["h"], t["W1"], t["b1"], t["Wout"], w.topk, t["topk_ids"], t["topk_vals"], hws)
+    mb.medusa_build_tree(tree, t["root_tokens"], t["topk_ids"], t["seq_lens"], t["tree_tokens"], t["candidates"],
+                         t["position_ids"])
+    parent = device.parent_tensor(tree.tables()["parent"])
+    device.plant(t["base_logits"], t["tree_tokens"], parent, w.agreement, w.seed + 7919 * sub_l)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream()
+    launches_per_step = (w.B + 3) // 4 + 1 + 1 + 2 + 2
+
+    def step():
+        t["seq_lens"].copy_(t["seq_lens0"])
+        mb.medusa_step(args, ws)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, a.warmup)):
+            step()
+    torch.cuda.synchronize()
+    st, det = mb.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} detail {det} after warm-up")
+
+    graph = None
+    if not a.no_graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step()
+            graph = g
+            with torch.cuda.stream(stream):
+                for _ in range(a.warmup):
+                    graph.replay()
+            torch.cuda.synchronize()
+        except Exception as ex:   # capture not possible: time eager launches
+            print(f"# graph capture failed, timing eager launches: {ex}", file=sys.stderr)
+            graph = None
+            torch.cuda.synchronize()
+
+    def run_k(k):
+        with torch.cuda.stream(stream):
+            for _ in range(k):
+                graph.replay() if graph is not None else step()
+
+    # ---- timed region --------------------------------------------------
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev_index)
+    with sampler:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        run_k(a.steps)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    ms = ev0.elapsed_time(ev1) / a.steps
+    if world > 1:
+        tm = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        ms = float(tm.item())
+    clocks = sampler.summary()
+    st, det = mb.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} detail {det} after the timed region")
+
+    # ---- per-stage breakdown (eager, CUDA events on the launching stream) ----
+    peak, peak_kind = load_peaks()
+    stage = {}
+    reps = max(5, min(a.steps, 30))
+    with torch.cuda.stream(stream):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        acc = [0.0] * 5
+        attn_ws = mb.workspace(mb.medusa_attention_workspace_size(tree, w.layers, w.B, w.H, w.hd,
+                                                                   mb.MEDUSA_BF16 if w.dtype == "bf16" else mb.MEDUSA_F32))
+        pws = mb.workspace(mb.medusa_posterior_workspace_size(tree, w.B))
+        for _ in range(reps):
+            t["seq_lens"].copy_(t["seq_lens0"])
+            evs[0].record(stream)
+            mb.medusa_heads_topk(t["h"], t["W1"], t["b1"], t["Wout"], w.topk, t["topk_ids"], t["topk_vals"], hws)
+            evs[1].record(stream)
+            mb.medusa_build_tree(tree, t["root_tokens"], t["topk_ids"], t["seq_lens"], t["tree_tokens"],
+                                 t["candidates"], t["position_ids"])
+            evs[2].record(stream)
+            mb.medusa_tree_attention(tree, t["q"], t["k_cache"], t["v_cache"], t["seq_lens"], w.hd ** -0.5,
+                                     t["attn_out"], attn_ws)
+            evs[3].record(stream)
+            mb.medusa_evaluate_posterior(tree, t["base_logits"], t["candidates"], mode, t["best_path"],
+                                         t["accept_len"], t["accepted_tokens"], t["next_token"], pws,
+                                         w.temperature, w.eps, w.alpha)
+            evs[4].record(stream)
+            mb.medusa_accept_kv(tree, t["k_cache"], t["v_cache"], t["seq_lens"], t["best_path"], t["accept_len"])
+            evs[5].record(stream)
+            torch.cuda.synchronize()
+            for i in range(5):
+                acc[i] += evs[i].elapsed_time(evs[i + 1])
+    names = ["heads_topk", "build_tree", "tree_attention", "posterior", "accept_kv"]
+    stage = {n: acc[i] / reps * 1e3 for i, n in enumerate(names)}
+    esz = 2 if w.dtype == "bf16" else 4
+    head_bytes = w.K * (w.d * w.d + w.d + w.V * w.d) * esz
+    kv_bytes = w.metric_bytes() - head_bytes
+    heads_gbs = head_bytes / (stage["heads_topk"] * 1e-6) / 1e9
+    attn_gbs = kv_bytes / (stage["tree_attention"] * 1e-6) / 1e9
+    traffic = None
+    tpath = os.path.join(REPO, "profiles", "heads_topk_traffic.json")
+    if os.path.exists(tpath):
+        tj = json.load(open(tpath))
+        if tj.get("workload") == w.name and tj.get("kernel_rev") == kernel_revision():
+            traffic = tj.get("dram_bytes_per_launch")
+
+    # ---- end to end through the public API with host buffers ----------
+    e2e = None
+    if not a.no_e2e:
+        pin = lambda x: x.cpu().pin_memory()
+        host_in = {"h": pin(t["h"]), "root_tokens": pin(t["root_tokens"]), "seq_lens": pin(t["seq_lens0"]),
+                   "q": pin(t["q"]), "base_logits": pin(t["base_logits"])}
+        lens = t["seq_lens0"].cpu()
+        kt = torch.stack([t["k_cache"][:, b, :, int(lens[b]):int(lens[b]) + w.T] for b in range(w.B)], 1)
+        vt = torch.stack([t["v_cache"][:, b, :, int(lens[b]):int(lens[b]) + w.T] for b in range(w.B)], 1)
+        host_in["k_tree"], host_in["v_tree"] = pin(kt), pin(vt)
+        host_out = {k: torch.empty_like(t[k], device="cpu").pin_memory()
+                    for k in ("best_path", "accept_len", "accepted_tokens", "next_token")}
+        dev_map = dict(t)
+        h2d = sum(x.numel() * x.element_size() for x in host_in.values())
+        d2h = sum(x.numel() * x.element_size() for x in host_out.values())
+        e_ms = []
+        for i in range(a.warmup + a.steps):
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            mb.medusa_step_from_host(args, ws, host_in, dev_map, host_out, stream)
+            s1.record(stream)
+            s1.synchronize()
+            if i >= a.warmup:
+                e_ms.append(s0.elapsed_time(s1))
+        e_ms_max = statistics.mean(e_ms)
+        if world > 1:
+            tm = torch.tensor([e_ms_max], device="cuda")
+            dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+            e_ms_max = float(tm.item())
+        e2e = {"value": e_ms_max * 1e3, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # ---- CPU baseline (rank 0, N = 1 only) -----------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        samp = OracleSample(w)
+        secs = [samp.step_seconds() for _ in range(2)]
+        cpu = {"value": min(secs) * 1e6, "unit": "us", "cores": samp.cores, "kind": "oracle", "sample": samp.desc}
+
+    if world > 1:
+        dist.barrier()
+        del graph
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    us = ms * 1e3
+    line = {
+        "metric": METRIC, "value": us, "unit": "us", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded counter-based generator; Vicuna-shaped random weights and KV)",
+        "config": workload_config(w, graph is not None),
+        "hbm_roofline_frac_8tbs": w.metric_bytes() / (us * 1e-6) / 1e9 / NOMINAL_HBM_GBS,
+        "achieved_step_gbs": w.metric_bytes() / (us * 1e-6) / 1e9,
+        "tree_tokens_per_s": world * w.B * w.T / (us * 1e-6),
+        "stage_us": stage,
+        "roofline": {"bound": "hbm", "kernel": "heads_topk", "achieved": heads_gbs, "peak": peak,
+                     "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback 6650 GB/s", "unit": "GB/s", "frac": heads_gbs / peak, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": head_bytes},
+        "attention_roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
+                               "frac": attn_gbs / peak, "algorithmic_bytes_per_launch": kv_bytes},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * a.steps, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def kernel_revision():
+    """Hash of the kernel sources; ncu traffic figures are valid only for the revision they were taken on."""
+    import hashlib
+    h = hashlib.sha1()
+    csrc = os.path.join(REPO, "speculative_decoding_heads_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def main():
+    a = parse()
+    from synth import workloads as W
+    w = W.get(a.workload or W.BENCH_WORKLOAD)
+    if a.impl == "reference":
+        return run_reference(a, w)
+    return run_ours(a, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

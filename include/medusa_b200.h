@@ -1,0 +1,283 @@
+/*
+ * libmedusa_b200 -- one Medusa verification step on NVIDIA B200 (sm_100a).
+ *
+ * The step (sources are cited by page title and section):
+ *   S1-S3  medusa_heads_topk        K residual heads on the last hidden state,
+ *                                   each with its own vocabulary projection,
+ *                                   and the top-k tokens of every head.
+ *          ["Medusa API参考：核心函数与类详解", MedusaConfig / MedusaModelABC;
+ *           "Medusa — 让大模型自己同时猜好几个 token", 是什么 and 核心要点]
+ *   S4     medusa_build_tree        candidate tree tokens (tree_indices gather),
+ *                                   per-path candidates (retrieve_indices) and
+ *                                   position ids.
+ *          ["Medusa API参考", 核心功能函数: generate_candidates, tree_decoding]
+ *   S5     medusa_tree_attention    attention of the T tree tokens against the
+ *                                   cached prefix and their own ancestors.
+ *          ["Medusa — 让大模型…", 核心要点 (tree attention) and 实践案例 case 3]
+ *   S6     medusa_evaluate_posterior greedy or typical acceptance, best path,
+ *                                   accept length, accepted tokens, next token.
+ *          ["Medusa API参考", evaluate_posterior; "Medusa — 让大模型…", 核心要点,
+ *           实践案例 case 1 step 4, 学到什么]
+ *   S7     medusa_accept_kv         move the accepted path's K/V rows to the
+ *                                   end of the cached prefix.
+ *          ["Medusa — 让大模型…", 实践案例 case 1 step 4]
+ *   medusa_step                     S1..S7 in order on one stream.
+ *
+ * Conventions shared by every call:
+ *   - Tensors are caller-owned DEVICE pointers unless a comment says "host".
+ *     No call allocates device memory, except medusa_tree_create (which owns
+ *     the tree tables it uploads).  No call synchronises its stream; all work
+ *     is enqueued on the caller's cudaStream_t.
+ *   - Arguments are checked on the host before any launch; a bad argument
+ *     returns MEDUSA_ERR_INVALID_ARG / MEDUSA_ERR_UNSUPPORTED and launches
+ *     nothing.  A launch failure returns MEDUSA_ERR_CUDA.  Conditions that
+ *     only the device can see (a sequence length that overflows the cache, a
+ *     bounded wait that ran out) set a per-device status word that
+ *     medusa_device_status() reads back; such a call still returns MEDUSA_OK.
+ *   - medusa_last_error() gives a thread-local message for the last failure.
+ *   - Index tensors are int32.  Logits (head and base) are always fp32.
+ *   - "workspace" buffers are caller-owned device memory of at least the size
+ *     the matching *_workspace_size() call returns, 256-byte aligned.  They
+ *     must be zero-filled once before their first use (cudaMemsetAsync); each
+ *     call leaves its counters at zero again when it completes.  After a call
+ *     that reported a device-side error, zero the workspace again.  Calls
+ *     that share a workspace must not run concurrently.
+ *
+ * Shapes (contiguous, row-major):
+ *   h       [B, d]            hidden state at the last cached position
+ *   W1      [K, d, d]         residual-block weight, out x in
+ *   b1      [K, d]            residual-block bias
+ *   Wout    [K, V, d]         per-head vocabulary projection, no bias
+ *   q, out  [layers, B, T, H, hd]           tree queries / attention output (fp32)
+ *   k_cache, v_cache [layers, B, H, Lcap, hd] with the tree's own K/V already
+ *                     at rows seq_lens[b] .. seq_lens[b]+T-1 of every slice
+ *   base logits [B, T, V]     base-model logits at every tree node (fp32)
+ */
+#ifndef MEDUSA_B200_H
+#define MEDUSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MEDUSA_ABI_VERSION 1
+#define MEDUSA_MAX_T 256     /* tree tokens including the root */
+#define MEDUSA_MAX_K 16      /* heads (so tree depth <= 16) */
+#define MEDUSA_MAX_TOPK 32   /* candidates per head */
+#define MEDUSA_MAX_B 64      /* sequences per call */
+
+typedef enum medusa_status {
+  MEDUSA_OK = 0,
+  MEDUSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad tree, bad mode */
+  MEDUSA_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels handle */
+  MEDUSA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  MEDUSA_ERR_TIMEOUT = 4,       /* device status: a bounded wait ran out */
+  MEDUSA_ERR_DEVICE_CHECK = 5   /* device status: a device-side check failed */
+} medusa_status_t;
+
+typedef enum medusa_dtype { MEDUSA_F32 = 0, MEDUSA_BF16 = 1 } medusa_dtype_t;
+
+typedef enum medusa_mode { MEDUSA_GREEDY = 0, MEDUSA_TYPICAL = 1 } medusa_mode_t;
+
+typedef struct medusa_tree medusa_tree_t;
+
+/* Thread-local text of the last error raised by a call on this thread. */
+const char* medusa_last_error(void);
+
+/* MEDUSA_ABI_VERSION of the loaded library. */
+int medusa_abi_version(void);
+
+/* Reads (and, when clear != 0, resets) the current device's status word:
+ * MEDUSA_OK, MEDUSA_ERR_TIMEOUT or MEDUSA_ERR_DEVICE_CHECK.  Synchronises the
+ * device.  *detail receives a kernel-specific code (may be NULL). */
+medusa_status_t medusa_device_status(int32_t* status, int32_t* detail, int clear);
+
+/* ------------------------------------------------------------------------ */
+/* Candidate tree                                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Host.  The static tree used by the Vicuna-shaped workloads: all rank tuples
+ * of length 1..K with entries in [0, topk), ordered by (rank sum, length,
+ * lexicographic), first n_nodes kept (a prefix-closed set).
+ * ranks: host [n_nodes * K], tuple i in ranks[i*K .. i*K+lens[i]-1], rest 0;
+ * lens: host [n_nodes].  The pages name the tree (medusa_choices of
+ * medusa_generate, "Medusa API参考") but not this construction; it is the
+ * reading used for the Vicuna-shaped workloads.  Errors: INVALID_ARG when
+ * n_nodes exceeds the number of tuples or MEDUSA_MAX_T-1. */
+medusa_status_t medusa_tree_choices_ranksum(int K, int topk, int n_nodes,
+                                            int32_t* ranks, int32_t* lens);
+
+/* Host (+ device when upload != 0).  Builds the tree tables from n_nodes rank
+ * tuples (same packing as above; any order).  Node 0 is the root; nodes are
+ * laid out breadth first, (length, lexicographic).  Node (r1..rj) takes head
+ * j's rank-rj token ["Medusa — 让大模型…", 核心要点; 实践案例 case 3].
+ * Checks: 1 <= len <= K <= MEDUSA_MAX_K, 0 <= rank < topk <= MEDUSA_MAX_TOPK,
+ * no duplicates, every tuple's parent present, T = n_nodes+1 <= MEDUSA_MAX_T.
+ * With upload != 0 the tables are copied (synchronously) to the current
+ * device and the tree may only be used on that device.  The caller owns
+ * *out and frees it with medusa_tree_destroy. */
+medusa_status_t medusa_tree_create(const int32_t* ranks, const int32_t* lens, int n_nodes,
+                                   int K, int topk, int upload, medusa_tree_t** out);
+
+void medusa_tree_destroy(medusa_tree_t* tree);
+
+/* Host.  T tree tokens (root included), P root-to-leaf paths, D max depth. */
+medusa_status_t medusa_tree_info(const medusa_tree_t* tree, int32_t* T, int32_t* P, int32_t* D);
+
+/* Host copies of the tables (any pointer may be NULL):
+ *   tree_indices [T]  index into [root, head1 top-k, ..., headK top-k]
+ *   parent [T] (-1 for the root), depth [T]
+ *   retrieve [P * (D+1)]  node ids along each path, leaf order, padded -1
+ *   anc [T * ((T+63)/64)] bit j of row i set when node j is i or an ancestor */
+medusa_status_t medusa_tree_tables(const medusa_tree_t* tree, int32_t* tree_indices,
+                                   int32_t* parent, int32_t* depth, int32_t* retrieve,
+                                   uint64_t* anc);
+
+/* ------------------------------------------------------------------------ */
+/* S1-S3: heads and top-k                                                    */
+/* ------------------------------------------------------------------------ */
+
+size_t medusa_heads_workspace_size(int B, int d, int V, int K, int topk);
+
+/* u[b,k] = h[b] + SiLU(W1[k] h[b] + b1[k])   (fp32, kept unrounded)
+ * z[b,k] = Wout[k] u[b,k]                     (fp32 head logits)
+ * topk_ids/vals[b,k,:] = the topk largest z[b,k,:], value descending, lower
+ * token id first on equal values.
+ * dtype: element type of h, W1, b1, Wout (MEDUSA_F32 or MEDUSA_BF16); all
+ * arithmetic is fp32.  head_logits [B,K,V] fp32 may be NULL (not written).
+ * topk_ids [B,K,topk] int32, topk_vals [B,K,topk] fp32.
+ * Supported: d a multiple of 256 (bf16) / 128 (f32), d <= 8192 (bf16) /
+ * 4096 (f32), topk <= min(V, MEDUSA_MAX_TOPK), 1 <= B <= MEDUSA_MAX_B,
+ * 1 <= K <= MEDUSA_MAX_K.  Pointers must be 16-byte aligned. */
+medusa_status_t medusa_heads_topk(const void* h, const void* W1, const void* b1,
+                                  const void* Wout, int B, int d, int V, int K, int topk,
+                                  medusa_dtype_t dtype, float* head_logits, int32_t* topk_ids,
+                                  float* topk_vals, void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* S4: candidate assembly                                                    */
+/* ------------------------------------------------------------------------ */
+
+/* flat[b] = [root_tokens[b], topk_ids[b,0,:], ..., topk_ids[b,K-1,:]]
+ * tree_tokens[b,i]    = flat[b][tree_indices[i]]                [B, T]
+ * candidates[b,p,j]   = tree_tokens[b, retrieve[p,j]] or -1      [B, P, D+1]
+ * position_ids[b,i]   = seq_lens[b] + depth[i]                   [B, T]
+ * topk_ids must be [B, K_tree, topk_tree] for the tree's own K and topk. */
+medusa_status_t medusa_build_tree(const medusa_tree_t* tree, int B, const int32_t* root_tokens,
+                                  const int32_t* topk_ids, const int32_t* seq_lens,
+                                  int32_t* tree_tokens, int32_t* candidates,
+                                  int32_t* position_ids, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* S5: tree attention                                                        */
+/* ------------------------------------------------------------------------ */
+
+size_t medusa_attention_workspace_size(const medusa_tree_t* tree, int layers, int B, int H,
+                                       int hd, medusa_dtype_t dtype);
+
+/* For every layer l, sequence b, head e and tree node i (L = seq_lens[b]):
+ *   out[l,b,i,e] = sum_j softmax_j(scale * q[l,b,i,e] . k[l,b,e,j]) v[l,b,e,j]
+ * over j in {0..L-1} and {L+t : t is i or an ancestor of i}.
+ * q/out [layers,B,T,H,hd]; caches [layers,B,H,Lcap,hd]; dtype is that of q
+ * and the caches; out is always fp32 (fp32 softmax and accumulation).  Requires seq_lens[b]+T <= Lcap (a
+ * violation sets MEDUSA_ERR_DEVICE_CHECK and leaves that slice unwritten).
+ * Supported: hd <= 256 and a multiple of 32 (bf16 hd = 128 takes the
+ * tensor-core kernel).  Pointers 16-byte aligned. */
+medusa_status_t medusa_tree_attention(const medusa_tree_t* tree, int layers, int B, int H,
+                                      int hd, medusa_dtype_t dtype, const void* q,
+                                      const void* k_cache, const void* v_cache, int Lcap,
+                                      const int32_t* seq_lens, float scale, void* out,
+                                      void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* S6: posterior                                                             */
+/* ------------------------------------------------------------------------ */
+
+size_t medusa_posterior_workspace_size(const medusa_tree_t* tree, int B);
+
+/* Per node i of sequence b: g_i = argmax_v logits[b,i,v] (lowest id on ties);
+ * typical: p_i = softmax(logits[b,i,:] / temperature), H_i = -sum p ln p,
+ * thr_i = min(eps, alpha * exp(-H_i)).
+ * Path p accepts depth j when candidates[b,p,j] == g_parent (GREEDY) or
+ * p_parent(candidates[b,p,j]) > thr_parent (TYPICAL); acc_p counts leading
+ * accepted depths.  best_path[b] = lowest p with the largest acc_p;
+ * accept_len[b] = a = acc_best (0..D); accepted_tokens[b, 0..D] =
+ * candidates[b, best, 0..a], -1 after; next_token[b] = g at node
+ * retrieve[best, a].  TYPICAL needs temperature > 0 (defaults of the pages:
+ * eps = 0.09, alpha = 0.3).  logits [B,T,V] fp32; candidates [B,P,D+1]. */
+medusa_status_t medusa_evaluate_posterior(const medusa_tree_t* tree, int B, int V,
+                                          const float* logits, const int32_t* candidates,
+                                          medusa_mode_t mode, float temperature, float eps,
+                                          float alpha, int32_t* best_path, int32_t* accept_len,
+                                          int32_t* accepted_tokens, int32_t* next_token,
+                                          void* workspace, size_t workspace_bytes,
+                                          cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* S7: keep the accepted path's K/V                                          */
+/* ------------------------------------------------------------------------ */
+
+/* In place, for every layer, sequence b and head (L = seq_lens[b], a =
+ * accept_len[b], n_j = retrieve[best_path[b], j]):
+ *   cache row L+j  <-  cache row L+n_j,   j = 0..a   (K and V)
+ * read before any write (n_j can equal a destination of a later j), then
+ * seq_lens[b] = L + a + 1. */
+medusa_status_t medusa_accept_kv(const medusa_tree_t* tree, int layers, int B, int H, int hd,
+                                 medusa_dtype_t dtype, void* k_cache, void* v_cache, int Lcap,
+                                 int32_t* seq_lens, const int32_t* best_path,
+                                 const int32_t* accept_len, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* The whole step                                                            */
+/* ------------------------------------------------------------------------ */
+
+typedef struct medusa_step_args {
+  const medusa_tree_t* tree;
+  int B, d, V, K, topk;           /* heads */
+  int layers, H, hd, Lcap;        /* attention */
+  medusa_dtype_t dtype;
+  const void* h;
+  const void* W1;
+  const void* b1;
+  const void* Wout;
+  const int32_t* root_tokens;     /* [B] the base model's own next token */
+  const void* q;
+  void* k_cache;
+  void* v_cache;
+  int32_t* seq_lens;              /* [B], advanced by a+1 */
+  const float* base_logits;       /* [B, T, V] */
+  float scale;                    /* attention scale, usually 1/sqrt(hd) */
+  medusa_mode_t mode;
+  float temperature, eps, alpha;
+  float* head_logits;             /* nullable */
+  int32_t* topk_ids;
+  float* topk_vals;
+  int32_t* tree_tokens;
+  int32_t* candidates;
+  int32_t* position_ids;
+  void* attn_out;
+  int32_t* best_path;
+  int32_t* accept_len;
+  int32_t* accepted_tokens;
+  int32_t* next_token;
+} medusa_step_args_t;
+
+size_t medusa_step_workspace_size(const medusa_step_args_t* args);
+
+/* medusa_heads_topk, medusa_build_tree, medusa_tree_attention,
+ * medusa_evaluate_posterior and medusa_accept_kv, in that order, on stream.
+ * Capturable in a CUDA graph (no allocation, no synchronisation). */
+medusa_status_t medusa_step(const medusa_step_args_t* args, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MEDUSA_B200_H */

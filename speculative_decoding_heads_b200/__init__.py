@@ -1,0 +1,337 @@
+"""Python binding of libmedusa_b200 (one Medusa verification step on B200).
+
+Argument marshalling only: every function passes device pointers, sizes and
+the current CUDA stream to the C ABI declared in ``include/medusa_b200.h``;
+all computation happens in the library's sm_100a kernels.  There is no
+fallback: importing this package fails when the shared library is missing.
+
+Tensors are torch tensors on the CUDA device (torch is used for device
+memory and streams only).  Names follow the C ABI.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmedusa_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libmedusa_b200.so not found at {LIB_PATH}; build it with "
+        "`python -m speculative_decoding_heads_b200._build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+MEDUSA_OK = 0
+MEDUSA_ERR_INVALID_ARG = 1
+MEDUSA_ERR_UNSUPPORTED = 2
+MEDUSA_ERR_CUDA = 3
+MEDUSA_ERR_TIMEOUT = 4
+MEDUSA_ERR_DEVICE_CHECK = 5
+MEDUSA_F32 = 0
+MEDUSA_BF16 = 1
+MEDUSA_GREEDY = 0
+MEDUSA_TYPICAL = 1
+MAX_T, MAX_K, MAX_TOPK, MAX_B = 256, 16, 32, 64
+
+# Every symbol the header declares (checked by the CPU tests).
+EXPORTED = [
+    "medusa_last_error", "medusa_abi_version", "medusa_device_status",
+    "medusa_tree_choices_ranksum", "medusa_tree_create", "medusa_tree_destroy",
+    "medusa_tree_info", "medusa_tree_tables",
+    "medusa_heads_workspace_size", "medusa_heads_topk",
+    "medusa_build_tree",
+    "medusa_attention_workspace_size", "medusa_tree_attention",
+    "medusa_posterior_workspace_size", "medusa_evaluate_posterior",
+    "medusa_accept_kv",
+    "medusa_step_workspace_size", "medusa_step",
+]
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int
+_f32 = ctypes.c_float
+_sz = ctypes.c_size_t
+_pi32 = ctypes.POINTER(ctypes.c_int32)
+_pu64 = ctypes.POINTER(ctypes.c_uint64)
+
+
+class StepArgs(ctypes.Structure):
+    """Mirror of ``medusa_step_args_t``."""
+    _fields_ = [
+        ("tree", _vp),
+        ("B", _i32), ("d", _i32), ("V", _i32), ("K", _i32), ("topk", _i32),
+        ("layers", _i32), ("H", _i32), ("hd", _i32), ("Lcap", _i32),
+        ("dtype", _i32),
+        ("h", _vp), ("W1", _vp), ("b1", _vp), ("Wout", _vp),
+        ("root_tokens", _vp),
+        ("q", _vp), ("k_cache", _vp), ("v_cache", _vp),
+        ("seq_lens", _vp),
+        ("base_logits", _vp),
+        ("scale", _f32),
+        ("mode", _i32),
+        ("temperature", _f32), ("eps", _f32), ("alpha", _f32),
+        ("head_logits", _vp), ("topk_ids", _vp), ("topk_vals", _vp),
+        ("tree_tokens", _vp), ("candidates", _vp), ("position_ids", _vp),
+        ("attn_out", _vp),
+        ("best_path", _vp), ("accept_len", _vp), ("accepted_tokens", _vp), ("next_token", _vp),
+    ]
+
+
+def _sig(name, restype, argtypes):
+    fn = getattr(_lib, name)
+    fn.restype = restype
+    fn.argtypes = argtypes
+    return fn
+
+
+_sig("medusa_last_error", ctypes.c_char_p, [])
+_sig("medusa_abi_version", _i32, [])
+_sig("medusa_device_status", _i32, [_pi32, _pi32, _i32])
+_sig("medusa_tree_choices_ranksum", _i32, [_i32, _i32, _i32, _pi32, _pi32])
+_sig("medusa_tree_create", _i32, [_pi32, _pi32, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp)])
+_sig("medusa_tree_destroy", None, [_vp])
+_sig("medusa_tree_info", _i32, [_vp, _pi32, _pi32, _pi32])
+_sig("medusa_tree_tables", _i32, [_vp, _pi32, _pi32, _pi32, _pi32, _pu64])
+_sig("medusa_heads_workspace_size", _sz, [_i32] * 5)
+_sig("medusa_heads_topk", _i32, [_vp, _vp, _vp, _vp] + [_i32] * 5 + [_i32, _vp, _vp, _vp, _vp, _sz, _vp])
+_sig("medusa_build_tree", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp])
+_sig("medusa_attention_workspace_size", _sz, [_vp, _i32, _i32, _i32, _i32, _i32])
+_sig("medusa_tree_attention", _i32,
+     [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _f32, _vp, _vp, _sz, _vp])
+_sig("medusa_posterior_workspace_size", _sz, [_vp, _i32])
+_sig("medusa_evaluate_posterior", _i32,
+     [_vp, _i32, _i32, _vp, _vp, _i32, _f32, _f32, _f32, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
+_sig("medusa_accept_kv", _i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp])
+_sig("medusa_step_workspace_size", _sz, [ctypes.POINTER(StepArgs)])
+_sig("medusa_step", _i32, [ctypes.POINTER(StepArgs), _vp, _sz, _vp])
+
+
+class MedusaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+def _check(st: int):
+    if st != MEDUSA_OK:
+        raise MedusaError(st, (_lib.medusa_last_error() or b"").decode())
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MEDUSA_BF16
+    if t.dtype == torch.float32:
+        return MEDUSA_F32
+    raise MedusaError(MEDUSA_ERR_UNSUPPORTED, f"unsupported dtype {t.dtype}")
+
+
+def abi_version() -> int:
+    return _lib.medusa_abi_version()
+
+
+def device_status(clear: bool = True) -> Tuple[int, int]:
+    st, det = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(_lib.medusa_device_status(ctypes.byref(st), ctypes.byref(det), int(clear)))
+    return st.value, det.value
+
+
+# ---------------------------------------------------------------------------
+# tree
+# ---------------------------------------------------------------------------
+
+
+def _pack_choices(choices: Sequence[Sequence[int]], K: int):
+    n = len(choices)
+    ranks = (ctypes.c_int32 * max(1, n * K))()
+    lens = (ctypes.c_int32 * max(1, n))()
+    for i, c in enumerate(choices):
+        lens[i] = len(c)
+        for j, r in enumerate(c):
+            if j < K:
+                ranks[i * K + j] = int(r)
+    return ranks, lens
+
+
+def medusa_tree_choices_ranksum(K: int, topk: int, n_nodes: int) -> List[Tuple[int, ...]]:
+    ranks = (ctypes.c_int32 * max(1, n_nodes * K))()
+    lens = (ctypes.c_int32 * max(1, n_nodes))()
+    _check(_lib.medusa_tree_choices_ranksum(K, topk, n_nodes, ranks, lens))
+    return [tuple(ranks[i * K + j] for j in range(lens[i])) for i in range(n_nodes)]
+
+
+class Tree:
+    """A candidate tree (``medusa_tree_t``); ``upload=False`` keeps it host-only."""
+
+    def __init__(self, choices: Sequence[Sequence[int]], K: int, topk: int, upload: bool = True):
+        ranks, lens = _pack_choices(choices, K)
+        h = ctypes.c_void_p()
+        _check(_lib.medusa_tree_create(ranks, lens, len(choices), K, topk, int(upload), ctypes.byref(h)))
+        self._h = h
+        self.K, self.topk = K, topk
+        T, P, D = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        _check(_lib.medusa_tree_info(h, ctypes.byref(T), ctypes.byref(P), ctypes.byref(D)))
+        self.T, self.P, self.D = T.value, P.value, D.value
+        self.W = (self.T + 63) // 64
+
+    @property
+    def handle(self):
+        return self._h
+
+    def tables(self):
+        T, P, D, W = self.T, self.P, self.D, self.W
+        ti = (ctypes.c_int32 * T)()
+        par = (ctypes.c_int32 * T)()
+        dep = (ctypes.c_int32 * T)()
+        ret = (ctypes.c_int32 * (P * (D + 1)))()
+        anc = (ctypes.c_uint64 * (T * W))()
+        _check(_lib.medusa_tree_tables(self._h, ti, par, dep, ret, anc))
+        return dict(tree_indices=list(ti), parent=list(par), depth=list(dep),
+                    retrieve=[list(ret[p * (D + 1):(p + 1) * (D + 1)]) for p in range(P)],
+                    anc=[list(anc[i * W:(i + 1) * W]) for i in range(T)])
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.medusa_tree_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ---------------------------------------------------------------------------
+# step calls
+# ---------------------------------------------------------------------------
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zero-filled device workspace of at least ``nbytes`` (256-byte aligned)."""
+    return torch.zeros(max(256, int(nbytes)), dtype=torch.uint8, device=device or "cuda")
+
+
+def medusa_heads_workspace_size(B, d, V, K, topk) -> int:
+    return int(_lib.medusa_heads_workspace_size(B, d, V, K, topk))
+
+
+def medusa_heads_topk(h, W1, b1, Wout, topk, topk_ids, topk_vals, ws, head_logits=None, stream=None):
+    B, d = h.shape
+    K, V = Wout.shape[0], Wout.shape[1]
+    _check(_lib.medusa_heads_topk(_p(h), _p(W1), _p(b1), _p(Wout), B, d, V, K, topk, _dtype(h),
+                                  _p(head_logits), _p(topk_ids), _p(topk_vals), _p(ws),
+                                  ws.numel(), _stream(stream)))
+
+
+def medusa_build_tree(tree: Tree, root_tokens, topk_ids, seq_lens, tree_tokens, candidates,
+                      position_ids, stream=None):
+    _check(_lib.medusa_build_tree(tree.handle, root_tokens.shape[0], _p(root_tokens), _p(topk_ids),
+                                  _p(seq_lens), _p(tree_tokens), _p(candidates), _p(position_ids),
+                                  _stream(stream)))
+
+
+def medusa_attention_workspace_size(tree: Tree, layers, B, H, hd, dtype) -> int:
+    return int(_lib.medusa_attention_workspace_size(tree.handle, layers, B, H, hd, dtype))
+
+
+def medusa_tree_attention(tree: Tree, q, k_cache, v_cache, seq_lens, scale, out, ws=None, stream=None):
+    layers, B, T, H, hd = q.shape
+    Lcap = k_cache.shape[3]
+    _check(_lib.medusa_tree_attention(tree.handle, layers, B, H, hd, _dtype(q), _p(q), _p(k_cache),
+                                      _p(v_cache), Lcap, _p(seq_lens), float(scale), _p(out), _p(ws),
+                                      0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def medusa_posterior_workspace_size(tree: Tree, B) -> int:
+    return int(_lib.medusa_posterior_workspace_size(tree.handle, B))
+
+
+def medusa_evaluate_posterior(tree: Tree, logits, candidates, mode, best_path, accept_len,
+                              accepted_tokens, next_token, ws, temperature=0.0, eps=0.09,
+                              alpha=0.3, stream=None):
+    B, T, V = logits.shape
+    _check(_lib.medusa_evaluate_posterior(tree.handle, B, V, _p(logits), _p(candidates), int(mode),
+                                          float(temperature), float(eps), float(alpha),
+                                          _p(best_path), _p(accept_len), _p(accepted_tokens),
+                                          _p(next_token), _p(ws), ws.numel(), _stream(stream)))
+
+
+def medusa_accept_kv(tree: Tree, k_cache, v_cache, seq_lens, best_path, accept_len, stream=None):
+    layers, B, H, Lcap, hd = k_cache.shape
+    _check(_lib.medusa_accept_kv(tree.handle, layers, B, H, hd, _dtype(k_cache), _p(k_cache),
+                                 _p(v_cache), Lcap, _p(seq_lens), _p(best_path), _p(accept_len),
+                                 _stream(stream)))
+
+
+def make_step_args(tree: Tree, t: dict, mode: int, temperature=0.0, eps=0.09, alpha=0.3,
+                   scale=None) -> StepArgs:
+    """Builds ``medusa_step_args_t`` from a dict of device tensors (see ``StepBuffers``)."""
+    layers, B, T, H, hd = t["q"].shape
+    a = StepArgs()
+    a.tree = tree.handle
+    a.B, a.d = t["h"].shape
+    a.K, a.V = t["Wout"].shape[0], t["Wout"].shape[1]
+    a.topk = tree.topk
+    a.layers, a.H, a.hd, a.Lcap = layers, H, hd, t["k_cache"].shape[3]
+    a.dtype = _dtype(t["h"])
+    for name in ("h", "W1", "b1", "Wout", "root_tokens", "q", "k_cache", "v_cache", "seq_lens",
+                 "base_logits", "topk_ids", "topk_vals", "tree_tokens", "candidates",
+                 "position_ids", "attn_out", "best_path", "accept_len", "accepted_tokens",
+                 "next_token"):
+        setattr(a, name, t[name].data_ptr())
+    a.head_logits = t["head_logits"].data_ptr() if t.get("head_logits") is not None else None
+    a.scale = float(scale if scale is not None else hd ** -0.5)
+    a.mode = int(mode)
+    a.temperature, a.eps, a.alpha = float(temperature), float(eps), float(alpha)
+    return a
+
+
+def medusa_step_workspace_size(args: StepArgs) -> int:
+    return int(_lib.medusa_step_workspace_size(ctypes.byref(args)))
+
+
+def medusa_step(args: StepArgs, ws, stream=None):
+    _check(_lib.medusa_step(ctypes.byref(args), _p(ws), ws.numel(), _stream(stream)))
+
+
+def medusa_step_from_host(args: StepArgs, ws, host_in: dict, dev: dict, host_out: dict, stream=None):
+    """One step through the public API with host buffers.
+
+    Copies every per-step input from pinned host memory (``host_in``: name ->
+    pinned tensor, copied into ``dev[name]``; the tree's own K/V rows are
+    given as ``k_tree``/``v_tree`` [layers, B, H, T, hd] and scattered into
+    the caches at each sequence's current length), runs ``medusa_step`` and
+    reads the results back into the pinned ``host_out`` tensors.  All copies
+    are enqueued on ``stream``; the caller synchronises.
+    """
+    s = stream or torch.cuda.current_stream()
+    with torch.cuda.stream(s):
+        for name, src in host_in.items():
+            if name in ("k_tree", "v_tree"):
+                continue
+            dev[name].copy_(src, non_blocking=True)
+        if "k_tree" in host_in:
+            lens = host_in["seq_lens"]
+            T = host_in["k_tree"].shape[3]
+            for b in range(lens.shape[0]):
+                L = int(lens[b])
+                dev["k_cache"][:, b, :, L:L + T, :].copy_(host_in["k_tree"][:, b], non_blocking=True)
+                dev["v_cache"][:, b, :, L:L + T, :].copy_(host_in["v_tree"][:, b], non_blocking=True)
+        medusa_step(args, ws, s)
+        for name, dst in host_out.items():
+            dst.copy_(dev[name], non_blocking=True)

@@ -1,0 +1,685 @@
+// S1-S3: the Medusa heads and their per-head top-k, as one persistent,
+// HBM-streaming kernel.
+//
+// Each head k is one residual block followed by its own vocabulary
+// projection ("Medusa API参考：核心函数与类详解", MedusaModelABC: medusa_head is
+// residual blocks plus a linear layer; "Medusa — 让大模型自己同时猜好几个 token",
+// 是什么: a one-layer MLP with a residual on the last hidden state):
+//     u[b,k] = h[b] + SiLU(W1[k] h[b] + b1[k])        (fp32, never rounded)
+//     z[b,k] = Wout[k] u[b,k]                         (fp32 head logits)
+// and each head's top-k tokens become the candidates of tree depth k
+// (核心要点: the heads' top-k assembled into a prefix tree).
+//
+// Design (batch 1..4 per launch, weights read exactly once per launch):
+//  * One CTA per SM, launched cooperatively so all CTAs are resident.  The
+//    W1 rows (K*d) and then the Wout rows (K*V) are split evenly over the
+//    CTAs; every CTA streams its rows through a ring of shared-memory stages
+//    filled by 1-D TMA bulk copies (cp.async.bulk + mbarrier complete_tx),
+//    with an L2 evict-first hint because every weight byte is read once.
+//  * Thread t owns the 16-byte column vectors t, t+NT, ... of every row and
+//    keeps the matching slice of h (phase 1) or u (phase 2) in registers, so
+//    shared memory only carries the weights.  A stage of R rows gives R*NB
+//    partial dot products per thread, reduced by warp shuffles and then
+//    across warps through a small double-buffered shared array.
+//  * Phase 1 writes u to the workspace and, once all of a CTA's W1 rows are
+//    done, bumps a release counter.  Phase 2 issues its first Wout copies
+//    before it waits (acquire, bounded) for every CTA's phase 1, so the
+//    weight stream never stops at the S1 -> S2 boundary.
+//  * Warp 0 keeps a running top-k per (sequence, head) in shared memory; a
+//    new logit is inserted only when it beats the current k-th entry.  At the
+//    end each CTA publishes its lists, and the last CTA to finish merges
+//    them (k rounds of a warp arg-max over the published candidates) and
+//    resets the counters for the next call.
+#include <cfloat>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace medusa {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kMaxNB = 4;             // sequences per launch
+constexpr int kStageTarget = 200 * 1024;
+constexpr int kMaxStages = 8;
+
+struct HeadsArgs {
+  const void* h;
+  const void* W1;
+  const void* b1;
+  const void* Wout;
+  int B, d, V, K, topk;
+  int b0, nb;             // sequences [b0, b0+nb) in this launch
+  float* head_logits;     // nullable [B, K, V]
+  int32_t* topk_ids;      // [B, K, topk]
+  float* topk_vals;
+  float* u;               // workspace [B, K, d]
+  float* cand_vals;       // workspace [kMaxNB, K, G, topk]
+  int32_t* cand_ids;
+  unsigned* counters;     // workspace: [0] CTAs done with phase 1, [1] with phase 2
+  int* status;
+  int G;
+  int NS;                 // stages in the ring
+  int nvec;               // 16-byte vectors per row
+};
+
+template <typename TW>
+struct Elem;
+template <>
+struct Elem<float> {
+  static constexpr int E = 4;
+};
+template <>
+struct Elem<uint16_t> {
+  static constexpr int E = 8;
+};
+
+// First row of CTA c when n rows are split evenly over G CTAs.
+__device__ __forceinline__ int part_lo(int n, int c, int G) {
+  return static_cast<int>(static_cast<long long>(n) * c / G);
+}
+
+// The stages of one CTA: its phase-1 rows, then its phase-2 rows, at most R
+// rows each and never across a head boundary.  All 32-bit and incremental:
+// the only divisions happen when the cursor enters a phase.
+struct Cursor {
+  int phase;      // 1, 2, or 3 (done)
+  int row, n;     // stage rows [row, row + n) of the phase's matrix
+  int end;        // end of this CTA's rows in the current phase
+  int head;       // head of `row`
+  int head_end;   // first row of the next head
+  int p2_lo, p2_hi;
+};
+
+template <int R>
+__device__ __forceinline__ void cursor_fix(Cursor& c, const HeadsArgs& a) {
+  if (c.phase == 1 && c.row >= c.end) {
+    c.phase = 2;
+    c.row = c.p2_lo;
+    c.end = c.p2_hi;
+    c.head = c.row / a.V;
+    c.head_end = (c.head + 1) * a.V;
+  }
+  if (c.phase == 2 && c.row >= c.end) {
+    c.phase = 3;
+    c.n = 0;
+    return;
+  }
+  const int lim = c.end < c.head_end ? c.end : c.head_end;
+  c.n = lim - c.row < R ? lim - c.row : R;
+}
+
+template <int R>
+__device__ __forceinline__ void cursor_start(Cursor& c, const HeadsArgs& a, int p1_lo, int p1_hi, int p2_lo,
+                                             int p2_hi) {
+  c.phase = 1;
+  c.row = p1_lo;
+  c.end = p1_hi;
+  c.head = p1_lo / a.d;
+  c.head_end = (c.head + 1) * a.d;
+  c.p2_lo = p2_lo;
+  c.p2_hi = p2_hi;
+  cursor_fix<R>(c, a);
+}
+
+template <int R>
+__device__ __forceinline__ void cursor_next(Cursor& c, const HeadsArgs& a) {
+  c.row += c.n;
+  if (c.row >= c.head_end) {
+    ++c.head;
+    c.head_end += (c.phase == 1) ? a.d : a.V;
+  }
+  cursor_fix<R>(c, a);
+}
+
+template <typename TW>
+__device__ __forceinline__ const char* stage_src(const HeadsArgs& a, const Cursor& c) {
+  const size_t row_bytes = static_cast<size_t>(a.d) * sizeof(TW);
+  const char* base = static_cast<const char*>(c.phase == 1 ? a.W1 : a.Wout);
+  return base + static_cast<size_t>(c.row) * row_bytes;
+}
+
+// Loads the E elements of vector `v` of row vector x (element type TX) as fp32.
+template <typename TX>
+__device__ __forceinline__ void load_vec(const TX* x, int v, float* out);
+template <>
+__device__ __forceinline__ void load_vec<float>(const float* x, int v, float* out) {
+  const float4 a = __ldcg(reinterpret_cast<const float4*>(x) + v);
+  out[0] = a.x;
+  out[1] = a.y;
+  out[2] = a.z;
+  out[3] = a.w;
+}
+template <>
+__device__ __forceinline__ void load_vec<uint16_t>(const uint16_t* x, int v, float* out) {
+  const uint4 a = __ldcg(reinterpret_cast<const uint4*>(x) + v);
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    out[2 * i] = bf16lo(w[i]);
+    out[2 * i + 1] = bf16hi(w[i]);
+  }
+}
+
+// fp32 u (phase 2) for a bf16 model: 8 floats per 16-byte weight vector.
+__device__ __forceinline__ void load_u_vec(const float* u, int v, int E, float* out) {
+  const float4* p = reinterpret_cast<const float4*>(u) + static_cast<size_t>(v) * (E / 4);
+  for (int i = 0; i < E / 4; ++i) {
+    const float4 a = __ldcg(p + i);
+    out[4 * i] = a.x;
+    out[4 * i + 1] = a.y;
+    out[4 * i + 2] = a.z;
+    out[4 * i + 3] = a.w;
+  }
+}
+
+template <typename TW>
+__device__ __forceinline__ float to_f32(TW x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<uint16_t>(uint16_t x) {
+  return __uint_as_float(static_cast<uint32_t>(x) << 16);
+}
+
+// acc[b] += dot(16-byte weight vector w, x[b][0..E)) for b < NB.
+template <typename TW, int NB, int VPT>
+__device__ __forceinline__ void dot_vec(const uint4 w, const float (&x)[NB * VPT][Elem<TW>::E], int j,
+                                        float* acc) {
+  constexpr int E = Elem<TW>::E;
+  float f[E];
+  if constexpr (E == 8) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = bf16lo(ww[i]);
+      f[2 * i + 1] = bf16hi(ww[i]);
+    }
+  } else {
+    f[0] = __uint_as_float(w.x);
+    f[1] = __uint_as_float(w.y);
+    f[2] = __uint_as_float(w.z);
+    f[3] = __uint_as_float(w.w);
+  }
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[b] = fmaf(f[e], x[b * VPT + j][e], acc[b]);
+}
+
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
+
+// CTA of row r when n rows are split evenly over G CTAs (inverse of part_lo).
+__device__ __forceinline__ int part_of(int r, int n, int G) {
+  return static_cast<int>((static_cast<long long>(r + 1) * G - 1) / n);
+}
+
+// Sums C values over the 32 lanes of a warp by repeated halving: at each
+// step a lane keeps half of its values and trades the other half with its
+// partner, so C values need C-1 + log2(32/C) shuffles instead of 5*C.  On
+// return v[0] holds the full sum of value `idx`; lanes whose low
+// log2(32/C) bits are zero hold each value exactly once.
+template <int C, int O>
+struct WarpFold {
+  static __device__ __forceinline__ void run(float* v, int lane, int& idx) {
+    if constexpr (O == 0) {
+      return;
+    } else if constexpr (C > 1) {
+      const bool up = (lane & O) != 0;
+#pragma unroll
+      for (int i = 0; i < C / 2; ++i) {
+        const float send = up ? v[i] : v[i + C / 2];
+        const float keep = up ? v[i + C / 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+      }
+      if (up) idx += C / 2;
+      WarpFold<C / 2, O / 2>::run(v, lane, idx);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+      WarpFold<1, O / 2>::run(v, lane, idx);
+    }
+  }
+};
+
+// Warp 0: insert (v, id) into the sorted list (lv, lid, *cnt) of capacity topk.
+__device__ __forceinline__ void list_insert(float* lv, int* lid, int* cnt_p, int topk, float v, int id,
+                                            int lane) {
+  const int cnt = *cnt_p;
+  float ev = -FLT_MAX;
+  int ei = -1;
+  if (lane < cnt) {
+    ev = lv[lane];
+    ei = lid[lane];
+  }
+  const bool before = lane < cnt && ranks_before(ev, ei, v, id);
+  const int pos = __popc(__ballot_sync(0xffffffffu, before));
+  const float pv = __shfl_up_sync(0xffffffffu, ev, 1);
+  const int pi = __shfl_up_sync(0xffffffffu, ei, 1);
+  __syncwarp();
+  if (pos < topk && lane < topk && lane >= pos && lane <= cnt) {
+    lv[lane] = (lane == pos) ? v : pv;
+    lid[lane] = (lane == pos) ? id : pi;
+  }
+  __syncwarp();
+  if (lane == 0 && pos < topk && cnt < topk) *cnt_p = cnt + 1;
+  __syncwarp();
+}
+
+constexpr int kMergeRegs = 16;   // candidates per lane held in registers by the merge
+
+template <typename TW, int NB, int VPT, int R>
+__global__ void __launch_bounds__(kThreads, 1) heads_kernel(const HeadsArgs a) {
+  constexpr int E = Elem<TW>::E;
+  constexpr int RNB = R * NB;
+  static_assert(RNB <= 32 && (32 % RNB) == 0, "stage epilogue uses one lane per (row, sequence)");
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int NW = blockDim.x >> 5;
+  const int cta = blockIdx.x;
+  const int G = a.G;
+  const size_t row_bytes = static_cast<size_t>(a.d) * sizeof(TW);
+  const size_t stage_bytes = row_bytes * R;
+
+  // shared-memory carve-up
+  unsigned char* stages = smem;
+  float* partial = reinterpret_cast<float*>(smem + stage_bytes * a.NS);   // [2][NW][RNB]
+  float* list_v = partial + 2 * NW * RNB;                                  // [NB][K][topk]
+  int* list_i = reinterpret_cast<int*>(list_v + NB * a.K * a.topk);
+  int* list_n = list_i + NB * a.K * a.topk;                                // [NB][K]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(list_n + NB * a.K) + 15) & ~uintptr_t(15));  // [NS]
+  int* flag = reinterpret_cast<int*>(bars + a.NS);
+
+  const int n1 = a.K * a.d;
+  const int n2 = a.K * a.V;
+  const int p1_lo = part_lo(n1, cta, G), p1_hi = part_lo(n1, cta + 1, G);
+  const int p2_lo = part_lo(n2, cta, G), p2_hi = part_lo(n2, cta + 1, G);
+
+  for (int i = tid; i < NB * a.K * a.topk; i += blockDim.x) {
+    list_v[i] = -FLT_MAX;
+    list_i[i] = -1;
+  }
+  for (int i = tid; i < NB * a.K; i += blockDim.x) list_n[i] = 0;
+  if (tid == 0) {
+    for (int s = 0; s < a.NS; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+    flag[0] = 0;
+  }
+  __syncthreads();
+
+  const uint64_t policy = l2_evict_first_policy();
+  // Producer cursor (thread 0 only): the first NS stages go out now.
+  Cursor pc;
+  cursor_start<R>(pc, a, p1_lo, p1_hi, p2_lo, p2_hi);
+  int issued = 0;
+  if (tid == 0) {
+    for (; issued < a.NS && pc.phase != 3; ++issued) {
+      const uint32_t bytes = static_cast<uint32_t>(pc.n * row_bytes);
+      mbar_arrive_expect_tx(&bars[issued], bytes);
+      tma_load_1d(stages + issued * stage_bytes, stage_src<TW>(a, pc), bytes, &bars[issued], policy);
+      cursor_next<R>(pc, a);
+    }
+  }
+
+  // x[b*VPT+j][e]: h (phase 1) or u of the current head (phase 2), for the
+  // thread's column vectors tid + j*NT.
+  float x[NB * VPT][E];
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * blockDim.x;
+      if (b < a.nb && v < a.nvec) {
+        load_vec<TW>(static_cast<const TW*>(a.h) + static_cast<size_t>(a.b0 + b) * a.d, v, x[b * VPT + j]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[b * VPT + j][e] = 0.f;
+      }
+    }
+
+  Cursor cc;
+  cursor_start<R>(cc, a, p1_lo, p1_hi, p2_lo, p2_hi);
+  int cur_head2 = -1;   // head whose u sits in x during phase 2
+  bool published = false;
+  bool aborted = false;
+  int s = 0;
+  for (; cc.phase != 3; ++s) {
+    const int slot = s % a.NS;
+    if (cc.phase == 2 && !published) {
+      // First phase-2 stage: publish this CTA's phase 1, then wait (bounded)
+      // until every CTA has published.  The Wout copies are already in flight.
+      published = true;
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();
+        atom_add_release_gpu(&a.counters[0], 1u);
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(&a.counters[0]) < static_cast<unsigned>(G)) {
+          if (globaltimer_ns() - t0 > kSpinLimitNs) {
+            set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsS1Wait);
+            flag[0] = 1;
+            break;
+          }
+          __nanosleep(64);
+        }
+      }
+      __syncthreads();
+      if (flag[0]) {
+        aborted = true;
+        break;
+      }
+    }
+    const int khead = cc.head;   // uniform per stage
+    if (cc.phase == 2 && khead != cur_head2) {
+      cur_head2 = khead;
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+          const int v = tid + j * blockDim.x;
+          if (b < a.nb && v < a.nvec)
+            load_u_vec(a.u + (static_cast<size_t>(a.b0 + b) * a.K + khead) * a.d, v, E, x[b * VPT + j]);
+        }
+    }
+
+    if (!mbar_wait(&bars[slot], static_cast<uint32_t>((s / a.NS) & 1))) {
+      set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsStageWait);
+      aborted = true;
+      break;
+    }
+
+    float acc[RNB];
+#pragma unroll
+    for (int i = 0; i < RNB; ++i) acc[i] = 0.f;
+    const unsigned char* st = stages + slot * stage_bytes;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (r < cc.n) {
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+          const int v = tid + j * blockDim.x;
+          if (v < a.nvec) {
+            const uint4 w = *reinterpret_cast<const uint4*>(st + r * row_bytes + static_cast<size_t>(v) * 16);
+            dot_vec<TW, NB, VPT>(w, x, j, acc + r * NB);
+          }
+        }
+      }
+    }
+    int idx = 0;
+    WarpFold<RNB, 16>::run(acc, lane, idx);
+    float* pbuf = partial + (s & 1) * NW * RNB;
+    if ((lane & (32 / RNB - 1)) == 0) pbuf[warp * RNB + idx] = acc[0];
+    __syncthreads();   // the stage slot is free and the partials are complete
+
+    if (tid == 0 && pc.phase != 3) {
+      const uint32_t bytes = static_cast<uint32_t>(pc.n * row_bytes);
+      mbar_arrive_expect_tx(&bars[slot], bytes);
+      tma_load_1d(stages + slot * stage_bytes, stage_src<TW>(a, pc), bytes, &bars[slot], policy);
+      cursor_next<R>(pc, a);
+      ++issued;
+    }
+
+    if (warp == 0) {
+      // Cross-warp sum: lane l adds entries l, l+32, ... (all of value l % RNB),
+      // then lanes with equal l % RNB combine.
+      float val = 0.f;
+      for (int e = lane; e < NW * RNB; e += 32) val += pbuf[e];
+#pragma unroll
+      for (int o = RNB; o < 32; o <<= 1) val += __shfl_xor_sync(0xffffffffu, val, o);
+      // Stage epilogue: lane t < RNB owns row t / NB and sequence t % NB.
+      const int r = lane / NB, b = lane % NB;
+      const bool live = lane < RNB && r < cc.n && b < a.nb;
+      const int local = cc.row - khead * (cc.phase == 1 ? a.d : a.V) + r;   // row within the head
+      if (cc.phase == 1) {
+        if (live) {
+          const float hb = to_f32<TW>(static_cast<const TW*>(a.h)[static_cast<size_t>(a.b0 + b) * a.d + local]);
+          const float bb = to_f32<TW>(static_cast<const TW*>(a.b1)[static_cast<size_t>(khead) * a.d + local]);
+          a.u[(static_cast<size_t>(a.b0 + b) * a.K + khead) * a.d + local] = hb + silu(val + bb);
+          __threadfence();
+        }
+      } else {
+        if (live && a.head_logits)
+          a.head_logits[(static_cast<size_t>(a.b0 + b) * a.K + khead) * a.V + local] = val;
+        bool cand = false;
+        if (live) {
+          const int li = b * a.K + khead;
+          cand = list_n[li] < a.topk ||
+                 ranks_before(val, local, list_v[li * a.topk + a.topk - 1], list_i[li * a.topk + a.topk - 1]);
+        }
+        unsigned m = __ballot_sync(0xffffffffu, cand);
+        while (m) {
+          const int src = __ffs(m) - 1;
+          m &= m - 1;
+          const float nv = __shfl_sync(0xffffffffu, val, src);
+          const int nid = __shfl_sync(0xffffffffu, local, src);
+          const int li = (src % NB) * a.K + khead;
+          list_insert(list_v + li * a.topk, list_i + li * a.topk, list_n + li, a.topk, nv, nid, lane);
+        }
+      }
+    }
+    cursor_next<R>(cc, a);
+  }
+
+  if (aborted) {
+    // Drain the copies this CTA issued so that none lands after it exits.
+    if (tid == 0)
+      for (int t = s; t < issued; ++t) mbar_wait(&bars[t % a.NS], static_cast<uint32_t>((t / a.NS) & 1));
+    __syncthreads();
+    return;
+  }
+  __syncthreads();
+  if (!published && tid == 0) {
+    // No phase-2 rows here: still count this CTA's phase 1.
+    __threadfence();
+    atom_add_release_gpu(&a.counters[0], 1u);
+  }
+
+  // Publish the local lists of every head this CTA's phase-2 rows touched.
+  if (p2_hi > p2_lo) {
+    const int k_lo = p2_lo / a.V;
+    const int k_hi = (p2_hi - 1) / a.V;
+    for (int k = k_lo; k <= k_hi; ++k)
+      for (int i = tid; i < NB * a.topk; i += blockDim.x) {
+        const int b = i / a.topk, j = i % a.topk;
+        const int li = b * a.K + k;
+        const size_t o = ((static_cast<size_t>(b) * a.K + k) * G + cta) * a.topk + j;
+        a.cand_vals[o] = list_v[li * a.topk + j];
+        a.cand_ids[o] = list_i[li * a.topk + j];
+      }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned done = atom_add_acq_rel_gpu(&a.counters[1], 1u);
+    flag[0] = (done == static_cast<unsigned>(G - 1)) ? 2 : 0;
+  }
+  __syncthreads();
+  if (flag[0] != 2) return;
+
+  // Last CTA: merge the published lists of every (sequence, head).  The
+  // candidates of one list are loaded once; each of the topk rounds picks
+  // the best candidate that ranks strictly after the previous pick.
+  __threadfence();
+  for (int li = warp; li < a.nb * a.K; li += NW) {
+    const int b = li / a.K, k = li % a.K;
+    const int hk_lo = k * a.V;
+    const int c_lo = part_of(hk_lo, n2, G);
+    const int c_hi = part_of(hk_lo + a.V - 1, n2, G);
+    const int ncand = (c_hi - c_lo + 1) * a.topk;
+    const size_t base = ((static_cast<size_t>(b) * a.K + k) * G + c_lo) * a.topk;
+    float cv[kMergeRegs];
+    int ci[kMergeRegs];
+#pragma unroll
+    for (int m = 0; m < kMergeRegs; ++m) {
+      const int i = lane + 32 * m;
+      cv[m] = -FLT_MAX;
+      ci[m] = -1;
+      if (i < ncand) {
+        cv[m] = __ldcg(a.cand_vals + base + i);
+        ci[m] = __ldcg(a.cand_ids + base + i);
+      }
+    }
+    float prev_v = FLT_MAX;
+    int prev_i = -1;
+    for (int r = 0; r < a.topk; ++r) {
+      float bv = -FLT_MAX;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int m = 0; m < kMergeRegs; ++m)
+        if (ci[m] >= 0 && ranks_before(prev_v, prev_i, cv[m], ci[m]) && ranks_before(cv[m], ci[m], bv, bi)) {
+          bv = cv[m];
+          bi = ci[m];
+        }
+      for (int i = lane + 32 * kMergeRegs; i < ncand; i += 32) {   // large lists only
+        const float v = __ldcg(a.cand_vals + base + i);
+        const int id = __ldcg(a.cand_ids + base + i);
+        if (id >= 0 && ranks_before(prev_v, prev_i, v, id) && ranks_before(v, id, bv, bi)) {
+          bv = v;
+          bi = id;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ranks_before(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (lane == 0) {
+        const size_t o = (static_cast<size_t>(a.b0 + b) * a.K + k) * a.topk + r;
+        a.topk_ids[o] = bi;
+        a.topk_vals[o] = bv;
+      }
+      prev_v = bv;
+      prev_i = bi;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    a.counters[0] = 0u;
+    a.counters[1] = 0u;
+    __threadfence();
+  }
+}
+
+struct Plan {
+  int NT, VPT, NS, R;
+  size_t smem;
+};
+
+// Rows per stage: 8 when the batch group is at most 2 and 8 rows fit in
+// 64 KB, else 4.  Stages: as many as fit in ~200 KB (at least 2, at most 8).
+template <typename TW>
+Plan make_plan(int d, int nb, int K, int topk) {
+  constexpr int E = Elem<TW>::E;
+  Plan p{};
+  const int nvec = d / E;
+  p.NT = nvec >= kThreads ? kThreads : ((nvec + 31) / 32) * 32;
+  p.VPT = (nvec + p.NT - 1) / p.NT;
+  const size_t row = static_cast<size_t>(d) * sizeof(TW);
+  p.R = (nb <= 2 && row * 8 <= 64 * 1024) ? 8 : 4;
+  const size_t stage = row * p.R;
+  const int ns = static_cast<int>(kStageTarget / stage);
+  p.NS = ns < 2 ? 2 : (ns > kMaxStages ? kMaxStages : ns);
+  const int NW = p.NT / 32;
+  p.smem = stage * p.NS + 2 * NW * 32 * sizeof(float) + kMaxNB * K * topk * (sizeof(float) + sizeof(int)) +
+           kMaxNB * K * sizeof(int) + 16 + p.NS * sizeof(uint64_t) + 64;
+  return p;
+}
+
+template <typename TW, int NB, int VPT, int R>
+cudaError_t launch_one(const HeadsArgs& a, const Plan& p, cudaStream_t stream) {
+  auto fn = heads_kernel<TW, NB, VPT, R>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(p.smem));
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, p.NT, p.smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  void* args[] = {const_cast<HeadsArgs*>(&a)};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(fn), dim3(a.G), dim3(p.NT), args,
+                                     p.smem, stream);
+}
+
+template <typename TW, int NB, int VPT>
+cudaError_t dispatch_r(const HeadsArgs& a, const Plan& p, cudaStream_t stream) {
+  if constexpr (NB <= 2) {
+    if (p.R == 8) return launch_one<TW, NB, VPT, 8>(a, p, stream);
+  }
+  return launch_one<TW, NB, VPT, 4>(a, p, stream);
+}
+
+template <typename TW, int NB>
+cudaError_t dispatch_vpt(const HeadsArgs& a, const Plan& p, cudaStream_t stream) {
+  if (p.VPT == 1) return dispatch_r<TW, NB, 1>(a, p, stream);
+  return dispatch_r<TW, NB, 2>(a, p, stream);
+}
+
+template <typename TW>
+cudaError_t dispatch_nb(const HeadsArgs& a, const Plan& p, cudaStream_t stream) {
+  if (a.nb == 1) return dispatch_vpt<TW, 1>(a, p, stream);
+  if (a.nb == 2) return dispatch_vpt<TW, 2>(a, p, stream);
+  return dispatch_vpt<TW, 4>(a, p, stream);
+}
+
+}  // namespace
+
+size_t heads_workspace_bytes(int B, int d, int V, int K, int topk) {
+  (void)V;
+  const int G = sm_count();
+  size_t off = align_up(static_cast<size_t>(B) * K * d * sizeof(float), 256);
+  off += align_up(static_cast<size_t>(kMaxNB) * K * G * topk * sizeof(float), 256);
+  off += align_up(static_cast<size_t>(kMaxNB) * K * G * topk * sizeof(int32_t), 256);
+  off += 256;  // counters
+  return off;
+}
+
+medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, const void* Wout,
+                             int B, int d, int V, int K, int topk, medusa_dtype_t dtype,
+                             float* head_logits, int32_t* topk_ids, float* topk_vals, void* ws,
+                             cudaStream_t stream) {
+  const int G = sm_count();
+  HeadsArgs a{};
+  a.h = h;
+  a.W1 = W1;
+  a.b1 = b1;
+  a.Wout = Wout;
+  a.B = B;
+  a.d = d;
+  a.V = V;
+  a.K = K;
+  a.topk = topk;
+  a.head_logits = head_logits;
+  a.topk_ids = topk_ids;
+  a.topk_vals = topk_vals;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  size_t off = 0;
+  a.u = reinterpret_cast<float*>(w + off);
+  off += align_up(static_cast<size_t>(B) * K * d * sizeof(float), 256);
+  a.cand_vals = reinterpret_cast<float*>(w + off);
+  off += align_up(static_cast<size_t>(kMaxNB) * K * G * topk * sizeof(float), 256);
+  a.cand_ids = reinterpret_cast<int32_t*>(w + off);
+  off += align_up(static_cast<size_t>(kMaxNB) * K * G * topk * sizeof(int32_t), 256);
+  a.counters = reinterpret_cast<unsigned*>(w + off);
+  a.status = device_status_ptr();
+  a.G = G;
+  a.nvec = (dtype == MEDUSA_BF16) ? d / 8 : d / 4;
+  for (int b0 = 0; b0 < B; b0 += kMaxNB) {
+    a.b0 = b0;
+    a.nb = (B - b0) < kMaxNB ? (B - b0) : kMaxNB;
+    const int nbt = a.nb == 1 ? 1 : (a.nb == 2 ? 2 : 4);
+    const Plan p = (dtype == MEDUSA_BF16) ? make_plan<uint16_t>(d, nbt, K, topk) : make_plan<float>(d, nbt, K, topk);
+    a.NS = p.NS;
+    cudaError_t e = (dtype == MEDUSA_BF16) ? dispatch_nb<uint16_t>(a, p, stream) : dispatch_nb<float>(a, p, stream);
+    if (e != cudaSuccess) return cuda_fail("medusa_heads_topk: launch", e);
+  }
+  return MEDUSA_OK;
+}
+
+}  // namespace medusa

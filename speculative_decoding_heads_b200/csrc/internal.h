@@ -1,0 +1,79 @@
+// Internal declarations shared by the host-side sources of libmedusa_b200.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "medusa_b200.h"
+
+namespace medusa {
+
+// Device-side view of a tree, passed to kernels by value.
+struct TreeDev {
+  int T, P, D, K, topk, W;        // W = 64-bit words per ancestor-mask row
+  const int32_t* tree_indices;    // [T]
+  const int32_t* parent;          // [T]
+  const int32_t* depth;           // [T]
+  const int32_t* retrieve;        // [P * (D+1)]
+  const uint64_t* anc;            // [T * W]
+};
+
+}  // namespace medusa
+
+struct medusa_tree {
+  int T = 0, P = 0, D = 0, K = 0, topk = 0, W = 0;
+  int device = -1;                // device holding the uploaded tables, -1 if none
+  std::vector<std::vector<int32_t>> nodes;   // rank tuple of every node, nodes[0] empty
+  std::vector<int32_t> tree_indices, parent, depth, retrieve;
+  std::vector<uint64_t> anc;
+  void* dev_block = nullptr;      // one device allocation holding every table
+  medusa::TreeDev dev{};
+};
+
+namespace medusa {
+
+// Thread-local error text; returns the status for convenient `return fail(...)`.
+medusa_status_t fail(medusa_status_t st, const std::string& msg);
+medusa_status_t cuda_fail(const char* what, int err);
+
+// Status word on the current device (set by kernels, read by medusa_device_status).
+medusa_status_t device_status_read(int32_t* status, int32_t* detail, int clear);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Kernel launchers (heads.cu, tree_kernels.cu, attention.cu, posterior.cu, accept.cu).
+size_t heads_workspace_bytes(int B, int d, int V, int K, int topk);
+medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, const void* Wout,
+                             int B, int d, int V, int K, int topk, medusa_dtype_t dtype,
+                             float* head_logits, int32_t* topk_ids, float* topk_vals, void* ws,
+                             cudaStream_t stream);
+
+medusa_status_t launch_build_tree(const TreeDev& t, int B, const int32_t* root_tokens,
+                                  const int32_t* topk_ids, const int32_t* seq_lens,
+                                  int32_t* tree_tokens, int32_t* candidates,
+                                  int32_t* position_ids, cudaStream_t stream);
+
+size_t attention_workspace_bytes(const TreeDev& t, int layers, int B, int H, int hd,
+                                 medusa_dtype_t dtype);
+medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int hd,
+                                 medusa_dtype_t dtype, const void* q, const void* k_cache,
+                                 const void* v_cache, int Lcap, const int32_t* seq_lens,
+                                 float scale, void* out, void* ws, cudaStream_t stream);
+
+size_t posterior_workspace_bytes(const TreeDev& t, int B);
+medusa_status_t launch_posterior(const TreeDev& t, int B, int V, const float* logits,
+                                 const int32_t* candidates, medusa_mode_t mode, float temperature,
+                                 float eps, float alpha, int32_t* best_path, int32_t* accept_len,
+                                 int32_t* accepted_tokens, int32_t* next_token, void* ws,
+                                 cudaStream_t stream);
+
+medusa_status_t launch_accept_kv(const TreeDev& t, int layers, int B, int H, int hd,
+                                 medusa_dtype_t dtype, void* k_cache, void* v_cache, int Lcap,
+                                 int32_t* seq_lens, const int32_t* best_path,
+                                 const int32_t* accept_len, cudaStream_t stream);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace medusa
