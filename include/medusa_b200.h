@@ -159,6 +159,28 @@ medusa_status_t medusa_heads_topk(const void* h, const void* W1, const void* b1,
                                   float* topk_vals, void* workspace, size_t workspace_bytes,
                                   cudaStream_t stream);
 
+/* The same computation as medusa_heads_topk for callers that cannot allocate
+ * device memory: a host that reserves all device memory up front and gives
+ * this library no allocator, or code running where allocating is not
+ * allowed.  Instead of a caller workspace it uses a fixed 4 MiB scratch array
+ * that the library keeps in device memory (every GPU that loads the library
+ * holds those 4 MiB until the process exits); it calls no cudaMalloc,
+ * cudaFree or allocating routine.  The paper has no counterpart: this is an
+ * interface choice of this library.
+ *  - Arguments, layouts and outputs are those of medusa_heads_topk.
+ *  - Shapes whose scratch need (medusa_heads_workspace_size) exceeds 4 MiB
+ *    are rejected with MEDUSA_ERR_UNSUPPORTED before anything is enqueued.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; each call clears the part it uses on `stream` before launching.
+ *    Calls whose work overlaps on the GPU (other streams, other threads)
+ *    race on the array: serialise them. */
+medusa_status_t medusa_heads_topk_noalloc(const void* h, const void* W1, const void* b1,
+                                          const void* Wout, int B, int d, int V, int K, int topk,
+                                          medusa_dtype_t dtype, float* head_logits,
+                                          int32_t* topk_ids, float* topk_vals, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* S4: candidate assembly                                                    */
 /* ------------------------------------------------------------------------ */

@@ -44,7 +44,7 @@ EXPORTED = [
     "medusa_last_error", "medusa_abi_version", "medusa_device_status",
     "medusa_tree_choices_ranksum", "medusa_tree_create", "medusa_tree_destroy",
     "medusa_tree_info", "medusa_tree_tables",
-    "medusa_heads_workspace_size", "medusa_heads_topk",
+    "medusa_heads_workspace_size", "medusa_heads_topk", "medusa_heads_topk_noalloc",
     "medusa_build_tree",
     "medusa_attention_workspace_size", "medusa_tree_attention",
     "medusa_posterior_workspace_size", "medusa_evaluate_posterior",
@@ -99,6 +99,7 @@ _sig("medusa_tree_info", _i32, [_vp, _pi32, _pi32, _pi32])
 _sig("medusa_tree_tables", _i32, [_vp, _pi32, _pi32, _pi32, _pi32, _pu64])
 _sig("medusa_heads_workspace_size", _sz, [_i32] * 5)
 _sig("medusa_heads_topk", _i32, [_vp, _vp, _vp, _vp] + [_i32] * 5 + [_i32, _vp, _vp, _vp, _vp, _sz, _vp])
+_sig("medusa_heads_topk_noalloc", _i32, [_vp, _vp, _vp, _vp] + [_i32] * 5 + [_i32, _vp, _vp, _vp, _vp])
 _sig("medusa_build_tree", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp])
 _sig("medusa_attention_workspace_size", _sz, [_vp, _i32, _i32, _i32, _i32, _i32])
 _sig("medusa_tree_attention", _i32,
@@ -236,6 +237,14 @@ def medusa_heads_topk(h, W1, b1, Wout, topk, topk_ids, topk_vals, ws, head_logit
     _check(_lib.medusa_heads_topk(_p(h), _p(W1), _p(b1), _p(Wout), B, d, V, K, topk, _dtype(h),
                                   _p(head_logits), _p(topk_ids), _p(topk_vals), _p(ws),
                                   ws.numel(), _stream(stream)))
+
+
+def medusa_heads_topk_noalloc(h, W1, b1, Wout, topk, topk_ids, topk_vals, head_logits=None, stream=None):
+    """medusa_heads_topk without a workspace (the library's fixed scratch array)."""
+    B, d = h.shape
+    K, V = Wout.shape[0], Wout.shape[1]
+    _check(_lib.medusa_heads_topk_noalloc(_p(h), _p(W1), _p(b1), _p(Wout), B, d, V, K, topk, _dtype(h),
+                                          _p(head_logits), _p(topk_ids), _p(topk_vals), _stream(stream)))
 
 
 def medusa_build_tree(tree: Tree, root_tokens, topk_ids, seq_lens, tree_tokens, candidates,
