@@ -440,13 +440,12 @@ def run_ours(a, w):
 
 
 def kernel_revision():
-    """Hash of the kernel sources; ncu traffic figures are valid only for the revision they were taken on."""
+    """Hash of the heads kernel's sources; its ncu traffic figure holds only for that revision."""
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(REPO, "speculative_decoding_heads_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in ("heads.cu", "common.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:12]
 
 
