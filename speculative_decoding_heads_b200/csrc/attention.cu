@@ -21,6 +21,7 @@
 // keeps the result within 2e-3 of the exact value even when a few keys
 // dominate the softmax.
 #include <cfloat>
+#include <cstdlib>
 
 #include "common.cuh"
 
@@ -361,7 +362,22 @@ __global__ void __launch_bounds__(kMaxWarps * 32) tree_attn_mma(const TreeDev t,
   }
 }
 
+// MEDUSA_ATTN_MMA_SYNC=1 selects the legacy mma.sync kernel (kept for A/B
+// comparison while the tcgen05 kernel is validated).
+bool use_legacy_mma() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MEDUSA_ATTN_MMA_SYNC");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 }  // namespace
+
+medusa_status_t launch_attention_tc(const TreeDev& t, int layers, int B, int H, const void* q, const void* k_cache,
+                                    const void* v_cache, int Lcap, const int32_t* seq_lens, float scale_log2,
+                                    float* out, int* status, cudaStream_t stream);
 
 size_t attention_workspace_bytes(const TreeDev& t, int layers, int B, int H, int hd, medusa_dtype_t dtype) {
   (void)t;
@@ -381,6 +397,10 @@ medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int
   const int n_slices = layers * B * H;
   int* status = device_status_ptr();
   cudaError_t e;
+  if (dtype == MEDUSA_BF16 && hd == kHd && !use_legacy_mma()) {
+    return launch_attention_tc(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, scale * kLog2e,
+                               static_cast<float*>(out), status, stream);
+  }
   if (dtype == MEDUSA_BF16 && hd == kHd) {
     e = cudaFuncSetAttribute(tree_attn_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return cuda_fail("medusa_tree_attention: smem attribute", e);
