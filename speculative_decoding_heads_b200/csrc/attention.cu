@@ -375,10 +375,6 @@ bool use_legacy_mma() {
 
 }  // namespace
 
-medusa_status_t launch_attention_tc(const TreeDev& t, int layers, int B, int H, const void* q, const void* k_cache,
-                                    const void* v_cache, int Lcap, const int32_t* seq_lens, float scale_log2,
-                                    float* out, int* status, cudaStream_t stream);
-
 size_t attention_workspace_bytes(const TreeDev& t, int layers, int B, int H, int hd, medusa_dtype_t dtype) {
   (void)t;
   (void)layers;
@@ -398,6 +394,9 @@ medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int
   int* status = device_status_ptr();
   cudaError_t e;
   if (dtype == MEDUSA_BF16 && hd == kHd && !use_legacy_mma()) {
+    if (t.T <= 64)
+      return launch_attention_tc64(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, scale * kLog2e,
+                                   static_cast<float*>(out), status, stream);
     return launch_attention_tc(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, scale * kLog2e,
                                static_cast<float*>(out), status, stream);
   }

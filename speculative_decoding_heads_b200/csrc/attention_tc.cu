@@ -335,26 +335,27 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1)
 
 // ---- host side --------------------------------------------------------------
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+}  // namespace
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+void* tensor_map_encoder() {
+  static void* fn = nullptr;
   if (!fn) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+      fn = p;
   }
   return fn;
 }
-
-}  // namespace
 
 // Encodes the three tensor maps and launches the tcgen05 kernel.  Returns
 // MEDUSA_ERR_UNSUPPORTED when the shape does not fit it (caller falls back).
 medusa_status_t launch_attention_tc(const TreeDev& t, int layers, int B, int H, const void* q, const void* k_cache,
                                     const void* v_cache, int Lcap, const int32_t* seq_lens, float scale_log2,
                                     float* out, int* status, cudaStream_t stream) {
-  auto enc = encode_fn();
+  auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!enc) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: cuTensorMapEncodeTiled unavailable");
   const int M = t.T <= 64 ? 64 : 128;
   const int groups = (t.T + M - 1) / M;

@@ -74,6 +74,16 @@ medusa_status_t launch_accept_kv(const TreeDev& t, int layers, int B, int H, int
                                  int32_t* seq_lens, const int32_t* best_path,
                                  const int32_t* accept_len, cudaStream_t stream);
 
+// cuTensorMapEncodeTiled (PFN_cuTensorMapEncodeTiled_v12000), or null.
+void* tensor_map_encoder();
+
+medusa_status_t launch_attention_tc(const TreeDev& t, int layers, int B, int H, const void* q, const void* k_cache,
+                                    const void* v_cache, int Lcap, const int32_t* seq_lens, float scale_log2,
+                                    float* out, int* status, cudaStream_t stream);
+medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H, const void* q,
+                                      const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
+                                      float scale_log2, float* out, int* status, cudaStream_t stream);
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace medusa
