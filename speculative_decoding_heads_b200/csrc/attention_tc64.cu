@@ -16,8 +16,10 @@
 // Tensor memory (512 columns, M = 64 accumulators use lanes 0-15 of each
 // lane quarter; a second M = 64 accumulator can sit at lane offset 16):
 //   S     cols [0, 64)    lanes 0-15: keys 0-63 of the step, lanes 16-31: keys 64-127
-//   P     cols [64, 128)  the same lanes, P as bf16 pairs: high part in
-//                         [64, 96), remainder in [96, 128) (two keys per column)
+//   P     cols [64, 128) and [384, 448), alternating by step: the same lanes,
+//                         P as bf16 pairs (high part, then remainder; two keys
+//                         per column), so the softmax of step g+1 never waits
+//                         for the P V of step g
 //   O     cols [128, 256) and [256, 384), one per slice parity; lanes 0-15
 //                         accumulate keys 0-63 of every step, lanes 16-31
 //                         keys 64-127; the two are summed once per slice.
@@ -43,19 +45,21 @@ constexpr int kHalfTile = kStep * 128;         // 128 keys x 64 dims x 2 B = 16 
 constexpr int kTile = 2 * kHalfTile;           // one K or V tile: 32 KB
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColPhi = 64, kColPlo = 96, kColO = 128;
+constexpr uint32_t kColS = 0;                                             // 128 fp32 columns
+__device__ __forceinline__ uint32_t col_p(int buf) { return 128u + 64u * buf; }   // 64 packed columns
+__device__ __forceinline__ uint32_t col_o(int buf) { return 256u + 128u * buf; }  // 128 fp32 columns
 constexpr float kRescaleLog2 = 8.0f;
 
 // Shared memory (offsets from a 1024-byte aligned base).
-constexpr int kOffQ = 0;                                 // 2 x 16 KB
-constexpr int kOffKV = 2 * kRows * 256;                  // 3 stages x (K 32 KB + V 32 KB)
+constexpr int kOffQ = 0;                                 // 128 rows (each query twice) x 256 B
+constexpr int kOffKV = 128 * 256;                        // 3 stages x (K 32 KB + V 32 KB)
 constexpr int kOffBars = kOffKV + kStages * 2 * kTile;
 constexpr int kSmemBytes = kOffBars + 512 + 1024;
 
 struct Bars {
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full, q_empty;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full, s_free, p_full, pv_done;
+  uint64_t s_full, s_free, p_full, pv_done[2];   // pv_done[b]: the P V that read P buffer b
   uint64_t o_full[2], o_free[2];
   uint32_t tmem_base;
   int abort;
@@ -115,9 +119,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int T = p.t.T;
 
   if (tid == 0) {
+    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->q_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar->q_full[i], 1);
-      mbar_init(&bar->q_empty[i], 1);
       mbar_init(&bar->o_full[i], 1);
       mbar_init(&bar->o_free[i], 4);
     }
@@ -128,7 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar->s_full, 1);
     mbar_init(&bar->s_free, 4);
     mbar_init(&bar->p_full, 4);
-    mbar_init(&bar->pv_done, 1);
+    mbar_init(&bar->pv_done[0], 1);
+    mbar_init(&bar->pv_done[1], 1);
     bar->abort = 0;
     fence_barrier_init();
   }
@@ -143,56 +148,89 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
+    // Two streams, each issued as soon as its buffer is free: K/V tiles of
+    // every step, and the Q rows of every slice (Q waits for the last S of
+    // the previous slice; K/V of the next slice keep flowing meanwhile).
     tc::prefetch_tensormap(&q_map);
     tc::prefetch_tensormap(&k_map);
     tc::prefetch_tensormap(&v_map);
-    int g = 0, k = 0;
-    for (int kk = 0;; ++kk) {
-      const Slice s = slice_info(kk, p.total, p.B, p.H, T, p.Lcap, p.seq_lens);
-      if (s.slice >= p.total) break;
-      if (s.steps == 0) continue;
-      const int qb = k & 1;
-      if (k >= 2 && !wait_bar(&bar->q_empty[qb], ((k >> 1) - 1) & 1, bar, p.status)) break;
-      unsigned char* qd = smem + kOffQ + qb * kRows * 256;
-      mbar_arrive_expect_tx(&bar->q_full[qb], kRows * 256);
-      tc::tma_load_4d(qd, &q_map, 0, s.e, 0, s.lb, &bar->q_full[qb]);
-      tc::tma_load_4d(qd + kRows * 128, &q_map, 64, s.e, 0, s.lb, &bar->q_full[qb]);
-      for (int t = 0; t < s.steps; ++t, ++g) {
+    int g = 0, kv_kk = 0, kv_t = 0;            // K/V cursor: global step, slice, step within slice
+    int qk = 0, q_kk = 0;                      // Q cursor: slice count, slice index
+    Slice kvs = slice_info(0, p.total, p.B, p.H, T, p.Lcap, p.seq_lens);
+    while (kvs.slice < p.total && kvs.steps == 0) kvs = slice_info(++kv_kk, p.total, p.B, p.H, T, p.Lcap, p.seq_lens);
+    Slice qs = kvs;
+    q_kk = kv_kk;
+    const uint64_t t0 = globaltimer_ns();
+    uint64_t last = t0;
+    while ((kvs.slice < p.total || qs.slice < p.total) && !bar->abort) {
+      bool progressed = false;
+      if (qs.slice < p.total && (qk == 0 || mbar_test(&bar->q_empty, (qk - 1) & 1))) {
+        // Q rows 32q + 16c + i (c = 0, 1) both hold query 16q + i: one M = 128
+        // product then gives each lane pair the full 128-key row.
+        unsigned char* qd = smem + kOffQ;
+        mbar_arrive_expect_tx(&bar->q_full, 128 * 256);
+        for (int qq = 0; qq < 4; ++qq)
+          for (int c = 0; c < 2; ++c)
+            for (int rg = 0; rg < 2; ++rg)
+              tc::tma_load_4d(qd + rg * 128 * 128 + (32 * qq + 16 * c) * 128, &q_map, 64 * rg, qs.e, 16 * qq, qs.lb,
+                              &bar->q_full);
+        ++qk;
+        do {
+          qs = slice_info(++q_kk, p.total, p.B, p.H, T, p.Lcap, p.seq_lens);
+        } while (qs.slice < p.total && qs.steps == 0);
+        progressed = true;
+      }
+      if (kvs.slice < p.total) {
         const int st = g % kStages;
-        if (g >= kStages && !wait_bar(&bar->kv_empty[st], ((g / kStages) - 1) & 1, bar, p.status)) break;
-        unsigned char* kd = smem + kOffKV + st * 2 * kTile;
-        unsigned char* vd = kd + kTile;
-        mbar_arrive_expect_tx(&bar->kv_full[st], 2 * kTile);
-        if (p.kv_one_box) {
-          tc::tma_load_4d(kd, &k_map, 0, t * kStep, 0, s.slice, &bar->kv_full[st]);
-          tc::tma_load_4d(vd, &v_map, 0, t * kStep, 0, s.slice, &bar->kv_full[st]);
-        } else {
-          tc::tma_load_3d(kd, &k_map, 0, t * kStep, s.slice, &bar->kv_full[st]);
-          tc::tma_load_3d(kd + kHalfTile, &k_map, 64, t * kStep, s.slice, &bar->kv_full[st]);
-          tc::tma_load_3d(vd, &v_map, 0, t * kStep, s.slice, &bar->kv_full[st]);
-          tc::tma_load_3d(vd + kHalfTile, &v_map, 64, t * kStep, s.slice, &bar->kv_full[st]);
+        if (g < kStages || mbar_test(&bar->kv_empty[st], ((g / kStages) - 1) & 1)) {
+          unsigned char* kd = smem + kOffKV + st * 2 * kTile;
+          unsigned char* vd = kd + kTile;
+          mbar_arrive_expect_tx(&bar->kv_full[st], 2 * kTile);
+          if (p.kv_one_box) {
+            tc::tma_load_4d(kd, &k_map, 0, kv_t * kStep, 0, kvs.slice, &bar->kv_full[st]);
+            tc::tma_load_4d(vd, &v_map, 0, kv_t * kStep, 0, kvs.slice, &bar->kv_full[st]);
+          } else {
+            tc::tma_load_3d(kd, &k_map, 0, kv_t * kStep, kvs.slice, &bar->kv_full[st]);
+            tc::tma_load_3d(kd + kHalfTile, &k_map, 64, kv_t * kStep, kvs.slice, &bar->kv_full[st]);
+            tc::tma_load_3d(vd, &v_map, 0, kv_t * kStep, kvs.slice, &bar->kv_full[st]);
+            tc::tma_load_3d(vd + kHalfTile, &v_map, 64, kv_t * kStep, kvs.slice, &bar->kv_full[st]);
+          }
+          ++g;
+          if (++kv_t == kvs.steps) {
+            kv_t = 0;
+            do {
+              kvs = slice_info(++kv_kk, p.total, p.B, p.H, T, p.Lcap, p.seq_lens);
+            } while (kvs.slice < p.total && kvs.steps == 0);
+          }
+          progressed = true;
         }
       }
-      if (bar->abort) break;
-      ++k;
+      if (progressed) {
+        last = globaltimer_ns();
+      } else {
+        if (globaltimer_ns() - last > kSpinLimitNs) {
+          set_device_status(p.status, MEDUSA_ERR_TIMEOUT, kDetailAttnStageWait);
+          bar->abort = 1;
+          break;
+        }
+        __nanosleep(64);
+      }
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
-    constexpr uint32_t idS = tc::idesc_bf16_f32(64, 64, 0);
-    constexpr uint32_t idO = tc::idesc_bf16_f32(64, kHd, 1);
-    // S of global step g (slice k, step t): two M = 64 products, keys 0-63
-    // into lanes 0-15 and keys 64-127 into lanes 16-31.
-    auto issue_s = [&](int g, int k) {
-      const uint32_t qa = sbase + kOffQ + (k & 1) * kRows * 256;
+    constexpr uint32_t idS = tc::idesc_bf16_f32(128, kStep, 0);
+    constexpr uint32_t idO = tc::idesc_bf16_f32(128, kHd, 1);
+    // S of global step g: one M = 128, N = 128 product per 16 dims (8 in all);
+    // lane R gets all 128 keys of the query in Q row R.
+    auto issue_s = [&](int g) {
+      const uint32_t qa = sbase + kOffQ;
       const uint32_t kb = sbase + kOffKV + (g % kStages) * 2 * kTile;
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint64_t ad = tc::smem_desc_sw128(qa + (c >> 2) * kRows * 128 + (c & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::smem_desc_sw128(kb + (c >> 2) * kHalfTile + h * 64 * 128 + (c & 3) * 32, 16, 1024);
-          tc::mma_ss(tmem + (static_cast<uint32_t>(16 * h) << 16) + kColS, ad, bd, idS, c > 0 ? 1u : 0u);
-        }
+      for (int c = 0; c < 8; ++c) {
+        const uint64_t ad = tc::smem_desc_sw128(qa + (c >> 2) * 128 * 128 + (c & 3) * 32, 16, 1024);
+        const uint64_t bd = tc::smem_desc_sw128(kb + (c >> 2) * kHalfTile + (c & 3) * 32, 16, 1024);
+        tc::mma_ss(tmem + kColS, ad, bd, idS, c > 0 ? 1u : 0u);
+      }
       tc::mma_commit(&bar->s_full);
     };
     // Walk the same (slice, step) sequence as the producer, one step ahead for S.
@@ -200,11 +238,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     Slice cur = slice_info(0, p.total, p.B, p.H, T, p.Lcap, p.seq_lens);
     while (cur.slice < p.total && cur.steps == 0) cur = slice_info(++kk, p.total, p.B, p.H, T, p.Lcap, p.seq_lens);
     bool ok = cur.slice < p.total;
-    if (ok) ok = wait_bar(&bar->q_full[0], 0, bar, p.status) && wait_bar(&bar->kv_full[0], 0, bar, p.status);
+    if (ok) ok = wait_bar(&bar->q_full, 0, bar, p.status) && wait_bar(&bar->kv_full[0], 0, bar, p.status);
     if (ok) {
       tc::fence_after_sync();
-      issue_s(0, 0);
-      if (cur.steps == 1) tc::mma_commit(&bar->q_empty[0]);
+      issue_s(0);
+      if (cur.steps == 1) tc::mma_commit(&bar->q_empty);
     }
     while (ok) {
       for (int t = 0; ok && t < cur.steps; ++t, ++g) {
@@ -219,39 +257,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             nxt = slice_info(++nkk, p.total, p.B, p.H, T, p.Lcap, p.seq_lens);
           } while (nxt.slice < p.total && nxt.steps == 0);
         }
-        if (nxt.slice < p.total) {
-          if (nt == 0) ok = wait_bar(&bar->q_full[nk & 1], (nk >> 1) & 1, bar, p.status);
-          ok = ok && wait_bar(&bar->kv_full[(g + 1) % kStages], ((g + 1) / kStages) & 1, bar, p.status) &&
-               wait_bar(&bar->s_free, g & 1, bar, p.status);
-          if (!ok) break;
-          tc::fence_after_sync();
-          issue_s(g + 1, nk);
-          if (nt == nxt.steps - 1) tc::mma_commit(&bar->q_empty[nk & 1]);
-        }
-        // P V of step g into this slice's O buffer
-        if (!wait_bar(&bar->p_full, g & 1, bar, p.status)) {
-          ok = false;
-          break;
-        }
-        if (t == 0 && k >= 2 && !wait_bar(&bar->o_free[k & 1], ((k >> 1) - 1) & 1, bar, p.status)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-        const uint32_t vb = sbase + kOffKV + (g % kStages) * 2 * kTile + kTile;
-        const uint32_t ocol = kColO + (k & 1) * 128;
+        // Issue S of the next step and P V of this step in whichever order
+        // their inputs become ready (non-blocking tests, bounded overall).
+        bool need_s = nxt.slice < p.total;
+        bool need_pv = true;
+        const uint64_t t0 = globaltimer_ns();
+        while (need_s || need_pv) {
+          bool progressed = false;
+          if (need_s && (nt != 0 || mbar_test(&bar->q_full, nk & 1)) &&
+              mbar_test(&bar->kv_full[(g + 1) % kStages], ((g + 1) / kStages) & 1) && mbar_test(&bar->s_free, g & 1)) {
+            tc::fence_after_sync();
+            issue_s(g + 1);
+            if (nt == nxt.steps - 1) tc::mma_commit(&bar->q_empty);
+            need_s = false;
+            progressed = true;
+          }
+          if (need_pv && mbar_test(&bar->p_full, g & 1) &&
+              (t != 0 || k < 2 || mbar_test(&bar->o_free[k & 1], ((k >> 1) - 1) & 1))) {
+            tc::fence_after_sync();
+            const uint32_t vb = sbase + kOffKV + (g % kStages) * 2 * kTile + kTile;
+            // O (lanes with the high part of P) and O' (lanes with the
+            // remainder) += P V over the step's 128 keys, 16 keys per product.
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t lanes = static_cast<uint32_t>(16 * h) << 16;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint64_t bd = tc::smem_desc_sw128(vb + h * 64 * 128 + c * 16 * 128, kHalfTile, 1024);
-            tc::mma_ts(tmem + lanes + ocol, tmem + lanes + kColPhi + c * 8, bd, idO, (t > 0 || c > 0) ? 1u : 0u);
-            tc::mma_ts(tmem + lanes + ocol, tmem + lanes + kColPlo + c * 8, bd, idO, 1u);
+            for (int c = 0; c < 8; ++c) {
+              const uint64_t bd = tc::smem_desc_sw128(vb + c * 16 * 128, kHalfTile, 1024);
+              tc::mma_ts(tmem + col_o(k & 1), tmem + col_p(g & 1) + c * 8, bd, idO, (t > 0 || c > 0) ? 1u : 0u);
+            }
+            need_pv = false;
+            progressed = true;
+          }
+          if (!progressed) {
+            if (bar->abort || globaltimer_ns() - t0 > kSpinLimitNs) {
+              set_device_status(p.status, MEDUSA_ERR_TIMEOUT, kDetailAttnStageWait);
+              bar->abort = 1;
+              ok = false;
+              break;
+            }
+            __nanosleep(20);
           }
         }
+        if (!ok) break;
         tc::mma_commit(&bar->kv_empty[g % kStages]);
-        tc::mma_commit(&bar->pv_done);
+        tc::mma_commit(&bar->pv_done[g & 1]);
         if (t == cur.steps - 1) tc::mma_commit(&bar->o_full[k & 1]);
       }
       if (!ok) break;
@@ -288,10 +335,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc::fence_after_sync();
+        // tcgen05.ld addresses are warp-uniform: read both 64-key halves of
+        // the row and keep this lane's half (h).
         float sv[64];
-        tc::tmem_ld32(tmem + la + kColS, sv);
-        tc::tmem_ld32(tmem + la + kColS + 32, sv + 32);
-        tc::tmem_wait_ld();
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          float a[32], b[32];
+          tc::tmem_ld32(tmem + la + kColS + 32 * part, a);
+          tc::tmem_ld32(tmem + la + kColS + 64 + 32 * part, b);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sv[32 * part + c] = h ? b[c] : a[c];
+        }
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&bar->s_free);
@@ -332,17 +387,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           ps += sv[c];
         }
         lsum = lsum * factor + ps;
-        // P V of the previous step must be done: P is about to be overwritten
-        // and O may be rescaled.
-        if (g > 0) {
-          if (!wait_bar(&bar->pv_done, (g - 1) & 1, bar, p.status)) {
+        // O is rescaled only after every P V issued into it is done (rare);
+        // P buffer g&1 is rewritten once the P V of step g-2 has read it.
+        const uint32_t ocol = col_o(k & 1);
+        if (t > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
+          if (!wait_bar(&bar->pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, bar, p.status)) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
-        }
-        const uint32_t ocol = kColO + (k & 1) * 128;
-        if (t > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
 #pragma unroll 1
           for (int c0 = 0; c0 < kHd; c0 += 32) {
             float o[32];
@@ -353,6 +406,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::tmem_st32(tmem + la + ocol + c0, o);
           }
         }
+        if (g >= 2) {
+          if (!wait_bar(&bar->pv_done[g & 1], ((g - 2) >> 1) & 1, bar, p.status)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+        }
         float hi[32], lo[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -361,8 +421,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           hi[c] = __uint_as_float(ph);
           lo[c] = __uint_as_float(pack2(a0 - __uint_as_float(ph << 16), a1 - __uint_as_float(ph & 0xffff0000u)));
         }
-        tc::tmem_st32(tmem + la + kColPhi, hi);
-        tc::tmem_st32(tmem + la + kColPlo, lo);
+        // Lane pair (h = 0, 1) of a query: the h = 0 lane stores the high
+        // parts of all 128 keys, the h = 1 lane the remainders, so one M = 128
+        // product accumulates both; each lane hands its partner the half it
+        // lacks.
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float send = h == 0 ? lo[c] : hi[c];
+          const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+          if (h == 0) lo[c] = recv;   // lo[] now: high parts of keys 64-127
+          else hi[c] = recv;          // hi[] now: remainders of keys 0-63
+        }
+        tc::tmem_st32(tmem + la + col_p(g & 1), hi);
+        tc::tmem_st32(tmem + la + col_p(g & 1) + 32, lo);
         tc::tmem_wait_st();
         if (t == s.steps - 1 && t * kStep + kStep > s.n) {
           // V rows past the slice's last key: zero them so 0 * (stale value) stays 0.
@@ -442,7 +513,7 @@ medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H
                                 static_cast<cuuint64_t>(t.T), static_cast<cuuint64_t>(layers) * B};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHd) * 2, static_cast<cuuint64_t>(H) * kHd * 2,
                                    static_cast<cuuint64_t>(t.T) * H * kHd * 2};
-    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kRows), 1};
+    const cuuint32_t box[4] = {64, 1, 16, 1};
     const cuuint32_t es[4] = {1, 1, 1, 1};
     if (enc(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
