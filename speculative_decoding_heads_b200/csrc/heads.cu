@@ -14,22 +14,25 @@
 //  * One CTA per SM, launched cooperatively so all CTAs are resident.  The
 //    W1 rows (K*d) and then the Wout rows (K*V) are split evenly over the
 //    CTAs; every CTA streams its rows through a ring of shared-memory stages
-//    filled by 1-D TMA bulk copies (cp.async.bulk + mbarrier complete_tx),
-//    with an L2 evict-first hint because every weight byte is read once.
-//  * Thread t owns the 16-byte column vectors t, t+NT, ... of every row and
-//    keeps the matching slice of h (phase 1) or u (phase 2) in registers, so
-//    shared memory only carries the weights.  A stage of R rows gives R*NB
-//    partial dot products per thread, reduced by warp shuffles and then
-//    across warps through a small double-buffered shared array.
-//  * Phase 1 writes u to the workspace and, once all of a CTA's W1 rows are
-//    done, bumps a release counter.  Phase 2 issues its first Wout copies
-//    before it waits (acquire, bounded) for every CTA's phase 1, so the
-//    weight stream never stops at the S1 -> S2 boundary.
-//  * Warp 0 keeps a running top-k per (sequence, head) in shared memory; a
-//    new logit is inserted only when it beats the current k-th entry.  At the
-//    end each CTA publishes its lists, and the last CTA to finish merges
-//    them (k rounds of a warp arg-max over the published candidates) and
-//    resets the counters for the next call.
+//    (R rows each) filled by 1-D TMA bulk copies (cp.async.bulk + mbarrier
+//    complete_tx) with an L2 evict-first hint: every weight byte is read once.
+//  * Warp-specialised: warp 0 issues the copies and refills a stage as soon
+//    as every consumer warp has released it; the consumer warps (thread t
+//    owns the 16-byte column vectors t, t+NT, ... of every row and keeps the
+//    matching slice of h or u in registers) turn a stage into R*NB partial
+//    dot products per warp; warp 1 (epilogue) sums the partials of the
+//    consumer warps and applies S1's residual/SiLU or S3's running top-k.
+//    Stages, partial buffers and the epilogue are decoupled by mbarriers, so
+//    no CTA-wide barrier sits on the weight stream.
+//  * Phase 1 writes u to the workspace; once a CTA's last W1 row is done,
+//    the epilogue warp bumps a release counter and waits (acquire, bounded)
+//    for every CTA, then lets the consumers load u.  Wout copies keep
+//    flowing meanwhile, so the stream never stops at the S1 -> S2 boundary.
+//  * The epilogue warp keeps a running top-k per (sequence, head) in shared
+//    memory; a new logit is inserted only when it beats the current k-th
+//    entry.  At the end each CTA publishes its lists, and the last CTA to
+//    finish merges them (k rounds of a warp arg-max over the published
+//    candidates) and resets the counters for the next call.
 #include <cfloat>
 #include <cstdint>
 
@@ -38,10 +41,13 @@
 namespace medusa {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kMaxConsumers = 512;    // consumer threads
+constexpr int kRoleWarps = 2;         // producer + epilogue
+constexpr int kMaxThreads = kMaxConsumers + 32 * kRoleWarps;
 constexpr int kMaxNB = 4;             // sequences per launch
-constexpr int kStageTarget = 200 * 1024;
-constexpr int kMaxStages = 8;
+constexpr int kStageMax = 64 * 1024;  // bytes per stage: 8 rows when they fit, else 4
+constexpr int kRingTarget = 192 * 1024;
+constexpr int kMaxStages = 12;
 
 struct HeadsArgs {
   const void* h;
@@ -61,6 +67,8 @@ struct HeadsArgs {
   int G;
   int NS;                 // stages in the ring
   int nvec;               // 16-byte vectors per row
+  int NT;                 // consumer threads
+  int p1_max;             // most phase-1 rows of any CTA
 };
 
 template <typename TW>
@@ -267,31 +275,69 @@ __device__ __forceinline__ void list_insert(float* lv, int* lid, int* cnt_p, int
 
 constexpr int kMergeRegs = 16;   // candidates per lane held in registers by the merge
 
+// Shared-memory carve-up of one CTA (offsets in bytes; stages first, 128-byte aligned).
+struct Layout {
+  size_t stages, partial, pre_h, pre_b, list_v, list_i, list_n, bars, flags, total;
+};
+
+__host__ __device__ inline Layout make_layout(size_t stage_bytes, int NS, int NWC, int RNB, int NB, int K, int topk,
+                                              int p1_max) {
+  Layout l{};
+  size_t o = 0;
+  l.stages = o;
+  o += stage_bytes * NS;
+  l.partial = o;                                   // [NS][NWC][RNB] fp32
+  o += static_cast<size_t>(NS) * NWC * RNB * 4;
+  l.pre_h = o;                                     // [p1_max][NB] fp32: h[b][row within head]
+  o += static_cast<size_t>(p1_max) * NB * 4;
+  l.pre_b = o;                                     // [p1_max] fp32: b1[head][row within head]
+  o += static_cast<size_t>(p1_max) * 4;
+  l.list_v = o;                                    // [NB][K][topk]
+  o += static_cast<size_t>(NB) * K * topk * 4;
+  l.list_i = o;
+  o += static_cast<size_t>(NB) * K * topk * 4;
+  l.list_n = o;                                    // [NB][K]
+  o += static_cast<size_t>(NB) * K * 4;
+  o = (o + 15) & ~size_t(15);
+  l.bars = o;                                      // full, empty, pready, pfree [NS] each; u_ready
+  o += (4 * static_cast<size_t>(NS) + 1) * 8;
+  l.flags = o;                                     // [0] abort, [1] last-CTA flag
+  o += 16;
+  l.total = o;
+  return l;
+}
+
 template <typename TW, int NB, int VPT, int R>
-__global__ void __launch_bounds__(kThreads, 1) heads_kernel(const HeadsArgs a) {
+__global__ void __launch_bounds__(kMaxThreads, 1) heads_kernel(const HeadsArgs a) {
   constexpr int E = Elem<TW>::E;
   constexpr int RNB = R * NB;
-  static_assert(RNB <= 32 && (32 % RNB) == 0, "stage epilogue uses one lane per (row, sequence)");
+  static_assert(RNB <= 32 && (32 % RNB) == 0, "partials use one lane per (row, sequence)");
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const int NW = blockDim.x >> 5;
+  const int NWC = a.NT >> 5;                      // consumer warps
   const int cta = blockIdx.x;
   const int G = a.G;
+  const int NS = a.NS;
   const size_t row_bytes = static_cast<size_t>(a.d) * sizeof(TW);
   const size_t stage_bytes = row_bytes * R;
+  const Layout lay = make_layout(stage_bytes, NS, NWC, RNB, NB, a.K, a.topk, a.p1_max);
 
-  // shared-memory carve-up
-  unsigned char* stages = smem;
-  float* partial = reinterpret_cast<float*>(smem + stage_bytes * a.NS);   // [2][NW][RNB]
-  float* list_v = partial + 2 * NW * RNB;                                  // [NB][K][topk]
-  int* list_i = reinterpret_cast<int*>(list_v + NB * a.K * a.topk);
-  int* list_n = list_i + NB * a.K * a.topk;                                // [NB][K]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(list_n + NB * a.K) + 15) & ~uintptr_t(15));  // [NS]
-  int* flag = reinterpret_cast<int*>(bars + a.NS);
+  unsigned char* stages = smem + lay.stages;
+  float* partial = reinterpret_cast<float*>(smem + lay.partial);
+  float* pre_h = reinterpret_cast<float*>(smem + lay.pre_h);
+  float* pre_b = reinterpret_cast<float*>(smem + lay.pre_b);
+  float* list_v = reinterpret_cast<float*>(smem + lay.list_v);
+  int* list_i = reinterpret_cast<int*>(smem + lay.list_i);
+  int* list_n = reinterpret_cast<int*>(smem + lay.list_n);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
+  uint64_t* empty = full + NS;
+  uint64_t* pready = empty + NS;
+  uint64_t* pfree = pready + NS;
+  uint64_t* u_ready = pfree + NS;
+  volatile int* flag = reinterpret_cast<volatile int*>(smem + lay.flags);
 
   const int n1 = a.K * a.d;
   const int n2 = a.K * a.V;
@@ -304,56 +350,146 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(const HeadsArgs a) {
   }
   for (int i = tid; i < NB * a.K; i += blockDim.x) list_n[i] = 0;
   if (tid == 0) {
-    for (int s = 0; s < a.NS; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NWC);
+      mbar_init(&pready[s], NWC * RNB);
+      mbar_init(&pfree[s], 1);
+    }
+    mbar_init(u_ready, 1);
     fence_barrier_init();
     flag[0] = 0;
+    flag[1] = 0;
   }
   __syncthreads();
 
-  const uint64_t policy = l2_evict_first_policy();
-  // Producer cursor (thread 0 only): the first NS stages go out now.
-  Cursor pc;
-  cursor_start<R>(pc, a, p1_lo, p1_hi, p2_lo, p2_hi);
-  int issued = 0;
-  if (tid == 0) {
-    for (; issued < a.NS && pc.phase != 3; ++issued) {
-      const uint32_t bytes = static_cast<uint32_t>(pc.n * row_bytes);
-      mbar_arrive_expect_tx(&bars[issued], bytes);
-      tma_load_1d(stages + issued * stage_bytes, stage_src<TW>(a, pc), bytes, &bars[issued], policy);
-      cursor_next<R>(pc, a);
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      const uint64_t policy = l2_evict_first_policy();
+      Cursor pc;
+      cursor_start<R>(pc, a, p1_lo, p1_hi, p2_lo, p2_hi);
+      int s = 0;
+      for (; pc.phase != 3; ++s) {
+        const int slot = s % NS;
+        if (s >= NS && !mbar_wait(&empty[slot], static_cast<uint32_t>(((s / NS) - 1) & 1))) {
+          set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsStageWait);
+          flag[0] = 1;
+          break;
+        }
+        if (flag[0]) break;
+        const uint32_t bytes = static_cast<uint32_t>(pc.n * row_bytes);
+        mbar_arrive_expect_tx(&full[slot], bytes);
+        tma_load_1d(stages + slot * stage_bytes, stage_src<TW>(a, pc), bytes, &full[slot], policy);
+        cursor_next<R>(pc, a);
+      }
+      // Every copy issued lands before the CTA exits (after an abort the
+      // consumers may not have waited for the last ones).
+      for (int t = s - NS < 0 ? 0 : s - NS; t < s; ++t)
+        mbar_wait(&full[t % NS], static_cast<uint32_t>((t / NS) & 1));
     }
   }
-
-  // x[b*VPT+j][e]: h (phase 1) or u of the current head (phase 2), for the
-  // thread's column vectors tid + j*NT.
-  float x[NB * VPT][E];
+  else if (warp >= kRoleWarps) {
+    // ---------------- consumers ----------------
+    const int ct = tid - 32 * kRoleWarps;
+    const int cw = warp - kRoleWarps;
+    // x[b*VPT+j][e]: h (phase 1) or u of the current head (phase 2), for the
+    // thread's column vectors ct + j*NT.
+    float x[NB * VPT][E];
 #pragma unroll
-  for (int b = 0; b < NB; ++b)
+    for (int b = 0; b < NB; ++b)
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      const int v = tid + j * blockDim.x;
-      if (b < a.nb && v < a.nvec) {
-        load_vec<TW>(static_cast<const TW*>(a.h) + static_cast<size_t>(a.b0 + b) * a.d, v, x[b * VPT + j]);
-      } else {
+      for (int j = 0; j < VPT; ++j) {
+        const int v = ct + j * a.NT;
+        if (b < a.nb && v < a.nvec) {
+          load_vec<TW>(static_cast<const TW*>(a.h) + static_cast<size_t>(a.b0 + b) * a.d, v, x[b * VPT + j]);
+        } else {
 #pragma unroll
-        for (int e = 0; e < E; ++e) x[b * VPT + j][e] = 0.f;
+          for (int e = 0; e < E; ++e) x[b * VPT + j][e] = 0.f;
+        }
       }
-    }
+    Cursor cc;
+    cursor_start<R>(cc, a, p1_lo, p1_hi, p2_lo, p2_hi);
+    int cur_head2 = -1;   // head whose u sits in x during phase 2
+    bool u_ok = false;
+    for (int s = 0; cc.phase != 3; ++s) {
+      const int slot = s % NS;
+      const int khead = cc.head;   // uniform per stage
+      if (cc.phase == 2 && khead != cur_head2) {
+        if (!u_ok) {
+          if (!mbar_wait(u_ready, 0u)) {
+            set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsS1Wait);
+            flag[0] = 1;
+          }
+          if (flag[0]) break;
+          u_ok = true;
+        }
+        cur_head2 = khead;
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int j = 0; j < VPT; ++j) {
+            const int v = ct + j * a.NT;
+            if (b < a.nb && v < a.nvec)
+              load_u_vec(a.u + (static_cast<size_t>(a.b0 + b) * a.K + khead) * a.d, v, E, x[b * VPT + j]);
+          }
+      }
+      if (!mbar_wait(&full[slot], static_cast<uint32_t>((s / NS) & 1))) {
+        set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsStageWait);
+        flag[0] = 1;
+      }
+      if (flag[0]) break;
 
-  Cursor cc;
-  cursor_start<R>(cc, a, p1_lo, p1_hi, p2_lo, p2_hi);
-  int cur_head2 = -1;   // head whose u sits in x during phase 2
-  bool published = false;
-  bool aborted = false;
-  int s = 0;
-  for (; cc.phase != 3; ++s) {
-    const int slot = s % a.NS;
-    if (cc.phase == 2 && !published) {
-      // First phase-2 stage: publish this CTA's phase 1, then wait (bounded)
-      // until every CTA has published.  The Wout copies are already in flight.
-      published = true;
-      __syncthreads();
-      if (tid == 0) {
+      float acc[RNB];
+#pragma unroll
+      for (int i = 0; i < RNB; ++i) acc[i] = 0.f;
+      const unsigned char* st = stages + slot * stage_bytes;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (r < cc.n) {
+#pragma unroll
+          for (int j = 0; j < VPT; ++j) {
+            const int v = ct + j * a.NT;
+            if (v < a.nvec) {
+              const uint4 w = *reinterpret_cast<const uint4*>(st + r * row_bytes + static_cast<size_t>(v) * 16);
+              dot_vec<TW, NB, VPT>(w, x, j, acc + r * NB);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cta(&empty[slot]);   // this warp is done with the stage's bytes
+      int idx = 0;
+      WarpFold<RNB, 16>::run(acc, lane, idx);
+      if (s >= NS && !mbar_wait(&pfree[slot], static_cast<uint32_t>(((s / NS) - 1) & 1))) {
+        set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsStageWait);
+        flag[0] = 1;
+        break;
+      }
+      if ((lane & (32 / RNB - 1)) == 0) {
+        partial[(slot * NWC + cw) * RNB + idx] = acc[0];
+        mbar_arrive_cta(&pready[slot]);
+      }
+      cursor_next<R>(cc, a);
+    }
+  } else {
+    // ---------------- epilogue (warp 1) ----------------
+    for (int i = lane; i < p1_hi - p1_lo; i += 32) {
+      const int row = p1_lo + i;
+      const int head = row / a.d;
+      const int local = row - head * a.d;
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        pre_h[i * NB + b] =
+            b < a.nb ? to_f32<TW>(static_cast<const TW*>(a.h)[static_cast<size_t>(a.b0 + b) * a.d + local]) : 0.f;
+      pre_b[i] = to_f32<TW>(static_cast<const TW*>(a.b1)[static_cast<size_t>(head) * a.d + local]);
+    }
+    __syncwarp();
+    // This CTA's u rows are written: count it, wait (bounded) for every CTA,
+    // then let the consumers read u.
+    auto publish = [&]() {
+      __syncwarp();
+      if (lane == 0) {
         __threadfence();
         atom_add_release_gpu(&a.counters[0], 1u);
         const uint64_t t0 = globaltimer_ns();
@@ -365,81 +501,41 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(const HeadsArgs a) {
           }
           __nanosleep(64);
         }
+        mbar_arrive_cta(u_ready);
       }
-      __syncthreads();
-      if (flag[0]) {
-        aborted = true;
-        break;
+      __syncwarp();
+    };
+    if (p1_hi == p1_lo) publish();
+    Cursor cc;
+    cursor_start<R>(cc, a, p1_lo, p1_hi, p2_lo, p2_hi);
+    for (int s = 0; cc.phase != 3; ++s) {
+      const int slot = s % NS;
+      if (!mbar_wait(&pready[slot], static_cast<uint32_t>((s / NS) & 1))) {
+        set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsStageWait);
+        flag[0] = 1;
       }
-    }
-    const int khead = cc.head;   // uniform per stage
-    if (cc.phase == 2 && khead != cur_head2) {
-      cur_head2 = khead;
-#pragma unroll
-      for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int j = 0; j < VPT; ++j) {
-          const int v = tid + j * blockDim.x;
-          if (b < a.nb && v < a.nvec)
-            load_u_vec(a.u + (static_cast<size_t>(a.b0 + b) * a.K + khead) * a.d, v, E, x[b * VPT + j]);
-        }
-    }
-
-    if (!mbar_wait(&bars[slot], static_cast<uint32_t>((s / a.NS) & 1))) {
-      set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsStageWait);
-      aborted = true;
-      break;
-    }
-
-    float acc[RNB];
-#pragma unroll
-    for (int i = 0; i < RNB; ++i) acc[i] = 0.f;
-    const unsigned char* st = stages + slot * stage_bytes;
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      if (r < cc.n) {
-#pragma unroll
-        for (int j = 0; j < VPT; ++j) {
-          const int v = tid + j * blockDim.x;
-          if (v < a.nvec) {
-            const uint4 w = *reinterpret_cast<const uint4*>(st + r * row_bytes + static_cast<size_t>(v) * 16);
-            dot_vec<TW, NB, VPT>(w, x, j, acc + r * NB);
-          }
-        }
-      }
-    }
-    int idx = 0;
-    WarpFold<RNB, 16>::run(acc, lane, idx);
-    float* pbuf = partial + (s & 1) * NW * RNB;
-    if ((lane & (32 / RNB - 1)) == 0) pbuf[warp * RNB + idx] = acc[0];
-    __syncthreads();   // the stage slot is free and the partials are complete
-
-    if (tid == 0 && pc.phase != 3) {
-      const uint32_t bytes = static_cast<uint32_t>(pc.n * row_bytes);
-      mbar_arrive_expect_tx(&bars[slot], bytes);
-      tma_load_1d(stages + slot * stage_bytes, stage_src<TW>(a, pc), bytes, &bars[slot], policy);
-      cursor_next<R>(pc, a);
-      ++issued;
-    }
-
-    if (warp == 0) {
-      // Cross-warp sum: lane l adds entries l, l+32, ... (all of value l % RNB),
-      // then lanes with equal l % RNB combine.
+      if (flag[0]) break;
+      // Cross-warp sum: lane l adds entries l, l+32, ... (all of value
+      // l % RNB), then lanes with equal l % RNB combine.
       float val = 0.f;
-      for (int e = lane; e < NW * RNB; e += 32) val += pbuf[e];
+      const float* pb = partial + slot * NWC * RNB;
+      for (int e = lane; e < NWC * RNB; e += 32) val += pb[e];
 #pragma unroll
       for (int o = RNB; o < 32; o <<= 1) val += __shfl_xor_sync(0xffffffffu, val, o);
-      // Stage epilogue: lane t < RNB owns row t / NB and sequence t % NB.
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cta(&pfree[slot]);
+      // Lane t < RNB owns row t / NB and sequence t % NB of the stage.
+      const int khead = cc.head;
       const int r = lane / NB, b = lane % NB;
       const bool live = lane < RNB && r < cc.n && b < a.nb;
       const int local = cc.row - khead * (cc.phase == 1 ? a.d : a.V) + r;   // row within the head
       if (cc.phase == 1) {
         if (live) {
-          const float hb = to_f32<TW>(static_cast<const TW*>(a.h)[static_cast<size_t>(a.b0 + b) * a.d + local]);
-          const float bb = to_f32<TW>(static_cast<const TW*>(a.b1)[static_cast<size_t>(khead) * a.d + local]);
-          a.u[(static_cast<size_t>(a.b0 + b) * a.K + khead) * a.d + local] = hb + silu(val + bb);
+          const int i = cc.row - p1_lo + r;
+          a.u[(static_cast<size_t>(a.b0 + b) * a.K + khead) * a.d + local] = pre_h[i * NB + b] + silu(val + pre_b[i]);
           __threadfence();
         }
+        if (cc.row + cc.n >= cc.end) publish();   // the CTA's last W1 stage
       } else {
         if (live && a.head_logits)
           a.head_logits[(static_cast<size_t>(a.b0 + b) * a.K + khead) * a.V + local] = val;
@@ -459,23 +555,11 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(const HeadsArgs a) {
           list_insert(list_v + li * a.topk, list_i + li * a.topk, list_n + li, a.topk, nv, nid, lane);
         }
       }
+      cursor_next<R>(cc, a);
     }
-    cursor_next<R>(cc, a);
-  }
-
-  if (aborted) {
-    // Drain the copies this CTA issued so that none lands after it exits.
-    if (tid == 0)
-      for (int t = s; t < issued; ++t) mbar_wait(&bars[t % a.NS], static_cast<uint32_t>((t / a.NS) & 1));
-    __syncthreads();
-    return;
   }
   __syncthreads();
-  if (!published && tid == 0) {
-    // No phase-2 rows here: still count this CTA's phase 1.
-    __threadfence();
-    atom_add_release_gpu(&a.counters[0], 1u);
-  }
+  if (flag[0]) return;   // aborted: the producer has drained its copies
 
   // Publish the local lists of every head this CTA's phase-2 rows touched.
   if (p2_hi > p2_lo) {
@@ -503,6 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1) heads_kernel(const HeadsArgs a) {
   // candidates of one list are loaded once; each of the topk rounds picks
   // the best candidate that ranks strictly after the previous pick.
   __threadfence();
+  const int NW = blockDim.x >> 5;
   for (int li = warp; li < a.nb * a.K; li += NW) {
     const int b = li / a.K, k = li % a.K;
     const int hk_lo = k * a.V;
@@ -572,23 +657,24 @@ struct Plan {
   size_t smem;
 };
 
-// Rows per stage: 8 when the batch group is at most 2 and 8 rows fit in
-// 64 KB, else 4.  Stages: as many as fit in ~200 KB (at least 2, at most 8).
+// Consumer threads: one per 16-byte column vector up to 512.  Stages of 8
+// rows when 8 rows fit in 64 KB, else 4: one bulk copy per stage, and on
+// this hardware a few large copies in flight stream HBM far better than
+// many small ones (64 KB stages reach ~94% of the copy bandwidth, 32 KB
+// ~68%).  As many stages as fit in ~192 KB (at least 2, at most 12).
 template <typename TW>
-Plan make_plan(int d, int nb, int K, int topk) {
+Plan make_plan(int d, int nb, int K, int topk, int p1_max) {
   constexpr int E = Elem<TW>::E;
   Plan p{};
   const int nvec = d / E;
-  p.NT = nvec >= kThreads ? kThreads : ((nvec + 31) / 32) * 32;
+  p.NT = nvec >= kMaxConsumers ? kMaxConsumers : ((nvec + 31) / 32) * 32;
   p.VPT = (nvec + p.NT - 1) / p.NT;
   const size_t row = static_cast<size_t>(d) * sizeof(TW);
-  p.R = (nb <= 2 && row * 8 <= 64 * 1024) ? 8 : 4;
+  p.R = row * 8 <= static_cast<size_t>(kStageMax) ? 8 : 4;
   const size_t stage = row * p.R;
-  const int ns = static_cast<int>(kStageTarget / stage);
+  const int ns = static_cast<int>(kRingTarget / stage);
   p.NS = ns < 2 ? 2 : (ns > kMaxStages ? kMaxStages : ns);
-  const int NW = p.NT / 32;
-  p.smem = stage * p.NS + 2 * NW * 32 * sizeof(float) + kMaxNB * K * topk * (sizeof(float) + sizeof(int)) +
-           kMaxNB * K * sizeof(int) + 16 + p.NS * sizeof(uint64_t) + 64;
+  p.smem = make_layout(stage, p.NS, p.NT / 32, p.R * nb, nb, K, topk, p1_max).total;
   return p;
 }
 
@@ -598,18 +684,20 @@ cudaError_t launch_one(const HeadsArgs& a, const Plan& p, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(p.smem));
   if (e != cudaSuccess) return e;
+  const int threads = p.NT + 32 * kRoleWarps;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, p.NT, p.smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, p.smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   void* args[] = {const_cast<HeadsArgs*>(&a)};
-  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(fn), dim3(a.G), dim3(p.NT), args,
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(fn), dim3(a.G), dim3(threads), args,
                                      p.smem, stream);
 }
 
+// Two vectors per thread means rows of at least 16 KB, hence 4-row stages.
 template <typename TW, int NB, int VPT>
 cudaError_t dispatch_r(const HeadsArgs& a, const Plan& p, cudaStream_t stream) {
-  if constexpr (NB <= 2) {
+  if constexpr (VPT == 1) {
     if (p.R == 8) return launch_one<TW, NB, VPT, 8>(a, p, stream);
   }
   return launch_one<TW, NB, VPT, 4>(a, p, stream);
@@ -670,12 +758,15 @@ medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, cons
   a.status = device_status_ptr();
   a.G = G;
   a.nvec = (dtype == MEDUSA_BF16) ? d / 8 : d / 4;
+  a.p1_max = static_cast<int>((static_cast<long long>(K) * d + G - 1) / G) + 1;
   for (int b0 = 0; b0 < B; b0 += kMaxNB) {
     a.b0 = b0;
     a.nb = (B - b0) < kMaxNB ? (B - b0) : kMaxNB;
     const int nbt = a.nb == 1 ? 1 : (a.nb == 2 ? 2 : 4);
-    const Plan p = (dtype == MEDUSA_BF16) ? make_plan<uint16_t>(d, nbt, K, topk) : make_plan<float>(d, nbt, K, topk);
+    const Plan p = (dtype == MEDUSA_BF16) ? make_plan<uint16_t>(d, nbt, K, topk, a.p1_max)
+                                          : make_plan<float>(d, nbt, K, topk, a.p1_max);
     a.NS = p.NS;
+    a.NT = p.NT;
     cudaError_t e = (dtype == MEDUSA_BF16) ? dispatch_nb<uint16_t>(a, p, stream) : dispatch_nb<float>(a, p, stream);
     if (e != cudaSuccess) return cuda_fail("medusa_heads_topk: launch", e);
   }
