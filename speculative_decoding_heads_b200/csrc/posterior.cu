@@ -4,14 +4,16 @@
 // "Medusa — 让大模型自己同时猜好几个 token", 核心要点: typical acceptance, and
 // 实践案例 case 1 step 4: keep the longest acceptable prefix from the root).
 //
-// Kernel 1, one CTA per (sequence, tree node): one pass over the node's V
-// base logits for the arg-max (lower id on ties) and, for typical
-// acceptance, a second pass for the tempered softmax statistics
+// One kernel, one CTA of 1024 threads per (sequence, tree node): the node's
+// V base logits are loaded once into registers (8 float4 per thread, all in
+// flight together), giving the arg-max (lower id on ties) and, for typical
+// acceptance, the tempered softmax statistics
 //     m = max z/T,  S = sum exp(z/T - m),  E = sum exp(z/T - m) (z/T - m)
 // so that H = ln S - E / S and thr = min(eps, alpha exp(-H)).
-// Kernel 2, one CTA per sequence, one thread per path: walk the path from
-// the root, count the leading accepted depths, then reduce (max count,
-// lowest path index) and write the step's outputs.
+// The last CTA of a sequence to finish (a self-resetting counter in the
+// workspace) then walks every path from the root with one thread per path,
+// counts the leading accepted depths, reduces (max count, lowest path index)
+// and writes the step's outputs.
 #include <cfloat>
 
 #include "common.cuh"
@@ -19,7 +21,9 @@
 namespace medusa {
 namespace {
 
-constexpr int kStatThreads = 256;
+constexpr int kThreads = 1024;
+constexpr int kVecPerThread = 8;          // float4 per thread held in registers per chunk
+constexpr int kChunk = kThreads * kVecPerThread * 4;   // logits per chunk (32768)
 
 struct NodeStat {
   int argmax;
@@ -35,101 +39,138 @@ __device__ __forceinline__ void argmax_merge(float& v, int& i, float ov, int oi)
   }
 }
 
-__global__ void __launch_bounds__(kStatThreads) node_stats_kernel(const float* __restrict__ logits, int V,
-                                                                  int typical, float inv_t_unused,
-                                                                  float temperature, float eps, float alpha,
-                                                                  NodeStat* __restrict__ stats) {
-  (void)inv_t_unused;
-  const int row = blockIdx.x;
-  const float* z = logits + static_cast<size_t>(row) * V;
-  __shared__ float red_v[kStatThreads / 32];
-  __shared__ int red_i[kStatThreads / 32];
-  __shared__ float red_s[kStatThreads / 32], red_e[kStatThreads / 32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  float bv = -FLT_MAX;
-  int bi = 0x7fffffff;
-  const bool vec_ok = (V % 4) == 0 && (reinterpret_cast<uintptr_t>(z) & 15) == 0;
-  if (vec_ok) {
-    const float4* z4 = reinterpret_cast<const float4*>(z);
-    for (int q = tid; q < V / 4; q += blockDim.x) {
-      const float4 c = __ldg(z4 + q);
-      argmax_merge(bv, bi, c.x, 4 * q);
-      argmax_merge(bv, bi, c.y, 4 * q + 1);
-      argmax_merge(bv, bi, c.z, 4 * q + 2);
-      argmax_merge(bv, bi, c.w, 4 * q + 3);
-    }
-  } else {
-    for (int v = tid; v < V; v += blockDim.x) argmax_merge(bv, bi, __ldg(z + v), v);
-  }
+// Block-wide reductions through a 32-entry shared array (all threads call).
+__device__ __forceinline__ void block_argmax(float& v, int& i, float* sv, int* si) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1)
-    argmax_merge(bv, bi, __shfl_xor_sync(0xffffffffu, bv, o), __shfl_xor_sync(0xffffffffu, bi, o));
+    argmax_merge(v, i, __shfl_xor_sync(0xffffffffu, v, o), __shfl_xor_sync(0xffffffffu, i, o));
   if (lane == 0) {
-    red_v[warp] = bv;
-    red_i[warp] = bi;
+    sv[warp] = v;
+    si[warp] = i;
   }
   __syncthreads();
-  if (warp == 0) {
-    bv = lane < (int)(blockDim.x / 32) ? red_v[lane] : -FLT_MAX;
-    bi = lane < (int)(blockDim.x / 32) ? red_i[lane] : 0x7fffffff;
+  v = sv[lane];
+  i = si[lane];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-      argmax_merge(bv, bi, __shfl_xor_sync(0xffffffffu, bv, o), __shfl_xor_sync(0xffffffffu, bi, o));
-    if (lane == 0) {
-      red_v[0] = bv;
-      red_i[0] = bi;
-    }
-  }
+  for (int o = 16; o > 0; o >>= 1)
+    argmax_merge(v, i, __shfl_xor_sync(0xffffffffu, v, o), __shfl_xor_sync(0xffffffffu, i, o));
   __syncthreads();
-  const float zmax = red_v[0];
-  const int amax = red_i[0];
-  if (!typical) {
-    if (tid == 0) stats[row] = NodeStat{amax, 0.f, 0.f, 0.f};
-    return;
-  }
-  // m = max(z / T) = max(z) / T for T > 0 (division is monotone).
-  const float m = zmax / temperature;
-  float s = 0.f, e = 0.f;
-  for (int v = tid; v < V; v += blockDim.x) {
-    const float y = __ldg(z + v) / temperature - m;
-    const float p = expf(y);
-    s += p;
-    e = fmaf(p, y, e);
-  }
+}
+
+__device__ __forceinline__ void block_sum2(float& a, float& b, float* sa, float* sb) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    s += __shfl_xor_sync(0xffffffffu, s, o);
-    e += __shfl_xor_sync(0xffffffffu, e, o);
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
   }
-  __syncthreads();
   if (lane == 0) {
-    red_s[warp] = s;
-    red_e[warp] = e;
+    sa[warp] = a;
+    sb[warp] = b;
   }
   __syncthreads();
-  if (tid == 0) {
-    float S = 0.f, Es = 0.f;
-    for (int w = 0; w < (int)(blockDim.x / 32); ++w) {
-      S += red_s[w];
-      Es += red_e[w];
+  a = 0.f;
+  b = 0.f;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < kThreads / 32; ++w) {   // fixed order
+      a += sa[w];
+      b += sb[w];
     }
-    const float H = logf(S) - Es / S;
-    const float thr = fminf(eps, alpha * expf(-H));
-    stats[row] = NodeStat{amax, m, S, thr};
+  __syncthreads();
+}
+
+// Loads logits c0 + 4 (tid + i kThreads) + j of row z into c[i] (-inf past
+// V): 16-byte loads when the row allows them, else one value at a time.
+__device__ __forceinline__ void load_chunk(const float* z, int V, int c0, bool vec, float4 (&c)[kVecPerThread]) {
+#pragma unroll
+  for (int i = 0; i < kVecPerThread; ++i) {
+    const int v0 = c0 + 4 * (threadIdx.x + i * kThreads);
+    if (vec) {
+      c[i] = v0 < V ? __ldg(reinterpret_cast<const float4*>(z + v0))
+                    : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    } else {
+      c[i].x = v0 < V ? __ldg(z + v0) : -INFINITY;
+      c[i].y = v0 + 1 < V ? __ldg(z + v0 + 1) : -INFINITY;
+      c[i].z = v0 + 2 < V ? __ldg(z + v0 + 2) : -INFINITY;
+      c[i].w = v0 + 3 < V ? __ldg(z + v0 + 3) : -INFINITY;
+    }
   }
 }
 
-__global__ void paths_kernel(const TreeDev t, int V, const float* __restrict__ logits,
-                             const int32_t* __restrict__ candidates, const NodeStat* __restrict__ stats,
-                             int typical, float temperature, int32_t* __restrict__ best_path,
-                             int32_t* __restrict__ accept_len, int32_t* __restrict__ accepted_tokens,
-                             int32_t* __restrict__ next_token, int* status) {
-  const int b = blockIdx.x;
-  const int p = threadIdx.x;
+__global__ void __launch_bounds__(kThreads) posterior_kernel(
+    const TreeDev t, int V, const float* __restrict__ logits, const int32_t* __restrict__ candidates, int typical,
+    float temperature, float eps, float alpha, NodeStat* stats, unsigned* counters, int32_t* __restrict__ best_path,
+    int32_t* __restrict__ accept_len, int32_t* __restrict__ accepted_tokens, int32_t* __restrict__ next_token,
+    int* status) {
+  __shared__ float red_v[32], red_s[32];
+  __shared__ int red_i[32];
+  __shared__ int s_last;
+  const int row = blockIdx.x;           // b * T + node
+  const int b = row / t.T;
+  const float* z = logits + static_cast<size_t>(row) * V;
+  const int tid = threadIdx.x;
+
+  // ---- node statistics
+  const bool vec = (V % 4) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0;
+  float4 c[kVecPerThread];
+  float bv = -INFINITY;
+  int bi = 0x7fffffff;
+  const bool one_chunk = V <= kChunk;
+  for (int c0 = 0; c0 < V; c0 += kChunk) {
+    load_chunk(z, V, c0, vec, c);
+#pragma unroll
+    for (int i = 0; i < kVecPerThread; ++i) {
+      const int v0 = c0 + 4 * (tid + i * kThreads);
+      argmax_merge(bv, bi, c[i].x, v0);
+      argmax_merge(bv, bi, c[i].y, v0 + 1);
+      argmax_merge(bv, bi, c[i].z, v0 + 2);
+      argmax_merge(bv, bi, c[i].w, v0 + 3);
+    }
+  }
+  block_argmax(bv, bi, red_v, red_i);
+  if (!typical) {
+    if (tid == 0) stats[row] = NodeStat{bi, 0.f, 0.f, 0.f};
+  } else {
+    // m = max(z / T) = max(z) / T for T > 0 (division is monotone).
+    const float m = bv / temperature;
+    float s = 0.f, e = 0.f;
+    for (int c0 = 0; c0 < V; c0 += kChunk) {
+      if (!one_chunk) load_chunk(z, V, c0, vec, c);
+#pragma unroll
+      for (int i = 0; i < kVecPerThread; ++i) {
+        const float zz[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (zz[j] != -INFINITY) {   // past the row's end (or a zero-probability logit)
+            const float y = zz[j] / temperature - m;
+            const float pp = expf(y);
+            s += pp;
+            e = fmaf(pp, y, e);
+          }
+        }
+      }
+    }
+    block_sum2(s, e, red_s, red_v);
+    if (tid == 0) {
+      const float H = logf(s) - e / s;
+      const float thr = fminf(eps, alpha * expf(-H));
+      stats[row] = NodeStat{bi, m, s, thr};
+    }
+  }
+
+  // ---- the last node of sequence b to finish evaluates the paths
+  if (tid == 0) {
+    __threadfence();
+    const unsigned done = atom_add_acq_rel_gpu(&counters[b], 1u);
+    s_last = done == static_cast<unsigned>(t.T - 1);
+    if (s_last) counters[b] = 0u;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
   const int D1 = t.D + 1;
-  __shared__ int red_a[32], red_p[32];
-  __shared__ int s_best, s_a;
+  const int p = tid;
   int acc = -1;  // threads without a path never win
   if (p < t.P) {
     acc = 0;
@@ -143,58 +184,39 @@ __global__ void paths_kernel(const TreeDev t, int V, const float* __restrict__ l
         set_device_status(status, MEDUSA_ERR_DEVICE_CHECK, kDetailPosteriorArgs);
         break;
       }
-      const NodeStat st = stats[b * t.T + par];
+      const NodeStat* sp = stats + b * t.T + par;
       bool ok;
       if (!typical) {
-        ok = tok == st.argmax;
+        ok = tok == __ldcg(&sp->argmax);
       } else {
-        const float y = logits[(static_cast<size_t>(b) * t.T + par) * V + tok] / temperature - st.m;
-        ok = expf(y) / st.S > st.thr;
+        const float y = logits[(static_cast<size_t>(b) * t.T + par) * V + tok] / temperature - __ldcg(&sp->m);
+        ok = expf(y) / __ldcg(&sp->S) > __ldcg(&sp->thr);
       }
       if (!ok) break;
       ++acc;
     }
   }
   // (max acc, then lowest p)
-  int ba = acc, bp = p;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const int oa = __shfl_xor_sync(0xffffffffu, ba, o);
-    const int op = __shfl_xor_sync(0xffffffffu, bp, o);
-    if (oa > ba || (oa == ba && op < bp)) {
-      ba = oa;
-      bp = op;
-    }
-  }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
-  if (lane == 0) {
-    red_a[warp] = ba;
-    red_p[warp] = bp;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < nw; ++w)
-      if (red_a[w] > ba || (red_a[w] == ba && red_p[w] < bp)) {
-        ba = red_a[w];
-        bp = red_p[w];
-      }
-    s_best = bp;
-    s_a = ba;
+  float av = static_cast<float>(acc);
+  int ap = p;
+  // ranks_before orders by larger value, then lower index: exactly (max acc, lowest p).
+  block_argmax(av, ap, red_v, red_i);
+  const int ba = static_cast<int>(av), bp = ap;
+  if (tid == 0) {
     best_path[b] = bp;
     accept_len[b] = ba;
     const int last = t.retrieve[bp * D1 + ba];
-    next_token[b] = stats[b * t.T + last].argmax;
+    next_token[b] = __ldcg(&stats[b * t.T + last].argmax);
   }
-  __syncthreads();
-  for (int j = threadIdx.x; j < D1; j += blockDim.x)
-    accepted_tokens[b * D1 + j] =
-        j <= s_a ? candidates[(static_cast<size_t>(b) * t.P + s_best) * D1 + j] : -1;
+  for (int j = tid; j < D1; j += blockDim.x)
+    accepted_tokens[b * D1 + j] = j <= ba ? candidates[(static_cast<size_t>(b) * t.P + bp) * D1 + j] : -1;
 }
 
 }  // namespace
 
 size_t posterior_workspace_bytes(const TreeDev& t, int B) {
-  return align_up(static_cast<size_t>(B) * t.T * sizeof(NodeStat), 256);
+  return align_up(static_cast<size_t>(B) * t.T * sizeof(NodeStat), 256) +
+         align_up(static_cast<size_t>(B) * sizeof(unsigned), 256);
 }
 
 medusa_status_t launch_posterior(const TreeDev& t, int B, int V, const float* logits,
@@ -202,17 +224,16 @@ medusa_status_t launch_posterior(const TreeDev& t, int B, int V, const float* lo
                                  float eps, float alpha, int32_t* best_path, int32_t* accept_len,
                                  int32_t* accepted_tokens, int32_t* next_token, void* ws,
                                  cudaStream_t stream) {
+  if (t.P > kThreads) return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_evaluate_posterior: more than 1024 paths");
   NodeStat* stats = static_cast<NodeStat*>(ws);
+  unsigned* counters = reinterpret_cast<unsigned*>(static_cast<unsigned char*>(ws) +
+                                                   align_up(static_cast<size_t>(B) * t.T * sizeof(NodeStat), 256));
   const int typical = mode == MEDUSA_TYPICAL ? 1 : 0;
-  node_stats_kernel<<<B * t.T, kStatThreads, 0, stream>>>(logits, V, typical, 0.f, temperature, eps, alpha,
-                                                          stats);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail("medusa_evaluate_posterior: stats launch", e);
-  const int threads = ((t.P + 31) / 32) * 32;
-  paths_kernel<<<B, threads, 0, stream>>>(t, V, logits, candidates, stats, typical, temperature, best_path,
-                                          accept_len, accepted_tokens, next_token, device_status_ptr());
-  e = cudaGetLastError();
-  return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_evaluate_posterior: paths launch", e);
+  posterior_kernel<<<B * t.T, kThreads, 0, stream>>>(t, V, logits, candidates, typical, temperature, eps, alpha,
+                                                     stats, counters, best_path, accept_len, accepted_tokens,
+                                                     next_token, device_status_ptr());
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_evaluate_posterior: launch", e);
 }
 
 }  // namespace medusa

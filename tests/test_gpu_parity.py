@@ -196,6 +196,16 @@ def test_posterior(mb, name, mode):
     _posterior_case(mb, w, mode)
 
 
+@pytest.mark.parametrize("V", [40001, 65540])
+@pytest.mark.parametrize("mode", ["greedy", "typical"])
+def test_posterior_vocab_shapes(mb, V, mode):
+    # V = 40001: rows not 16-byte aligned (one logit per load), more than one
+    # 32768-logit chunk per row; V = 65540: 16-byte loads over three chunks.
+    from synth.workloads import shrink
+    w = shrink(SMALL["b3_small"], name=f"b3_V{V}", V=V, modes=(mode,))
+    _posterior_case(mb, w, mode)
+
+
 @pytest.mark.parametrize("agreement,expect", [(0.0, "none"), (1.0, "leaf")])
 def test_posterior_extremes(mb, agreement, expect):
     ref = _posterior_case(mb, SMALL["v13b_small"], "greedy", agreement)
