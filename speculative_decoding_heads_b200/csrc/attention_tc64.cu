@@ -56,6 +56,7 @@ __device__ __forceinline__ uint32_t col_p(int buf) { return 128u + 64u * buf; } 
 __device__ __forceinline__ uint32_t col_o(int buf) { return 256u + 128u * buf; }  // 128 fp32 columns
 constexpr uint32_t kLaneHalf = 16u << 16;      // TMEM address offset of lane 16
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kLenTab = 160;                   // prefix lengths of a CTA's first slices, in shared memory
 
 struct Bars {
   uint64_t q_full[2], q_empty[2];
@@ -66,6 +67,7 @@ struct Bars {
   uint32_t tmem_base;
   int abort;
   float lsum[2][kRows];              // row sums handed to the epilogue warps
+  int lens[kLenTab];                 // lens[k]: prefix length of this CTA's slice k
 };
 
 // Shared memory (offsets from a 1024-byte aligned base).
@@ -73,7 +75,7 @@ constexpr int kOffQ = 0;                               // 2 x 16 KB
 constexpr int kOffK = 2 * kQBuf;                       // 3 x 32 KB
 constexpr int kOffV = kOffK + kStages * kTile;         // 3 x 32 KB
 constexpr int kOffBars = kOffV + kStages * kTile;
-constexpr int kBarsBytes = 1024;
+constexpr int kBarsBytes = 1664;
 constexpr int kSmemBytes = kOffBars + kBarsBytes + 1024;
 static_assert(sizeof(Bars) <= kBarsBytes, "barrier block too large");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -93,22 +95,24 @@ struct Params {
 };
 
 // Slice kk of this CTA; steps = 0 when it does not exist or fails its check.
-__device__ __forceinline__ Slice slice_info(int kk, const Params& p) {
+// The prefix length comes from the shared table for the first kLenTab
+// slices (no global load on any role's critical path at a slice boundary).
+__device__ __forceinline__ Slice slice_info(int kk, const Params& p, const int* lens) {
   Slice s{};
   s.slice = blockIdx.x + kk * gridDim.x;
   if (s.slice >= p.total) return s;
   s.e = s.slice % p.H;
   s.lb = s.slice / p.H;
-  s.L = p.seq_lens[s.lb % p.B];
+  s.L = kk < kLenTab ? lens[kk] : p.seq_lens[s.lb % p.B];
   s.n = s.L + p.t.T;
   s.steps = (s.L >= 0 && s.n <= p.Lcap) ? (s.n + kStep - 1) / kStep : 0;
   return s;
 }
 
 // First slice at or after kk that passes its check (kk is advanced to it).
-__device__ __forceinline__ Slice seek(int& kk, const Params& p) {
-  Slice s = slice_info(kk, p);
-  while (s.slice < p.total && s.steps == 0) s = slice_info(++kk, p);
+__device__ __forceinline__ Slice seek(int& kk, const Params& p, const int* lens) {
+  Slice s = slice_info(kk, p, lens);
+  while (s.slice < p.total && s.steps == 0) s = slice_info(++kk, p, lens);
   return s;
 }
 
@@ -141,7 +145,7 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
   tc::prefetch_tensormap(k_map);
   tc::prefetch_tensormap(v_map);
   int kkq = 0, kkk = 0, kkv = 0;
-  Slice sq = seek(kkq, p), sk = seek(kkk, p), sv = seek(kkv, p);
+  Slice sq = seek(kkq, p, bar->lens), sk = seek(kkk, p, bar->lens), sv = seek(kkv, p, bar->lens);
   int nq = 0, gk = 0, gv = 0, tk = 0, tv = 0;     // loads issued; step within slice
   uint64_t last = globaltimer_ns();
   while ((sq.slice < p.total || sk.slice < p.total || sv.slice < p.total) && !bar->abort) {
@@ -154,7 +158,7 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
       tc::tma_load_4d(qd + kQHalf, q_map, 64, sq.e, 0, sq.lb, fb);
       ++nq;
       ++kkq;
-      sq = seek(kkq, p);
+      sq = seek(kkq, p, bar->lens);
       progressed = true;
     }
     for (int which = 0; which < 2; ++which) {
@@ -180,7 +184,7 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
       if (++t == s.steps) {
         t = 0;
         ++kk;
-        s = seek(kk, p);
+        s = seek(kk, p, bar->lens);
       }
       progressed = true;
     }
@@ -221,7 +225,7 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
   constexpr uint32_t idS = tc::idesc_bf16_f32(64, kStep, 0);
   constexpr uint32_t idO = tc::idesc_bf16_f32(128, kHd, 1);
   int kks = 0, kkp = 0;
-  Slice ss = seek(kks, p), sp = seek(kkp, p);
+  Slice ss = seek(kks, p, bar->lens), sp = seek(kkp, p, bar->lens);
   int gs = 0, ts = 0, ks = 0;     // S cursor: global step, step in slice, slice count
   int gp = 0, tp = 0, kp = 0;     // P V cursor
   uint64_t last = globaltimer_ns();
@@ -248,7 +252,7 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
         ts = 0;
         ++ks;
         ++kks;
-        ss = seek(kks, p);
+        ss = seek(kks, p, bar->lens);
       }
       progressed = true;
     }
@@ -274,7 +278,7 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
         tp = 0;
         ++kp;
         ++kkp;
-        sp = seek(kkp, p);
+        sp = seek(kkp, p, bar->lens);
       }
       progressed = true;
     }
@@ -303,7 +307,7 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
   const uint64_t anc = r < T ? p.t.anc[r * p.t.W] : 0ull;   // T <= 64: one word per row
   int g = 0, k = 0;
   for (int kk = 0;; ++kk) {
-    const Slice s = slice_info(kk, p);
+    const Slice s = slice_info(kk, p, bar->lens);
     if (s.slice >= p.total) break;
     if (s.steps == 0) {
       if (lane == 0 && q == 0) set_device_status(p.status, MEDUSA_ERR_DEVICE_CHECK, kDetailAttnSeqLen);
@@ -429,7 +433,7 @@ __device__ void run_epilogue(const Params& p, uint32_t tmem, Bars* bar, int warp
   const uint32_t la = static_cast<uint32_t>(32 * q) << 16;
   int k = 0;
   for (int kk = 0;; ++kk) {
-    const Slice s = seek(kk, p);
+    const Slice s = seek(kk, p, bar->lens);
     if (s.slice >= p.total) break;
     if (!wait_bar(&bar->l_ready[k & 1], (k >> 1) & 1, bar, p.status)) return;
     if (!wait_bar(&bar->o_full[k & 1], (k >> 1) & 1, bar, p.status)) return;
@@ -487,6 +491,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     bar->abort = 0;
     fence_barrier_init();
+  }
+  for (int k = tid; k < kLenTab; k += blockDim.x) {
+    const int sl = blockIdx.x + k * gridDim.x;
+    bar->lens[k] = sl < p.total ? p.seq_lens[(sl / p.H) % p.B] : 0;
   }
   if (warp == 1) {
     tc::tmem_alloc(&bar->tmem_base, kTmemCols);
