@@ -135,6 +135,22 @@ def test_tree_attention(mb, dev, name):
     _attention_case(mb, dev, SMALL[name])
 
 
+@pytest.mark.parametrize("shape", [(2, 160, 200, 1), (1, 37, 131, 9)])
+def test_tree_attention_many_slices(mb, dev, shape):
+    # More (layer, sequence, head) slices than SMs: every persistent CTA walks
+    # several slices (Q, K/V, S, P and O buffers change hands between them);
+    # the second shape has ragged prefixes and slices split unevenly.
+    from synth.workloads import shrink
+    layers, H, prefix, B = shape
+    base = SMALL["v7b_small"] if B == 1 else SMALL["v13b_small"]
+    kw = dict(layers=layers, H=H, B=B)
+    if B == 1:
+        kw["prefix"] = prefix
+    else:
+        kw["prefix_range"] = (prefix // 4, prefix)
+    _attention_case(mb, dev, shrink(base, **kw))
+
+
 @pytest.mark.parametrize("variant", ["T200_two_row_groups", "hd64_bf16_generic", "hd256_f32", "chain_L0",
                                      "exact_capacity"])
 def test_tree_attention_edges(mb, dev, variant):
