@@ -5,9 +5,9 @@
 // j is i or one of its ancestors; the tree's own K/V already sit at rows
 // L..L+T-1 of the cache.
 //
-// bf16 with hd = 128 runs on the tcgen05 tensor cores: a persistent kernel
-// for trees of up to 64 tokens (attention_tc64.cu) and a CTA-per-slice
-// kernel for larger trees (attention_tc.cu).  Every other dtype / head size
+// bf16 with hd = 128 runs on the tcgen05 tensor cores in one persistent
+// kernel (attention_tc64.cu; one pass over a slice's K/V per 64 tree
+// tokens).  Every other dtype / head size
 // runs tree_attn_generic: one CTA per (slice, node), scores in shared memory,
 // plain fp32 arithmetic.  The output is fp32 on every path.
 #include <cfloat>
@@ -122,11 +122,8 @@ medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int
   int* status = device_status_ptr();
   cudaError_t e;
   if (dtype == MEDUSA_BF16 && hd == kHd) {
-    if (t.T <= 64)
-      return launch_attention_tc64(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, scale * kLog2e,
-                                   static_cast<float*>(out), status, stream);
-    return launch_attention_tc(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, scale * kLog2e,
-                               static_cast<float*>(out), status, stream);
+    return launch_attention_tc64(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, scale * kLog2e,
+                                 static_cast<float*>(out), status, stream);
   }
   {
     const size_t smem = static_cast<size_t>(hd + Lcap) * sizeof(float);

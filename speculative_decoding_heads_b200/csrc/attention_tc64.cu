@@ -1,14 +1,17 @@
-// S5 for trees of up to 64 tokens (bf16, hd = 128): a persistent tcgen05
-// kernel that streams every (layer, sequence, head) slice of K/V through
-// shared memory exactly once and keeps the memory pipeline full across
-// slice boundaries.
+// S5 (bf16, hd = 128): a persistent tcgen05 kernel that streams the K/V of
+// every (layer, sequence, head) slice through shared memory and keeps the
+// memory pipeline full across slice boundaries.  A work item is one slice and
+// one group of 64 tree tokens (query rows); trees of up to 64 tokens have one
+// group, so every K/V byte is read once; larger trees (up to 256 tokens)
+// stream a slice's K/V once per group.
 //
 // The mask is that of "Medusa — 让大模型自己同时猜好几个 token" (核心要点:
 // the candidate tree is verified in one forward under a tree mask; 实践案例
 // case 3: a node sees the cached prefix, its ancestors and itself).
 //
-// Layout of the work.  One CTA per SM walks the slices s = cta, cta + G, ...
-// Each slice is cut into steps of 128 keys.  K and V tiles (32 KB each, two
+// Layout of the work.  One CTA per SM walks the items w = cta, cta + grid, ...
+// (item w: slice w / groups, row group w % groups).  Each item is cut into
+// steps of 128 keys.  K and V tiles (32 KB each, two
 // 64-dim halves in 128-byte swizzle) arrive by TMA (no multicast) into two
 // three-stage rings: a K stage is released as soon as S of its step is done,
 // a V stage once P V of its step is done.  The 64 query rows of a slice sit
@@ -82,11 +85,13 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Slice {
   int slice, lb, e, L, n, steps;
+  int item, grp;   // work item index; query rows 64 grp .. 64 grp + 63
 };
 
 struct Params {
   TreeDev t;
-  int B, H, Lcap, total;
+  int B, H, Lcap, total;   // total: work items = slices x groups
+  int groups;              // ceil(T / 64)
   const int32_t* seq_lens;
   float scale_log2;
   float* out;
@@ -94,13 +99,19 @@ struct Params {
   int kv_one_box;   // 1: one 32 KB TMA box per tile (4-D map), 0: two 16 KB boxes
 };
 
-// Slice kk of this CTA; steps = 0 when it does not exist or fails its check.
-// The prefix length comes from the shared table for the first kLenTab
-// slices (no global load on any role's critical path at a slice boundary).
+// Work item kk of this CTA; steps = 0 when it does not exist or fails its
+// check (slice >= total marks the end).  The prefix length comes from the
+// shared table for the first kLenTab items (no global load on any role's
+// critical path at an item boundary).
 __device__ __forceinline__ Slice slice_info(int kk, const Params& p, const int* lens) {
   Slice s{};
-  s.slice = blockIdx.x + kk * gridDim.x;
-  if (s.slice >= p.total) return s;
+  s.item = blockIdx.x + kk * gridDim.x;
+  if (s.item >= p.total) {
+    s.slice = p.total;
+    return s;
+  }
+  s.slice = s.item / p.groups;
+  s.grp = s.item - s.slice * p.groups;
   s.e = s.slice % p.H;
   s.lb = s.slice / p.H;
   s.L = kk < kLenTab ? lens[kk] : p.seq_lens[s.lb % p.B];
@@ -154,8 +165,8 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
       unsigned char* qd = smem + kOffQ + (nq & 1) * kQBuf;
       uint64_t* fb = &bar->q_full[nq & 1];
       mbar_arrive_expect_tx(fb, kQBuf);
-      tc::tma_load_4d(qd, q_map, 0, sq.e, 0, sq.lb, fb);
-      tc::tma_load_4d(qd + kQHalf, q_map, 64, sq.e, 0, sq.lb, fb);
+      tc::tma_load_4d(qd, q_map, 0, sq.e, kRows * sq.grp, sq.lb, fb);
+      tc::tma_load_4d(qd + kQHalf, q_map, 64, sq.e, kRows * sq.grp, sq.lb, fb);
       ++nq;
       ++kkq;
       sq = seek(kkq, p, bar->lens);
@@ -295,16 +306,24 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
   }
 }
 
+// Bits o .. o + 63 (o >= 0) of a row of the ancestor mask held in four
+// words; zero past the last word.
+__device__ __forceinline__ uint64_t anc_window(const uint64_t (&a)[4], int o) {
+  if (o >= 256) return 0ull;
+  const int wi = o >> 6, sh = o & 63;
+  const uint64_t w0 = wi == 0 ? a[0] : wi == 1 ? a[1] : wi == 2 ? a[2] : a[3];
+  const uint64_t w1 = wi == 0 ? a[1] : wi == 1 ? a[2] : wi == 2 ? a[3] : 0ull;
+  return sh == 0 ? w0 : (w0 >> sh) | (w1 << (64 - sh));
+}
+
 // ---- softmax (warps 4-7) ------------------------------------------------------
 // Online softmax in the log2 domain with a lazy reference: the running
 // maximum moves (and O is rescaled) only when a step's maximum exceeds it by
 // more than 2^8, so P stays below 2^8 and O is rarely touched.
 __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem, Bars* bar, int warp, int lane) {
   const int q = warp & 3, h = lane >> 4, i = lane & 15;
-  const int r = 16 * q + i;                        // query row (tree token)
   const int T = p.t.T;
   const uint32_t la = static_cast<uint32_t>(32 * q) << 16;
-  const uint64_t anc = r < T ? p.t.anc[r * p.t.W] : 0ull;   // T <= 64: one word per row
   int g = 0, k = 0;
   for (int kk = 0;; ++kk) {
     const Slice s = slice_info(kk, p, bar->lens);
@@ -313,6 +332,14 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
       if (lane == 0 && q == 0) set_device_status(p.status, MEDUSA_ERR_DEVICE_CHECK, kDetailAttnSeqLen);
       continue;
     }
+    // This thread's tree token (query row) in the item's row group and its
+    // ancestor mask (up to four words; loaded now, first used at the item's
+    // last steps).
+    const int r = kRows * s.grp + 16 * q + i;
+    uint64_t anc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int wd = 0; wd < 4; ++wd)
+      if (r < T && wd < p.t.W) anc[wd] = p.t.anc[r * p.t.W + wd];
     float mref = -INFINITY, lsum = 0.f;
     for (int t = 0; t < s.steps; ++t, ++g) {
       if (!wait_bar(&bar->s_full[g & 1], (g >> 1) & 1, bar, p.status)) return;
@@ -333,7 +360,7 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
         // the tree tokens that are ancestors of (or equal to) row r.
         const int d = s.L - key0;                    // prefix keys in the window (< 64)
         uint64_t m = d > 0 ? (1ull << d) - 1ull : 0ull;
-        m |= d >= 0 ? (anc << d) : (d > -64 ? (anc >> -d) : 0ull);
+        m |= d >= 0 ? (anc[0] << d) : anc_window(anc, -d);
         const uint32_t mlo = static_cast<uint32_t>(m), mhi = static_cast<uint32_t>(m >> 32);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -416,7 +443,7 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
         // slice two back (same buffer).
         if (k >= 2 && !wait_bar(&bar->o_free[k & 1], ((k >> 1) - 1) & 1, bar, p.status)) return;
         const float total = lsum + __shfl_xor_sync(0xffffffffu, lsum, 16);
-        if (h == 0) bar->lsum[k & 1][r] = total;
+        if (h == 0) bar->lsum[k & 1][16 * q + i] = total;
         tc::mbar_arrive(&bar->l_ready[k & 1]);
       }
     }
@@ -428,7 +455,6 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
 // out[query] = (O(high-part lanes) + O(remainder lanes)) / row sum, in fp32.
 __device__ void run_epilogue(const Params& p, uint32_t tmem, Bars* bar, int warp, int lane) {
   const int q = warp & 3, h = lane >> 4, i = lane & 15;
-  const int r = 16 * q + i;
   const int T = p.t.T;
   const uint32_t la = static_cast<uint32_t>(32 * q) << 16;
   int k = 0;
@@ -438,7 +464,8 @@ __device__ void run_epilogue(const Params& p, uint32_t tmem, Bars* bar, int warp
     if (!wait_bar(&bar->l_ready[k & 1], (k >> 1) & 1, bar, p.status)) return;
     if (!wait_bar(&bar->o_full[k & 1], (k >> 1) & 1, bar, p.status)) return;
     tc::fence_after_sync();
-    const float inv = 1.f / bar->lsum[k & 1][r];
+    const int r = kRows * s.grp + 16 * q + i;   // tree token
+    const float inv = 1.f / bar->lsum[k & 1][16 * q + i];
     const uint32_t oa = tmem + la + col_o(k & 1);
     float* orow = p.out + ((static_cast<size_t>(s.lb) * T + r) * p.H + s.e) * kHd + 64 * h;
 #pragma unroll 1
@@ -493,8 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   for (int k = tid; k < kLenTab; k += blockDim.x) {
-    const int sl = blockIdx.x + k * gridDim.x;
-    bar->lens[k] = sl < p.total ? p.seq_lens[(sl / p.H) % p.B] : 0;
+    const int item = blockIdx.x + k * gridDim.x;
+    bar->lens[k] = item < p.total ? p.seq_lens[(item / p.groups / p.H) % p.B] : 0;
   }
   if (warp == 1) {
     tc::tmem_alloc(&bar->tmem_base, kTmemCols);
@@ -524,8 +551,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-// Tensor maps: Q as [layers*B][T][H][128] (box 64 dims x 64 rows, rows past
-// T read as zero), K and V as [slices][Lcap][128].  For K/V a 4-D view
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+void* tensor_map_encoder() {
+  static void* fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = ptr;
+  }
+  return fn;
+}
+
+// Tensor maps: Q as [layers*B][T][H][128] (box 64 dims x 64 rows starting at
+// row 64 x group, rows past T read as zero), K and V as [slices][Lcap][128].  For K/V a 4-D view
 // {64 dims, rows, 2 halves, slices} loads a whole 128-key tile (both 64-dim
 // halves, 32 KB) with one TMA instruction; if the driver rejects that view
 // the kernel falls back to two 16 KB boxes per tile.
@@ -534,8 +574,11 @@ medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H
                                       float scale_log2, float* out, int* status, cudaStream_t stream) {
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!enc) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: cuTensorMapEncodeTiled unavailable");
-  if (t.T > kRows || t.W != 1) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: more than 64 tree tokens");
+  if (t.T > 4 * kRows || t.W > 4) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: more than 256 tree tokens");
   const long long slices = static_cast<long long>(layers) * B * H;
+  const int groups = (t.T + kRows - 1) / kRows;
+  const long long items = slices * groups;
+  if (items >= (1ll << 31)) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: too many slices");
   CUtensorMap qm, km, vm;
   {
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHd), static_cast<cuuint64_t>(H),
@@ -582,13 +625,14 @@ medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H
   prm.B = B;
   prm.H = H;
   prm.Lcap = Lcap;
-  prm.total = static_cast<int>(slices);
+  prm.total = static_cast<int>(items);
+  prm.groups = groups;
   prm.seq_lens = seq_lens;
   prm.scale_log2 = scale_log2;
   prm.out = out;
   prm.status = status;
   prm.kv_one_box = one_box;
-  const int grid = static_cast<int>(slices < sm_count() ? slices : sm_count());
+  const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
   cudaError_t e = cudaFuncSetAttribute(tree_attn_tc64, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e == cudaSuccess) {
     tree_attn_tc64<<<grid, kThreads, kSmemBytes, stream>>>(qm, km, vm, prm);

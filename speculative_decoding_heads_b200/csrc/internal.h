@@ -77,9 +77,6 @@ medusa_status_t launch_accept_kv(const TreeDev& t, int layers, int B, int H, int
 // cuTensorMapEncodeTiled (PFN_cuTensorMapEncodeTiled_v12000), or null.
 void* tensor_map_encoder();
 
-medusa_status_t launch_attention_tc(const TreeDev& t, int layers, int B, int H, const void* q, const void* k_cache,
-                                    const void* v_cache, int Lcap, const int32_t* seq_lens, float scale_log2,
-                                    float* out, int* status, cudaStream_t stream);
 medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H, const void* q,
                                       const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
                                       float scale_log2, float* out, int* status, cudaStream_t stream);
