@@ -190,29 +190,49 @@ __device__ __forceinline__ float to_f32<uint16_t>(uint16_t x) {
   return __uint_as_float(static_cast<uint32_t>(x) << 16);
 }
 
-// acc[b] += dot(16-byte weight vector w, x[b][0..E)) for b < NB.
+// Two fp32 values in one 64-bit register pair, and the packed fp32 FMA of
+// sm_100 (two independent IEEE fmas per instruction).
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void fma_f2(uint64_t& acc, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ float sum_f2(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo + hi;
+}
+
+// acc[b] += dot(16-byte weight vector w, x[b]) for b < NB, where x[b] holds
+// the matching E activations as E/2 (even, odd) pairs and acc[b] keeps an
+// even and an odd partial sum.
 template <typename TW, int NB, int VPT>
-__device__ __forceinline__ void dot_vec(const uint4 w, const float (&x)[NB * VPT][Elem<TW>::E], int j,
-                                        float* acc) {
+__device__ __forceinline__ void dot_vec(const uint4 w, const uint64_t (&xp)[NB * VPT][Elem<TW>::E / 2], int j,
+                                        uint64_t* acc) {
   constexpr int E = Elem<TW>::E;
-  float f[E];
+  uint64_t wp[E / 2];
   if constexpr (E == 8) {
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = bf16lo(ww[i]);
-      f[2 * i + 1] = bf16hi(ww[i]);
-    }
+    for (int i = 0; i < 4; ++i) wp[i] = pack_f2(bf16lo(ww[i]), bf16hi(ww[i]));
   } else {
-    f[0] = __uint_as_float(w.x);
-    f[1] = __uint_as_float(w.y);
-    f[2] = __uint_as_float(w.z);
-    f[3] = __uint_as_float(w.w);
+    wp[0] = pack_f2(__uint_as_float(w.x), __uint_as_float(w.y));
+    wp[1] = pack_f2(__uint_as_float(w.z), __uint_as_float(w.w));
   }
 #pragma unroll
   for (int b = 0; b < NB; ++b)
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[b] = fmaf(f[e], x[b * VPT + j][e], acc[b]);
+    for (int i = 0; i < E / 2; ++i) fma_f2(acc[b], wp[i], xp[b * VPT + j][i]);
+}
+
+// Packs E activations into E/2 (even, odd) pairs.
+template <int E>
+__device__ __forceinline__ void pack_x(const float* f, uint64_t* xp) {
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) xp[i] = pack_f2(f[2 * i], f[2 * i + 1]);
 }
 
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
@@ -395,18 +415,20 @@ __global__ void __launch_bounds__(kMaxThreads, 1) heads_kernel(const HeadsArgs a
     const int cw = warp - kRoleWarps;
     // x[b*VPT+j][e]: h (phase 1) or u of the current head (phase 2), for the
     // thread's column vectors ct + j*NT.
-    float x[NB * VPT][E];
+    uint64_t xp[NB * VPT][E / 2];
 #pragma unroll
     for (int b = 0; b < NB; ++b)
 #pragma unroll
       for (int j = 0; j < VPT; ++j) {
         const int v = ct + j * a.NT;
+        float f[E];
         if (b < a.nb && v < a.nvec) {
-          load_vec<TW>(static_cast<const TW*>(a.h) + static_cast<size_t>(a.b0 + b) * a.d, v, x[b * VPT + j]);
+          load_vec<TW>(static_cast<const TW*>(a.h) + static_cast<size_t>(a.b0 + b) * a.d, v, f);
         } else {
 #pragma unroll
-          for (int e = 0; e < E; ++e) x[b * VPT + j][e] = 0.f;
+          for (int e = 0; e < E; ++e) f[e] = 0.f;
         }
+        pack_x<E>(f, xp[b * VPT + j]);
       }
     Cursor cc;
     cursor_start<R>(cc, a, p1_lo, p1_hi, p2_lo, p2_hi);
@@ -430,8 +452,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1) heads_kernel(const HeadsArgs a
 #pragma unroll
           for (int j = 0; j < VPT; ++j) {
             const int v = ct + j * a.NT;
-            if (b < a.nb && v < a.nvec)
-              load_u_vec(a.u + (static_cast<size_t>(a.b0 + b) * a.K + khead) * a.d, v, E, x[b * VPT + j]);
+            if (b < a.nb && v < a.nvec) {
+              float f[E];
+              load_u_vec(a.u + (static_cast<size_t>(a.b0 + b) * a.K + khead) * a.d, v, E, f);
+              pack_x<E>(f, xp[b * VPT + j]);
+            }
           }
       }
       if (!mbar_wait(&full[slot], static_cast<uint32_t>((s / NS) & 1))) {
@@ -440,22 +465,27 @@ __global__ void __launch_bounds__(kMaxThreads, 1) heads_kernel(const HeadsArgs a
       }
       if (flag[0]) break;
 
+      // Per row: an (even, odd) pair of partial sums per sequence, folded
+      // into one fp32 partial sum once the row is done.
       float acc[RNB];
-#pragma unroll
-      for (int i = 0; i < RNB; ++i) acc[i] = 0.f;
       const unsigned char* st = stages + slot * stage_bytes;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
+        uint64_t acc2[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc2[b] = 0ull;   // (+0.0f, +0.0f)
         if (r < cc.n) {
 #pragma unroll
           for (int j = 0; j < VPT; ++j) {
             const int v = ct + j * a.NT;
             if (v < a.nvec) {
               const uint4 w = *reinterpret_cast<const uint4*>(st + r * row_bytes + static_cast<size_t>(v) * 16);
-              dot_vec<TW, NB, VPT>(w, x, j, acc + r * NB);
+              dot_vec<TW, NB, VPT>(w, xp, j, acc2);
             }
           }
         }
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc[r * NB + b] = sum_f2(acc2[b]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_cta(&empty[slot]);   // this warp is done with the stage's bytes
@@ -488,9 +518,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) heads_kernel(const HeadsArgs a
     // This CTA's u rows are written: count it, wait (bounded) for every CTA,
     // then let the consumers read u.
     auto publish = [&]() {
+      __threadfence();   // every lane's u rows, once
       __syncwarp();
       if (lane == 0) {
-        __threadfence();
         atom_add_release_gpu(&a.counters[0], 1u);
         const uint64_t t0 = globaltimer_ns();
         while (ld_acquire_gpu(&a.counters[0]) < static_cast<unsigned>(G)) {
@@ -533,7 +563,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1) heads_kernel(const HeadsArgs a
         if (live) {
           const int i = cc.row - p1_lo + r;
           a.u[(static_cast<size_t>(a.b0 + b) * a.K + khead) * a.d + local] = pre_h[i * NB + b] + silu(val + pre_b[i]);
-          __threadfence();
         }
         if (cc.row + cc.n >= cc.end) publish();   // the CTA's last W1 stage
       } else {
