@@ -201,6 +201,17 @@ class OracleSample:
         return t_full + t_sample * self.scale_slices
 
 
+def reduce_max(x, world, device):
+    """The largest of a per-rank scalar over all ranks (every rank receives it)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(a, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -319,11 +330,7 @@ def run_ours(a, w):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-    ms = ev0.elapsed_time(ev1) / a.steps
-    if world > 1:
-        tm = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        ms = float(tm.item())
+    ms = reduce_max(ev0.elapsed_time(ev1) / a.steps, world, "cuda")
     clocks = sampler.summary()
     st, det = mb.device_status()
     if st != 0:
@@ -397,11 +404,7 @@ def run_ours(a, w):
             s1.synchronize()
             if i >= a.warmup:
                 e_ms.append(s0.elapsed_time(s1))
-        e_ms_max = statistics.mean(e_ms)
-        if world > 1:
-            tm = torch.tensor([e_ms_max], device="cuda")
-            dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-            e_ms_max = float(tm.item())
+        e_ms_max = reduce_max(statistics.mean(e_ms), world, "cuda")
         e2e = {"value": e_ms_max * 1e3, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ---- CPU baseline (rank 0, N = 1 only) -----------------------------
