@@ -282,7 +282,8 @@ def run_ours(a, w):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
-    launches_per_step = (w.B + 3) // 4 + 1 + 1 + 2 + 2
+    # heads (+ tree build) per group of <= 4 sequences, attention, posterior, accept rows, length update
+    launches_per_step = (w.B + 3) // 4 + 1 + 1 + 2
 
     def step():
         t["seq_lens"].copy_(t["seq_lens0"])

@@ -292,9 +292,13 @@ typedef struct medusa_step_args {
 
 size_t medusa_step_workspace_size(const medusa_step_args_t* args);
 
-/* medusa_heads_topk, medusa_build_tree, medusa_tree_attention,
- * medusa_evaluate_posterior and medusa_accept_kv, in that order, on stream.
- * Capturable in a CUDA graph (no allocation, no synchronisation). */
+/* The computations of medusa_heads_topk, medusa_build_tree,
+ * medusa_tree_attention, medusa_evaluate_posterior and medusa_accept_kv, in
+ * that order, on stream, with the same outputs.  The candidate tree is built
+ * by the heads kernel's last CTA (one launch for S1-S4 per group of up to
+ * four sequences); five launches per step at B <= 4.  Capturable in a CUDA
+ * graph (no allocation, no synchronisation).  Validation errors are returned
+ * before anything is enqueued. */
 medusa_status_t medusa_step(const medusa_step_args_t* args, void* workspace,
                             size_t workspace_bytes, cudaStream_t stream);
 

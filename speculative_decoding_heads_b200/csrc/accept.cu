@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(kThreads) accept_rows_kernel(
     const TreeDev t, int n_slices, int B, int H, int chunks, uint4* __restrict__ k_cache,
     uint4* __restrict__ v_cache, int Lcap, const int32_t* __restrict__ seq_lens,
     const int32_t* __restrict__ best_path, const int32_t* __restrict__ accept_len, int* status) {
+  allow_dependents();
+  wait_prior_grids();   // best path and accept length; attention done with the cache
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int per_slice = 2 * chunks;
   const long long slice = gid / per_slice;
@@ -45,6 +47,7 @@ __global__ void __launch_bounds__(kThreads) accept_rows_kernel(
 }
 
 __global__ void advance_lens_kernel(int B, int32_t* seq_lens, const int32_t* accept_len) {
+  wait_prior_grids();   // every slice has read seq_lens
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) seq_lens[b] += accept_len[b] + 1;
 }
@@ -54,18 +57,17 @@ __global__ void advance_lens_kernel(int B, int32_t* seq_lens, const int32_t* acc
 medusa_status_t launch_accept_kv(const TreeDev& t, int layers, int B, int H, int hd, medusa_dtype_t dtype,
                                  void* k_cache, void* v_cache, int Lcap, int32_t* seq_lens,
                                  const int32_t* best_path, const int32_t* accept_len,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, bool pdl) {
   const int row_bytes = hd * (dtype == MEDUSA_BF16 ? 2 : 4);
   const int chunks = row_bytes / 16;
   const long long n_slices = static_cast<long long>(layers) * B * H;
   const long long threads = n_slices * 2 * chunks;
-  accept_rows_kernel<<<static_cast<unsigned>((threads + kThreads - 1) / kThreads), kThreads, 0, stream>>>(
-      t, static_cast<int>(n_slices), B, H, chunks, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), Lcap,
-      seq_lens, best_path, accept_len, device_status_ptr());
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(accept_rows_kernel, dim3(static_cast<unsigned>((threads + kThreads - 1) / kThreads)),
+                                dim3(kThreads), 0, stream, pdl, t, static_cast<int>(n_slices), B, H, chunks,
+                                static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), Lcap,
+                                static_cast<const int32_t*>(seq_lens), best_path, accept_len, device_status_ptr());
   if (e != cudaSuccess) return cuda_fail("medusa_accept_kv: rows launch", e);
-  advance_lens_kernel<<<(B + 63) / 64, 64, 0, stream>>>(B, seq_lens, accept_len);
-  e = cudaGetLastError();
+  e = launch_kernel(advance_lens_kernel, dim3((B + 63) / 64), dim3(64), 0, stream, pdl, B, seq_lens, accept_len);
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_accept_kv: lens launch", e);
 }
 

@@ -329,18 +329,28 @@ extern "C" medusa_status_t medusa_step(const medusa_step_args_t* a, void* worksp
                     a->best_path, a->accept_len);
   if (st != MEDUSA_OK) return st;
 
+  // S1-S4 in one launch per batch group: the heads kernel's last CTA also
+  // builds the candidate tree from the final top-k.
+  TreeBuild tb{};
+  tb.t = a->tree->dev;
+  tb.root_tokens = a->root_tokens;
+  tb.seq_lens = a->seq_lens;
+  tb.tree_tokens = a->tree_tokens;
+  tb.candidates = a->candidates;
+  tb.position_ids = a->position_ids;
   st = launch_heads(a->h, a->W1, a->b1, a->Wout, a->B, a->d, a->V, a->K, a->topk, a->dtype, a->head_logits,
-                    a->topk_ids, a->topk_vals, ws_heads, stream);
+                    a->topk_ids, a->topk_vals, ws_heads, stream, &tb);
   if (st != MEDUSA_OK) return st;
-  st = launch_build_tree(a->tree->dev, a->B, a->root_tokens, a->topk_ids, a->seq_lens, a->tree_tokens, a->candidates,
-                         a->position_ids, stream);
-  if (st != MEDUSA_OK) return st;
+  // Attention, posterior and compaction start while the kernel before them
+  // drains (programmatic dependent launch); each waits for its predecessor
+  // before it touches that kernel's outputs.
   st = launch_attention(a->tree->dev, a->layers, a->B, a->H, a->hd, a->dtype, a->q, a->k_cache, a->v_cache, a->Lcap,
-                        a->seq_lens, a->scale, a->attn_out, ws_attn, stream);
+                        a->seq_lens, a->scale, a->attn_out, ws_attn, stream, true);
   if (st != MEDUSA_OK) return st;
   st = launch_posterior(a->tree->dev, a->B, a->V, a->base_logits, a->candidates, a->mode, a->temperature, a->eps,
-                        a->alpha, a->best_path, a->accept_len, a->accepted_tokens, a->next_token, ws_post, stream);
+                        a->alpha, a->best_path, a->accept_len, a->accepted_tokens, a->next_token, ws_post, stream,
+                        true);
   if (st != MEDUSA_OK) return st;
   return launch_accept_kv(a->tree->dev, a->layers, a->B, a->H, a->hd, a->dtype, a->k_cache, a->v_cache, a->Lcap,
-                          a->seq_lens, a->best_path, a->accept_len, stream);
+                          a->seq_lens, a->best_path, a->accept_len, stream, true);
 }

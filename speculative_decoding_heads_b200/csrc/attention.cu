@@ -116,14 +116,14 @@ size_t attention_workspace_bytes(const TreeDev& t, int layers, int B, int H, int
 medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int hd, medusa_dtype_t dtype,
                                  const void* q, const void* k_cache, const void* v_cache, int Lcap,
                                  const int32_t* seq_lens, float scale, void* out, void* ws,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, bool pdl) {
   (void)ws;
   const int n_slices = layers * B * H;
   int* status = device_status_ptr();
   cudaError_t e;
   if (dtype == MEDUSA_BF16 && hd == kHd) {
     return launch_attention_tc64(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, scale * kLog2e,
-                                 static_cast<float*>(out), status, stream);
+                                 static_cast<float*>(out), status, stream, pdl);
   }
   {
     const size_t smem = static_cast<size_t>(hd + Lcap) * sizeof(float);

@@ -531,6 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = bar->tmem_base;
+  allow_dependents();
 
   if (warp == 0) {
     if (lane == 0) run_producer(&q_map, &k_map, &v_map, p, smem, bar);
@@ -547,6 +548,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
+  // Launched inside medusa_step without waiting for the heads kernel (it reads
+  // none of its outputs); completing only after it keeps the stream's order
+  // for the kernels that follow.
+  wait_prior_grids();
 }
 
 }  // namespace
@@ -571,7 +576,7 @@ void* tensor_map_encoder() {
 // the kernel falls back to two 16 KB boxes per tile.
 medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H, const void* q,
                                       const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
-                                      float scale_log2, float* out, int* status, cudaStream_t stream) {
+                                      float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl) {
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!enc) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: cuTensorMapEncodeTiled unavailable");
   if (t.T > 4 * kRows || t.W > 4) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: more than 256 tree tokens");
@@ -634,10 +639,7 @@ medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H
   prm.kv_one_box = one_box;
   const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
   cudaError_t e = cudaFuncSetAttribute(tree_attn_tc64, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e == cudaSuccess) {
-    tree_attn_tc64<<<grid, kThreads, kSmemBytes, stream>>>(qm, km, vm, prm);
-    e = cudaGetLastError();
-  }
+  if (e == cudaSuccess) e = launch_kernel(tree_attn_tc64, dim3(grid), dim3(kThreads), kSmemBytes, stream, pdl, qm, km, vm, prm);
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_tree_attention: tcgen05 launch", e);
 }
 

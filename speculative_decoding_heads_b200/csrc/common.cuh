@@ -39,6 +39,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---- programmatic dependent launch ------------------------------------------
+// In a kernel launched with programmatic stream serialisation, wait_prior_grids()
+// returns once the preceding kernel of the stream has completed and its memory
+// is visible; allow_dependents() lets the next such kernel be scheduled early.
+// Both are no-ops in a kernel launched the ordinary way.
+__device__ __forceinline__ void wait_prior_grids() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- mbarrier -------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

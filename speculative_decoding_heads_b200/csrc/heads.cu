@@ -69,6 +69,8 @@ struct HeadsArgs {
   int nvec;               // 16-byte vectors per row
   int NT;                 // consumer threads
   int p1_max;             // most phase-1 rows of any CTA
+  int do_build;           // 1: the last CTA also builds the candidate tree (S4) for all B sequences
+  TreeBuild build;
 };
 
 template <typename TW>
@@ -587,6 +589,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) heads_kernel(const HeadsArgs a
       cursor_next<R>(cc, a);
     }
   }
+  allow_dependents();   // the next kernel of medusa_step may take SMs as CTAs finish
   __syncthreads();
   if (flag[0]) return;   // aborted: the producer has drained its copies
 
@@ -679,6 +682,30 @@ __global__ void __launch_bounds__(kMaxThreads, 1) heads_kernel(const HeadsArgs a
     a.counters[1] = 0u;
     __threadfence();
   }
+  if (a.do_build) {
+    // S4 from the final top-k (this CTA's merge above and the earlier batch
+    // groups' launches): the flat list [root, head 1 top-k, ..., head K
+    // top-k] gathered through tree_indices and retrieve, and the positions.
+    const TreeDev& t = a.build.t;
+    const int per_b = 2 * t.T + t.P * (t.D + 1);
+    for (int g = tid; g < a.B * per_b; g += blockDim.x) {
+      const int b = g / per_b;
+      int o = g - b * per_b;
+      auto flat = [&](int fi) -> int32_t {
+        return fi == 0 ? a.build.root_tokens[b] : a.topk_ids[(static_cast<size_t>(b) * t.K) * t.topk + (fi - 1)];
+      };
+      if (o < t.T) {
+        a.build.tree_tokens[b * t.T + o] = flat(t.tree_indices[o]);
+      } else if (o < 2 * t.T) {
+        o -= t.T;
+        a.build.position_ids[b * t.T + o] = a.build.seq_lens[b] + t.depth[o];
+      } else {
+        o -= 2 * t.T;
+        const int node = t.retrieve[o];
+        a.build.candidates[static_cast<size_t>(b) * t.P * (t.D + 1) + o] = node < 0 ? -1 : flat(t.tree_indices[node]);
+      }
+    }
+  }
 }
 
 struct Plan {
@@ -760,7 +787,7 @@ size_t heads_workspace_bytes(int B, int d, int V, int K, int topk) {
 medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, const void* Wout,
                              int B, int d, int V, int K, int topk, medusa_dtype_t dtype,
                              float* head_logits, int32_t* topk_ids, float* topk_vals, void* ws,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const TreeBuild* build) {
   const int G = sm_count();
   HeadsArgs a{};
   a.h = h;
@@ -796,6 +823,8 @@ medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, cons
                                           : make_plan<float>(d, nbt, K, topk, a.p1_max);
     a.NS = p.NS;
     a.NT = p.NT;
+    a.do_build = (build != nullptr && b0 + a.nb == B) ? 1 : 0;   // after the last batch group
+    if (build) a.build = *build;
     cudaError_t e = (dtype == MEDUSA_BF16) ? dispatch_nb<uint16_t>(a, p, stream) : dispatch_nb<float>(a, p, stream);
     if (e != cudaSuccess) return cuda_fail("medusa_heads_topk: launch", e);
   }

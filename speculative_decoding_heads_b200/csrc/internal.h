@@ -4,6 +4,9 @@
 #include <cstdint>
 #include <string>
 #include <vector>
+#include <utility>
+
+#include <cuda_runtime.h>
 
 #include "medusa_b200.h"
 
@@ -43,12 +46,22 @@ medusa_status_t device_status_read(int32_t* status, int32_t* detail, int clear);
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// S4 outputs, when the heads kernel also builds the candidate tree (medusa_step).
+struct TreeBuild {
+  TreeDev t;
+  const int32_t* root_tokens;   // [B]
+  const int32_t* seq_lens;      // [B]
+  int32_t* tree_tokens;         // [B, T]
+  int32_t* candidates;          // [B, P, D+1]
+  int32_t* position_ids;        // [B, T]
+};
+
 // Kernel launchers (heads.cu, tree_kernels.cu, attention.cu, posterior.cu, accept.cu).
 size_t heads_workspace_bytes(int B, int d, int V, int K, int topk);
 medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, const void* Wout,
                              int B, int d, int V, int K, int topk, medusa_dtype_t dtype,
                              float* head_logits, int32_t* topk_ids, float* topk_vals, void* ws,
-                             cudaStream_t stream);
+                             cudaStream_t stream, const TreeBuild* build = nullptr);
 
 medusa_status_t launch_build_tree(const TreeDev& t, int B, const int32_t* root_tokens,
                                   const int32_t* topk_ids, const int32_t* seq_lens,
@@ -57,29 +70,49 @@ medusa_status_t launch_build_tree(const TreeDev& t, int B, const int32_t* root_t
 
 size_t attention_workspace_bytes(const TreeDev& t, int layers, int B, int H, int hd,
                                  medusa_dtype_t dtype);
+// `pdl`: launch with programmatic stream serialisation (only inside medusa_step,
+// where the preceding kernel is this library's own and the kernel waits for it
+// before it touches that kernel's outputs).
 medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int hd,
                                  medusa_dtype_t dtype, const void* q, const void* k_cache,
                                  const void* v_cache, int Lcap, const int32_t* seq_lens,
-                                 float scale, void* out, void* ws, cudaStream_t stream);
+                                 float scale, void* out, void* ws, cudaStream_t stream, bool pdl = false);
 
 size_t posterior_workspace_bytes(const TreeDev& t, int B);
 medusa_status_t launch_posterior(const TreeDev& t, int B, int V, const float* logits,
                                  const int32_t* candidates, medusa_mode_t mode, float temperature,
                                  float eps, float alpha, int32_t* best_path, int32_t* accept_len,
                                  int32_t* accepted_tokens, int32_t* next_token, void* ws,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, bool pdl = false);
 
 medusa_status_t launch_accept_kv(const TreeDev& t, int layers, int B, int H, int hd,
                                  medusa_dtype_t dtype, void* k_cache, void* v_cache, int Lcap,
                                  int32_t* seq_lens, const int32_t* best_path,
-                                 const int32_t* accept_len, cudaStream_t stream);
+                                 const int32_t* accept_len, cudaStream_t stream, bool pdl = false);
 
 // cuTensorMapEncodeTiled (PFN_cuTensorMapEncodeTiled_v12000), or null.
 void* tensor_map_encoder();
 
 medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H, const void* q,
                                       const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
-                                      float scale_log2, float* out, int* status, cudaStream_t stream);
+                                      float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl);
+
+// cudaLaunchKernelEx with programmatic stream serialisation when `pdl` is set.
+template <typename... Params, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(kThreads) posterior_kernel(
   __shared__ float red_v[32], red_s[32];
   __shared__ int red_i[32];
   __shared__ int s_last;
+  allow_dependents();
   const int row = blockIdx.x;           // b * T + node
   const int b = row / t.T;
   const float* z = logits + static_cast<size_t>(row) * V;
@@ -159,7 +160,9 @@ __global__ void __launch_bounds__(kThreads) posterior_kernel(
     }
   }
 
-  // ---- the last node of sequence b to finish evaluates the paths
+  // ---- the last node of sequence b to finish evaluates the paths (the
+  // candidates come from an earlier kernel of the step)
+  wait_prior_grids();
   if (tid == 0) {
     __threadfence();
     const unsigned done = atom_add_acq_rel_gpu(&counters[b], 1u);
@@ -223,16 +226,15 @@ medusa_status_t launch_posterior(const TreeDev& t, int B, int V, const float* lo
                                  const int32_t* candidates, medusa_mode_t mode, float temperature,
                                  float eps, float alpha, int32_t* best_path, int32_t* accept_len,
                                  int32_t* accepted_tokens, int32_t* next_token, void* ws,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, bool pdl) {
   if (t.P > kThreads) return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_evaluate_posterior: more than 1024 paths");
   NodeStat* stats = static_cast<NodeStat*>(ws);
   unsigned* counters = reinterpret_cast<unsigned*>(static_cast<unsigned char*>(ws) +
                                                    align_up(static_cast<size_t>(B) * t.T * sizeof(NodeStat), 256));
   const int typical = mode == MEDUSA_TYPICAL ? 1 : 0;
-  posterior_kernel<<<B * t.T, kThreads, 0, stream>>>(t, V, logits, candidates, typical, temperature, eps, alpha,
-                                                     stats, counters, best_path, accept_len, accepted_tokens,
-                                                     next_token, device_status_ptr());
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = launch_kernel(posterior_kernel, dim3(B * t.T), dim3(kThreads), 0, stream, pdl, t, V, logits,
+                                     candidates, typical, temperature, eps, alpha, stats, counters, best_path,
+                                     accept_len, accepted_tokens, next_token, device_status_ptr());
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_evaluate_posterior: launch", e);
 }
 
