@@ -5,9 +5,10 @@
 // j is i or one of its ancestors; the tree's own K/V already sit at rows
 // L..L+T-1 of the cache.
 //
-// bf16 with hd = 128 runs on the tcgen05 tensor cores in one persistent
-// kernel (attention_tc64.cu; one pass over a slice's K/V per 64 tree
-// tokens).  Every other dtype / head size
+// bf16 with hd = 128 runs on the tcgen05 tensor cores in a persistent kernel:
+// attention_tc64.cu for trees of up to 64 tokens, attention_tc128.cu for
+// larger trees (one pass over a slice's K/V per 128 tree tokens).  Every
+// other dtype / head size
 // runs tree_attn_generic: one CTA per (slice, node), scores in shared memory,
 // plain fp32 arithmetic.  The output is fp32 on every path.
 #include <cfloat>
@@ -122,8 +123,19 @@ medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int
   int* status = device_status_ptr();
   cudaError_t e;
   if (dtype == MEDUSA_BF16 && hd == kHd) {
-    return launch_attention_tc64(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, scale * kLog2e,
-                                 static_cast<float*>(out), status, stream, pdl);
+    // Rows in groups of 128 where a group would hold more than 64 of them,
+    // the rest (at most 64) in one 64-row group.
+    float* o = static_cast<float*>(out);
+    const float sl = scale * kLog2e;
+    const int full = t.T <= 64 ? 0 : (t.T % 128 == 0 || t.T % 128 > 64 ? t.T : t.T / 128 * 128);
+    if (full > 0) {
+      const medusa_status_t st =
+          launch_attention_tc128(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, sl, o, status, stream, pdl, 0,
+                                 full);
+      if (st != MEDUSA_OK || full == t.T) return st;
+    }
+    return launch_attention_tc64(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, sl, o, status, stream, pdl,
+                                 full, t.T);
   }
   {
     const size_t smem = static_cast<size_t>(hd + Lcap) * sizeof(float);

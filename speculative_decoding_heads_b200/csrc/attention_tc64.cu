@@ -92,6 +92,7 @@ struct Params {
   TreeDev t;
   int B, H, Lcap, total;   // total: work items = slices x groups
   int groups;              // ceil(T / 64)
+  int row_lo, row_hi;      // tree tokens (query rows) handled by this launch
   const int32_t* seq_lens;
   float scale_log2;
   float* out;
@@ -165,8 +166,8 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
       unsigned char* qd = smem + kOffQ + (nq & 1) * kQBuf;
       uint64_t* fb = &bar->q_full[nq & 1];
       mbar_arrive_expect_tx(fb, kQBuf);
-      tc::tma_load_4d(qd, q_map, 0, sq.e, kRows * sq.grp, sq.lb, fb);
-      tc::tma_load_4d(qd + kQHalf, q_map, 64, sq.e, kRows * sq.grp, sq.lb, fb);
+      tc::tma_load_4d(qd, q_map, 0, sq.e, p.row_lo + kRows * sq.grp, sq.lb, fb);
+      tc::tma_load_4d(qd + kQHalf, q_map, 64, sq.e, p.row_lo + kRows * sq.grp, sq.lb, fb);
       ++nq;
       ++kkq;
       sq = seek(kkq, p, bar->lens);
@@ -335,11 +336,11 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
     // This thread's tree token (query row) in the item's row group and its
     // ancestor mask (up to four words; loaded now, first used at the item's
     // last steps).
-    const int r = kRows * s.grp + 16 * q + i;
+    const int r = p.row_lo + kRows * s.grp + 16 * q + i;
     uint64_t anc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int wd = 0; wd < 4; ++wd)
-      if (r < T && wd < p.t.W) anc[wd] = p.t.anc[r * p.t.W + wd];
+      if (r < p.row_hi && wd < p.t.W) anc[wd] = p.t.anc[r * p.t.W + wd];
     float mref = -INFINITY, lsum = 0.f;
     for (int t = 0; t < s.steps; ++t, ++g) {
       if (!wait_bar(&bar->s_full[g & 1], (g >> 1) & 1, bar, p.status)) return;
@@ -464,7 +465,7 @@ __device__ void run_epilogue(const Params& p, uint32_t tmem, Bars* bar, int warp
     if (!wait_bar(&bar->l_ready[k & 1], (k >> 1) & 1, bar, p.status)) return;
     if (!wait_bar(&bar->o_full[k & 1], (k >> 1) & 1, bar, p.status)) return;
     tc::fence_after_sync();
-    const int r = kRows * s.grp + 16 * q + i;   // tree token
+    const int r = p.row_lo + kRows * s.grp + 16 * q + i;   // tree token
     const float inv = 1.f / bar->lsum[k & 1][16 * q + i];
     const uint32_t oa = tmem + la + col_o(k & 1);
     float* orow = p.out + ((static_cast<size_t>(s.lb) * T + r) * p.H + s.e) * kHd + 64 * h;
@@ -474,7 +475,7 @@ __device__ void run_epilogue(const Params& p, uint32_t tmem, Bars* bar, int warp
       tc::tmem_ld32x2<64>(oa + 32 * cp, a);
       tc::tmem_ld32x2<64>(oa + kLaneHalf + 32 * cp, b);
       tc::tmem_wait_ld();
-      if (r < T) {
+      if (r < p.row_hi) {
         float* dst = orow + 32 * cp;
 #pragma unroll
         for (int c = 0; c < 32; c += 4)
@@ -576,12 +577,15 @@ void* tensor_map_encoder() {
 // the kernel falls back to two 16 KB boxes per tile.
 medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H, const void* q,
                                       const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
-                                      float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl) {
+                                      float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl,
+                                      int row_lo, int row_hi) {
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!enc) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: cuTensorMapEncodeTiled unavailable");
   if (t.T > 4 * kRows || t.W > 4) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: more than 256 tree tokens");
   const long long slices = static_cast<long long>(layers) * B * H;
-  const int groups = (t.T + kRows - 1) / kRows;
+  if (row_lo < 0 || row_hi > t.T || row_lo >= row_hi)
+    return fail(MEDUSA_ERR_INVALID_ARG, "tree attention: empty row range");
+  const int groups = (row_hi - row_lo + kRows - 1) / kRows;
   const long long items = slices * groups;
   if (items >= (1ll << 31)) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: too many slices");
   CUtensorMap qm, km, vm;
@@ -632,6 +636,8 @@ medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H
   prm.Lcap = Lcap;
   prm.total = static_cast<int>(items);
   prm.groups = groups;
+  prm.row_lo = row_lo;
+  prm.row_hi = row_hi;
   prm.seq_lens = seq_lens;
   prm.scale_log2 = scale_log2;
   prm.out = out;

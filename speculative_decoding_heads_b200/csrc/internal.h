@@ -95,7 +95,13 @@ void* tensor_map_encoder();
 
 medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H, const void* q,
                                       const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
-                                      float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl);
+                                      float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl,
+                                      int row_lo, int row_hi);
+
+medusa_status_t launch_attention_tc128(const TreeDev& t, int layers, int B, int H, const void* q,
+                                       const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
+                                       float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl,
+                                       int row_lo, int row_hi);
 
 // cudaLaunchKernelEx with programmatic stream serialisation when `pdl` is set.
 template <typename... Params, typename... Args>

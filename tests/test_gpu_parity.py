@@ -135,29 +135,33 @@ def test_tree_attention(mb, dev, name):
     _attention_case(mb, dev, SMALL[name])
 
 
-@pytest.mark.parametrize("shape", [(2, 160, 200, 1), (1, 37, 131, 9)])
+@pytest.mark.parametrize("shape", [("v7b_small", 2, 160, 200, 1), ("v13b_small", 1, 37, 131, 9),
+                                   ("v33b_small", 1, 90, 150, 2)])
 def test_tree_attention_many_slices(mb, dev, shape):
-    # More (layer, sequence, head) slices than SMs: every persistent CTA walks
-    # several slices (Q, K/V, S, P and O buffers change hands between them);
-    # the second shape has ragged prefixes and slices split unevenly.
+    # More work items than SMs: every persistent CTA walks several (Q, K/V,
+    # S, P and O buffers change hands between them).  T 64; T 49 with ragged
+    # prefixes and an uneven split; T 129 in two 128-token row groups.
     from synth.workloads import shrink
-    layers, H, prefix, B = shape
-    base = SMALL["v7b_small"] if B == 1 else SMALL["v13b_small"]
+    name, layers, H, prefix, B = shape
     kw = dict(layers=layers, H=H, B=B)
-    if B == 1:
-        kw["prefix"] = prefix
-    else:
+    if name == "v13b_small":
         kw["prefix_range"] = (prefix // 4, prefix)
-    _attention_case(mb, dev, shrink(base, **kw))
+    else:
+        kw["prefix"] = prefix
+    _attention_case(mb, dev, shrink(SMALL[name], **kw))
 
 
-@pytest.mark.parametrize("variant", ["T200_two_row_groups", "hd64_bf16_generic", "hd256_f32", "chain_L0",
-                                     "exact_capacity"])
+@pytest.mark.parametrize("variant", ["T200_two_row_groups", "T100_L0", "hd64_bf16_generic", "hd256_f32",
+                                     "chain_L0", "exact_capacity"])
 def test_tree_attention_edges(mb, dev, variant):
     base = SMALL["v7b_small"]
     from synth.workloads import shrink
     if variant == "T200_two_row_groups":
         w = shrink(base, K=5, topk=10, n_nodes=199, prefix=70, layers=1, H=2)
+        _attention_case(mb, dev, w)
+    elif variant == "T100_L0":
+        # every key is a tree key: the masked path on every step
+        w = shrink(base, K=5, topk=10, n_nodes=99, prefix=0, layers=1, H=3)
         _attention_case(mb, dev, w)
     elif variant == "hd64_bf16_generic":
         _attention_case(mb, dev, shrink(base, hd=64, layers=1, H=3, prefix=90))
@@ -167,7 +171,7 @@ def test_tree_attention_edges(mb, dev, variant):
         w = shrink(base, K=5, topk=1, n_nodes=5, prefix=0, layers=1, H=2)
         _attention_case(mb, dev, w)
     else:
-        # Lcap = L + T exactly, and L + T a multiple of the 64-key tile
+        # Lcap = L + T exactly, and L + T a multiple of the 128-key step
         w = shrink(base, prefix=128 - 64, layers=1, H=2)
         assert w.Lcap == 128
         _attention_case(mb, dev, w)
