@@ -151,13 +151,18 @@ def test_tree_attention_many_slices(mb, dev, shape):
     _attention_case(mb, dev, shrink(SMALL[name], **kw))
 
 
-@pytest.mark.parametrize("variant", ["T200_two_row_groups", "T100_L0", "hd64_bf16_generic", "hd256_f32",
-                                     "chain_L0", "exact_capacity"])
+@pytest.mark.parametrize("variant", ["T200_two_row_groups", "T256_max", "T100_L0", "hd64_bf16_generic",
+                                     "hd256_f32", "chain_L0", "exact_capacity"])
 def test_tree_attention_edges(mb, dev, variant):
     base = SMALL["v7b_small"]
     from synth.workloads import shrink
     if variant == "T200_two_row_groups":
         w = shrink(base, K=5, topk=10, n_nodes=199, prefix=70, layers=1, H=2)
+        _attention_case(mb, dev, w)
+    elif variant == "T256_max":
+        # the largest tree (MEDUSA_MAX_T tokens): two full 128-token row groups
+        w = shrink(base, K=5, topk=10, n_nodes=255, prefix=100, layers=1, H=2)
+        assert w.T == 256
         _attention_case(mb, dev, w)
     elif variant == "T100_L0":
         # every key is a tree key: the masked path on every step
