@@ -41,9 +41,16 @@
 namespace medusa {
 namespace {
 
-constexpr int kMaxConsumers = 512;    // consumer threads
+constexpr int kMaxConsumers = 512;    // consumer threads, one sequence per launch
+constexpr int kMaxConsumersMulti = 832;   // consumer threads with 2-4 sequences (one vector each)
 constexpr int kRoleWarps = 2;         // producer + epilogue
 constexpr int kMaxThreads = kMaxConsumers + 32 * kRoleWarps;
+constexpr int kMaxThreadsMulti = kMaxConsumersMulti + 32 * kRoleWarps;
+// With several sequences per launch a thread's work per vector grows with
+// the batch; rows of 513-832 vectors (4-row stages) then get one vector per
+// thread (more warps to hide the FMA chains) instead of two.
+template <int NB, int VPT, int R>
+constexpr int heads_threads() { return (NB > 1 && VPT == 1 && R == 4) ? kMaxThreadsMulti : kMaxThreads; }
 constexpr int kMaxNB = 4;             // sequences per launch
 constexpr int kStageMax = 64 * 1024;  // bytes per stage: 8 rows when they fit, else 4
 constexpr int kRingTarget = 192 * 1024;
@@ -330,7 +337,7 @@ __host__ __device__ inline Layout make_layout(size_t stage_bytes, int NS, int NW
 }
 
 template <typename TW, int NB, int VPT, int R>
-__global__ void __launch_bounds__(kMaxThreads, 1) heads_kernel(const HeadsArgs a) {
+__global__ void __launch_bounds__(heads_threads<NB, VPT, R>(), 1) heads_kernel(const HeadsArgs a) {
   constexpr int E = Elem<TW>::E;
   constexpr int RNB = R * NB;
   static_assert(RNB <= 32 && (32 % RNB) == 0, "partials use one lane per (row, sequence)");
@@ -723,10 +730,11 @@ Plan make_plan(int d, int nb, int K, int topk, int p1_max) {
   constexpr int E = Elem<TW>::E;
   Plan p{};
   const int nvec = d / E;
-  p.NT = nvec >= kMaxConsumers ? kMaxConsumers : ((nvec + 31) / 32) * 32;
-  p.VPT = (nvec + p.NT - 1) / p.NT;
   const size_t row = static_cast<size_t>(d) * sizeof(TW);
   p.R = row * 8 <= static_cast<size_t>(kStageMax) ? 8 : 4;
+  const int max_nt = (nb > 1 && p.R == 4 && nvec <= kMaxConsumersMulti) ? kMaxConsumersMulti : kMaxConsumers;
+  p.NT = nvec >= max_nt ? max_nt : ((nvec + 31) / 32) * 32;
+  p.VPT = (nvec + p.NT - 1) / p.NT;
   const size_t stage = row * p.R;
   const int ns = static_cast<int>(kRingTarget / stage);
   p.NS = ns < 2 ? 2 : (ns > kMaxStages ? kMaxStages : ns);
