@@ -90,6 +90,25 @@ def test_heads_topk(mb, dev, name):
     _status_clean(mb)
 
 
+@pytest.mark.parametrize("B", [4, 5])
+def test_heads_topk_wide_rows(mb, dev, B):
+    # d 5120 (640 16-byte vectors, 4-row stages): with 2-4 sequences per launch
+    # one vector per consumer thread (26 warps); B 5 runs groups of 4 and 1.
+    from synth.workloads import shrink
+    w = shrink(SMALL["v13b_small"], name=f"heads_wide_B{B}", d=5120, V=1500, B=B)
+    sub_h, u, z = pick_sub_h(w)
+    ids_ref, vals_ref = O.topk_desc(z, w.topk)
+    t = dev.materialise(w, sub_h=sub_h)
+    ws = mb.workspace(mb.medusa_heads_workspace_size(w.B, w.d, w.V, w.K, w.topk))
+    mb.medusa_heads_topk(t["h"], t["W1"], t["b1"], t["Wout"], w.topk, t["topk_ids"], t["topk_vals"], ws,
+                         head_logits=t["head_logits"])
+    torch.cuda.synchronize()
+    assert np.array_equal(_np(t["topk_ids"]), ids_ref)
+    check_logits(_np(t["head_logits"]), z)
+    check_logits(_np(t["topk_vals"]), vals_ref)
+    _status_clean(mb)
+
+
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_build_tree(mb, dev, name):
     w = SMALL[name]
