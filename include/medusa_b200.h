@@ -64,7 +64,7 @@
 extern "C" {
 #endif
 
-#define MEDUSA_ABI_VERSION 1
+#define MEDUSA_ABI_VERSION 2
 #define MEDUSA_MAX_T 256     /* tree tokens including the root */
 #define MEDUSA_MAX_K 16      /* heads (so tree depth <= 16) */
 #define MEDUSA_MAX_TOPK 32   /* candidates per head */
@@ -288,6 +288,12 @@ typedef struct medusa_step_args {
   int32_t* accept_len;
   int32_t* accepted_tokens;
   int32_t* next_token;
+  /* Optional (may be null): events the step waits for on `stream` right
+   * before tree attention (q and the tree's K/V rows in the caches are ready)
+   * and right before the posterior (base_logits ready), so that a caller can
+   * copy those inputs on another stream while the heads run. */
+  cudaEvent_t attn_inputs_ready;
+  cudaEvent_t posterior_inputs_ready;
 } medusa_step_args_t;
 
 size_t medusa_step_workspace_size(const medusa_step_args_t* args);

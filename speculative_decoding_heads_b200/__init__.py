@@ -26,6 +26,11 @@ if not os.path.exists(LIB_PATH):
         "`python -m speculative_decoding_heads_b200._build` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
+ABI_VERSION = 2   # layout of medusa_step_args_t (StepArgs below) and of every signature
+_lib.medusa_abi_version.restype = ctypes.c_int
+if _lib.medusa_abi_version() != ABI_VERSION:
+    raise ImportError(f"{LIB_PATH} has ABI version {_lib.medusa_abi_version()}, this binding needs "
+                      f"{ABI_VERSION}; rebuild it")
 
 MEDUSA_OK = 0
 MEDUSA_ERR_INVALID_ARG = 1
@@ -79,6 +84,7 @@ class StepArgs(ctypes.Structure):
         ("tree_tokens", _vp), ("candidates", _vp), ("position_ids", _vp),
         ("attn_out", _vp),
         ("best_path", _vp), ("accept_len", _vp), ("accepted_tokens", _vp), ("next_token", _vp),
+        ("attn_inputs_ready", _vp), ("posterior_inputs_ready", _vp),
     ]
 
 
@@ -318,22 +324,41 @@ def medusa_step(args: StepArgs, ws, stream=None):
     _check(_lib.medusa_step(ctypes.byref(args), _p(ws), ws.numel(), _stream(stream)))
 
 
-def medusa_step_from_host(args: StepArgs, ws, host_in: dict, dev: dict, host_out: dict, stream=None):
+def medusa_step_from_host(args: StepArgs, ws, host_in: dict, dev: dict, host_out: dict, stream=None,
+                          copy_stream=None):
     """One step through the public API with host buffers.
 
     Copies every per-step input from pinned host memory (``host_in``: name ->
     pinned tensor, copied into ``dev[name]``; the tree's own K/V rows are
     given as ``k_tree``/``v_tree`` [layers, B, H, T, hd] and scattered into
     the caches at each sequence's current length), runs ``medusa_step`` and
-    reads the results back into the pinned ``host_out`` tensors.  All copies
-    are enqueued on ``stream``; the caller synchronises.
+    reads the results back into the pinned ``host_out`` tensors.
+
+    The heads need only h, the root tokens and the lengths, which go first
+    on ``stream``; q, the tree's K/V rows and then the base logits go on
+    ``copy_stream`` (a second stream, created on first use when omitted)
+    while the heads run, and the step waits for them (through
+    ``attn_inputs_ready`` / ``posterior_inputs_ready``) only before tree
+    attention and before the posterior.  The caller synchronises ``stream``.
     """
     s = stream or torch.cuda.current_stream()
+    if copy_stream is None:
+        if getattr(args, "_copy_stream", None) is None:
+            args._copy_stream = torch.cuda.Stream()
+        copy_stream = args._copy_stream
+    if getattr(args, "_events", None) is None:
+        args._events = (torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event())
+    ev_start, ev_attn, ev_post = args._events
+    early = ("h", "root_tokens", "seq_lens")
     with torch.cuda.stream(s):
-        for name, src in host_in.items():
-            if name in ("k_tree", "v_tree"):
-                continue
-            dev[name].copy_(src, non_blocking=True)
+        for name in early:
+            if name in host_in:
+                dev[name].copy_(host_in[name], non_blocking=True)
+        ev_start.record(s)   # everything earlier on `stream` (the previous step) comes first
+    with torch.cuda.stream(copy_stream):
+        copy_stream.wait_event(ev_start)
+        if "q" in host_in:
+            dev["q"].copy_(host_in["q"], non_blocking=True)
         if "k_tree" in host_in:
             lens = host_in["seq_lens"]
             T = host_in["k_tree"].shape[3]
@@ -341,6 +366,20 @@ def medusa_step_from_host(args: StepArgs, ws, host_in: dict, dev: dict, host_out
                 L = int(lens[b])
                 dev["k_cache"][:, b, :, L:L + T, :].copy_(host_in["k_tree"][:, b], non_blocking=True)
                 dev["v_cache"][:, b, :, L:L + T, :].copy_(host_in["v_tree"][:, b], non_blocking=True)
-        medusa_step(args, ws, s)
-        for name, dst in host_out.items():
-            dst.copy_(dev[name], non_blocking=True)
+        for name, src in host_in.items():
+            if name not in early and name not in ("q", "k_tree", "v_tree", "base_logits"):
+                dev[name].copy_(src, non_blocking=True)
+        ev_attn.record(copy_stream)
+        if "base_logits" in host_in:
+            dev["base_logits"].copy_(host_in["base_logits"], non_blocking=True)
+        ev_post.record(copy_stream)
+    args.attn_inputs_ready = ctypes.c_void_p(ev_attn.cuda_event)
+    args.posterior_inputs_ready = ctypes.c_void_p(ev_post.cuda_event)
+    try:
+        with torch.cuda.stream(s):
+            medusa_step(args, ws, s)
+            for name, dst in host_out.items():
+                dst.copy_(dev[name], non_blocking=True)
+    finally:
+        args.attn_inputs_ready = None
+        args.posterior_inputs_ready = None

@@ -344,9 +344,17 @@ extern "C" medusa_status_t medusa_step(const medusa_step_args_t* a, void* worksp
   // Attention, posterior and compaction start while the kernel before them
   // drains (programmatic dependent launch); each waits for its predecessor
   // before it touches that kernel's outputs.
+  if (a->attn_inputs_ready) {
+    const cudaError_t e = cudaStreamWaitEvent(stream, a->attn_inputs_ready, 0);
+    if (e != cudaSuccess) return cuda_fail("medusa_step: wait for the attention inputs", e);
+  }
   st = launch_attention(a->tree->dev, a->layers, a->B, a->H, a->hd, a->dtype, a->q, a->k_cache, a->v_cache, a->Lcap,
                         a->seq_lens, a->scale, a->attn_out, ws_attn, stream, true);
   if (st != MEDUSA_OK) return st;
+  if (a->posterior_inputs_ready) {
+    const cudaError_t e = cudaStreamWaitEvent(stream, a->posterior_inputs_ready, 0);
+    if (e != cudaSuccess) return cuda_fail("medusa_step: wait for the posterior inputs", e);
+  }
   st = launch_posterior(a->tree->dev, a->B, a->V, a->base_logits, a->candidates, a->mode, a->temperature, a->eps,
                         a->alpha, a->best_path, a->accept_len, a->accepted_tokens, a->next_token, ws_post, stream,
                         true);

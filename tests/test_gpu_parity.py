@@ -400,3 +400,46 @@ def test_device_check_on_overflowing_sequence(mb, dev):
     assert st == mb.MEDUSA_ERR_DEVICE_CHECK
     assert (t["attn_out"] == 0).all()
     _status_clean(mb)
+
+
+def test_step_from_host_matches_device_step(mb, dev):
+    # The host-buffer step copies q, the tree's K/V rows and the base logits
+    # on a second stream while the heads run; the step waits for them through
+    # the two input-ready events.  Its results equal a step over device inputs.
+    w = SMALL["v7b_small"]
+    sub_h, _, _ = pick_sub_h(w)
+    tree = _tree(mb, w)
+    t = dev.materialise(w, sub_h=sub_h)
+    dev.tree_outputs(t, w.B, tree.T, tree.P, tree.D)
+    args = mb.make_step_args(tree, t, mb.MEDUSA_GREEDY)
+    ws = mb.workspace(mb.medusa_step_workspace_size(args))
+    lens0 = t["seq_lens"].clone()
+    kc0, vc0 = t["k_cache"].clone(), t["v_cache"].clone()
+    mb.medusa_step(args, ws)
+    torch.cuda.synchronize()
+    ref = {k: t[k].clone() for k in ("best_path", "accept_len", "accepted_tokens", "next_token", "attn_out",
+                                     "seq_lens", "k_cache")}
+    pin = lambda x: x.cpu().pin_memory()
+    L = lens0.cpu()
+    host_in = {"h": pin(t["h"]), "root_tokens": pin(t["root_tokens"]), "seq_lens": pin(lens0),
+               "q": pin(t["q"]), "base_logits": pin(t["base_logits"]),
+               "k_tree": pin(torch.stack([kc0[:, b, :, int(L[b]):int(L[b]) + w.T] for b in range(w.B)], 1)),
+               "v_tree": pin(torch.stack([vc0[:, b, :, int(L[b]):int(L[b]) + w.T] for b in range(w.B)], 1))}
+    host_out = {k: torch.empty_like(t[k], device="cpu").pin_memory()
+                for k in ("best_path", "accept_len", "accepted_tokens", "next_token")}
+    # clobber every input and output the host step must bring back
+    for k in ("q", "base_logits", "attn_out"):
+        t[k].fill_(float("nan"))
+    for k in ("best_path", "accept_len", "accepted_tokens", "next_token"):
+        t[k].fill_(-9)
+    t["k_cache"].copy_(kc0)
+    t["v_cache"].copy_(vc0)
+    stream = torch.cuda.Stream()
+    mb.medusa_step_from_host(args, ws, host_in, dict(t), host_out, stream)
+    stream.synchronize()
+    for k in host_out:
+        assert torch.equal(host_out[k], ref[k].cpu()), k
+    assert torch.equal(t["attn_out"], ref["attn_out"])
+    assert torch.equal(t["seq_lens"], ref["seq_lens"])
+    assert torch.equal(t["k_cache"], ref["k_cache"])
+    _status_clean(mb)
