@@ -52,6 +52,10 @@ constexpr uint32_t kColO = 256;
 __device__ __forceinline__ uint32_t col_q(int buf) { return 384u + 64u * buf; }
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kLenTab = 256;                   // prefix lengths of a CTA's first items, in shared memory
+// The polling loops of the producer and the MMA issuer give up after this
+// many SM cycles without progress (about 2 s at 2 GHz); the SM cycle counter
+// is read on every pass, the global timer is too slow for that.
+constexpr long long kSpinLimitCycles = 4000000000LL;
 
 struct Bars {
   uint64_t k_full[kStagesK], k_empty[kStagesK], v_full[kStagesV], v_empty[kStagesV];
@@ -163,7 +167,7 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
   Slice sk = seek(kkk, p, bar->lens), sv = seek(kkv, p, bar->lens);
   int ek = 0, gv = 0;     // K-ring entries and V tiles issued
   int tk = -1, tv = 0;    // step of the next K-ring entry (-1: the item's Q entry); of the next V tile
-  uint64_t last = globaltimer_ns();
+  long long last = clock64();
   while ((sk.slice < p.total || sv.slice < p.total) && !bar->abort) {
     bool progressed = false;
     if (sk.slice < p.total) {
@@ -212,9 +216,9 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
       }
     }
     if (progressed) {
-      last = globaltimer_ns();
+      last = clock64();
     } else {
-      if (globaltimer_ns() - last > kSpinLimitNs) {
+      if (clock64() - last > kSpinLimitCycles) {
         set_device_status(p.status, MEDUSA_ERR_TIMEOUT, kDetailAttnStageWait);
         bar->abort = 1;
         break;
@@ -234,7 +238,8 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
 // item two back, completed before S of the previous item could start: S has
 // one buffer).  S(g) = Q K^T: eight M = 128, N = 128, K = 16 products with Q
 // from tensor memory.  O += P_hi V + P_lo V: two products per 16 valid keys.
-// S runs at most one step ahead of P V.
+// S(g) waits for K(g) and for the softmax to have read S(g - 1), not for
+// P V(g - 1), so it runs while the softmax of step g - 1 still computes.
 __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* bar) {
   constexpr uint32_t idS = tc::idesc_bf16_f32(128, kStep, 0);
   constexpr uint32_t idO = tc::idesc_bf16_f32(128, kHd, 1);
@@ -243,7 +248,7 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
   int ek = 0;
   int gs = 0, ts = -1, ks = 0;     // S cursor (ts = -1: Q entry next)
   int gp = 0, tp = 0, kp = 0;      // P V cursor
-  uint64_t last = globaltimer_ns();
+  long long last = clock64();
   while ((ss.slice < p.total || sp.slice < p.total) && !bar->abort) {
     bool progressed = false;
     const int st = ek % kStagesK;
@@ -259,7 +264,7 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
         ++ek;
         ts = 0;
         progressed = true;
-      } else if (gs <= gp + 1 && (gs == 0 || mbar_test(&bar->s_free, (gs - 1) & 1))) {
+      } else if (gs == 0 || mbar_test(&bar->s_free, (gs - 1) & 1)) {
         tc::fence_after_sync();
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -306,9 +311,9 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
       progressed = true;
     }
     if (progressed) {
-      last = globaltimer_ns();
+      last = clock64();
     } else {
-      if (globaltimer_ns() - last > kSpinLimitNs) {
+      if (clock64() - last > kSpinLimitCycles) {
         set_device_status(p.status, MEDUSA_ERR_TIMEOUT, kDetailAttnStageWait);
         bar->abort = 1;
         break;

@@ -60,6 +60,10 @@ __device__ __forceinline__ uint32_t col_o(int buf) { return 256u + 128u * buf; }
 constexpr uint32_t kLaneHalf = 16u << 16;      // TMEM address offset of lane 16
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kLenTab = 160;                   // prefix lengths of a CTA's first slices, in shared memory
+// The polling loops of the producer and the MMA issuer give up after this
+// many SM cycles without progress (about 2 s at 2 GHz); the SM cycle counter
+// is read on every pass, the global timer is too slow for that.
+constexpr long long kSpinLimitCycles = 4000000000LL;
 
 struct Bars {
   uint64_t q_full[2], q_empty[2];
@@ -142,6 +146,22 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return r;
 }
 
+// Two fp32 values in one register pair, and the packed fp32 FMA of sm_100
+// (two independent IEEE fmas per instruction).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 // Keys of step t that belong to the slice (1..128).
 __device__ __forceinline__ int step_keys(const Slice& s, int t) {
   const int first = s.n - t * kStep;
@@ -159,7 +179,7 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
   int kkq = 0, kkk = 0, kkv = 0;
   Slice sq = seek(kkq, p, bar->lens), sk = seek(kkk, p, bar->lens), sv = seek(kkv, p, bar->lens);
   int nq = 0, gk = 0, gv = 0, tk = 0, tv = 0;     // loads issued; step within slice
-  uint64_t last = globaltimer_ns();
+  long long last = clock64();
   while ((sq.slice < p.total || sk.slice < p.total || sv.slice < p.total) && !bar->abort) {
     bool progressed = false;
     if (sq.slice < p.total && (nq < 2 || mbar_test(&bar->q_empty[nq & 1], ((nq >> 1) - 1) & 1))) {
@@ -201,9 +221,9 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
       progressed = true;
     }
     if (progressed) {
-      last = globaltimer_ns();
+      last = clock64();
     } else {
-      if (globaltimer_ns() - last > kSpinLimitNs) {
+      if (clock64() - last > kSpinLimitCycles) {
         set_device_status(p.status, MEDUSA_ERR_TIMEOUT, kDetailAttnStageWait);
         bar->abort = 1;
         break;
@@ -231,8 +251,9 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
 // ---- MMA issuer (one thread) ------------------------------------------------
 // S(g) = Q K^T of step g (M = 64, N = 128, 8 products over the head dim) and
 // O += P(g) V (M = 128, N = 128, one product per 16 valid keys).  Both are
-// issued as soon as their inputs are ready; S runs at most one step ahead of
-// P V.
+// issued as soon as their inputs are ready: S(g) needs K(g) and its TMEM lane
+// half back from the softmax of step g - 2, not P V(g - 1), so the products
+// of later steps run while the softmax of this one computes.
 __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* bar) {
   constexpr uint32_t idS = tc::idesc_bf16_f32(64, kStep, 0);
   constexpr uint32_t idO = tc::idesc_bf16_f32(128, kHd, 1);
@@ -240,10 +261,10 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
   Slice ss = seek(kks, p, bar->lens), sp = seek(kkp, p, bar->lens);
   int gs = 0, ts = 0, ks = 0;     // S cursor: global step, step in slice, slice count
   int gp = 0, tp = 0, kp = 0;     // P V cursor
-  uint64_t last = globaltimer_ns();
+  long long last = clock64();
   while ((ss.slice < p.total || sp.slice < p.total) && !bar->abort) {
     bool progressed = false;
-    if (ss.slice < p.total && gs <= gp + 1 && (ts != 0 || mbar_test(&bar->q_full[ks & 1], (ks >> 1) & 1)) &&
+    if (ss.slice < p.total && (ts != 0 || mbar_test(&bar->q_full[ks & 1], (ks >> 1) & 1)) &&
         mbar_test(&bar->k_full[gs % kStages], (gs / kStages) & 1) &&
         (gs < 2 || mbar_test(&bar->s_free[gs & 1], ((gs >> 1) - 1) & 1))) {
       tc::fence_after_sync();
@@ -295,9 +316,9 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
       progressed = true;
     }
     if (progressed) {
-      last = globaltimer_ns();
+      last = clock64();
     } else {
-      if (globaltimer_ns() - last > kSpinLimitNs) {
+      if (clock64() - last > kSpinLimitCycles) {
         set_device_status(p.status, MEDUSA_ERR_TIMEOUT, kDetailAttnStageWait);
         bar->abort = 1;
         break;
@@ -355,7 +376,11 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
       if (lane == 0) tc::mbar_arrive(&bar->s_free[g & 1]);
 
       const int key0 = t * kStep + h * 64;
-      float tmax = -INFINITY;
+      // Eight independent partial maxima (the maximum does not depend on the
+      // order; the short chains keep the one warp per scheduler busy).
+      float mx[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mx[j] = -INFINITY;
       if (key0 + 64 > s.L) {
         // Allowed keys of this window as a bit mask: the cached prefix, then
         // the tree tokens that are ancestors of (or equal to) row r.
@@ -367,12 +392,13 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
         for (int c = 0; c < 64; ++c) {
           const uint32_t bit = c < 32 ? (mlo >> c) & 1u : (mhi >> (c - 32)) & 1u;
           sv[c] = bit ? sv[c] : -INFINITY;
-          tmax = fmaxf(tmax, sv[c]);
+          mx[c & 7] = fmaxf(mx[c & 7], sv[c]);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) tmax = fmaxf(tmax, sv[c]);
+        for (int c = 0; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], sv[c]);
       }
+      float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16)) * p.scale_log2;   // both halves of the row
       float factor = 1.f;
       if (tmax > mref + kRescaleLog2 || (mref == -INFINITY && tmax > -INFINITY)) {
@@ -380,11 +406,24 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
         mref = tmax;
       }
       const float nmu = (mref == -INFINITY) ? 0.f : -mref;
+      // p = 2^(s * scale * log2(e) - m): the scaling as packed fmas, four
+      // packed partial sums of p.
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(nmu, nmu), one2 = f2_pack(1.f, 1.f);
+      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sc2, nm2), x0, x1);
+        sv[c] = tc::ex2_ftz(x0);
+        sv[c + 1] = tc::ex2_ftz(x1);
+        acc2[(c >> 1) & 3] = f2_fma(f2_pack(sv[c], sv[c + 1]), one2, acc2[(c >> 1) & 3]);
+      }
       float ps = 0.f;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        sv[c] = tc::ex2_ftz(fmaf(sv[c], p.scale_log2, nmu));
-        ps += sv[c];
+      for (int j = 0; j < 4; ++j) {
+        float a, b;
+        f2_unpack(acc2[j], a, b);
+        ps += a + b;
       }
       lsum = lsum * factor + ps;
 
