@@ -21,6 +21,9 @@
  *   S7     medusa_accept_kv         move the accepted path's K/V rows to the
  *                                   end of the cached prefix.
  *          ["Medusa — 让大模型…", 实践案例 case 1 step 4]
+ *   S3 over G ranks  medusa_topk_merge  the global top-k from the top-k lists
+ *                                   of G vocabulary shards (rows of Wout
+ *                                   split across ranks, lists all-gathered).
  *   medusa_step                     S1..S7 in order on one stream.
  *
  * Conventions shared by every call:
@@ -64,11 +67,12 @@
 extern "C" {
 #endif
 
-#define MEDUSA_ABI_VERSION 2
+#define MEDUSA_ABI_VERSION 3
 #define MEDUSA_MAX_T 256     /* tree tokens including the root */
 #define MEDUSA_MAX_K 16      /* heads (so tree depth <= 16) */
 #define MEDUSA_MAX_TOPK 32   /* candidates per head */
 #define MEDUSA_MAX_B 64      /* sequences per call */
+#define MEDUSA_MAX_SHARDS 64 /* vocabulary shards merged by medusa_topk_merge */
 
 typedef enum medusa_status {
   MEDUSA_OK = 0,
@@ -180,6 +184,29 @@ medusa_status_t medusa_heads_topk_noalloc(const void* h, const void* W1, const v
                                           const void* Wout, int B, int d, int V, int K, int topk,
                                           medusa_dtype_t dtype, float* head_logits,
                                           int32_t* topk_ids, float* topk_vals, cudaStream_t stream);
+
+/* S3 with the vocabulary split over G ranks.  Rank g holds rows
+ * [row0[g], row0[g] + n_g) of every Wout[k] (n_g = row0[g+1] - row0[g], the
+ * last shard ends at V) as a [K, n_g, d] array and runs medusa_heads_topk on
+ * it with V = n_g, which gives top-k lists with shard-local ids; the G lists
+ * are then gathered on every rank (an all-gather of G*B*K*topk values and
+ * ids, a few KB).  This call turns the gathered lists into the lists that
+ * medusa_heads_topk gives on the whole Wout:
+ *   vals, ids  [G, B, K, topk] device (ids shard-local, as written by
+ *              medusa_heads_topk)
+ *   row0       [G] HOST int32: row0[0] = 0, each shard at least topk rows
+ *              (row0[g+1] - row0[g] >= topk and V - row0[G-1] >= topk)
+ *   out_vals   [B, K, topk] fp32, out_ids [B, K, topk] int32 (global ids):
+ *              the topk best of the G*topk candidates, value descending,
+ *              lower token id first on equal values (NaN last).
+ * The heads kernel computes each logit the same way whatever V is, so the
+ * result equals the unsplit top-k bit for bit.  Pure selection; no
+ * workspace.  1 <= G <= MEDUSA_MAX_SHARDS, 1 <= B <= MEDUSA_MAX_B,
+ * 1 <= K <= MEDUSA_MAX_K, 1 <= topk <= MEDUSA_MAX_TOPK.
+ * ["Medusa — 让大模型自己同时猜好几个 token", 核心要点: per-head top-k] */
+medusa_status_t medusa_topk_merge(const float* vals, const int32_t* ids, const int32_t* row0, int G,
+                                  int V, int B, int K, int topk, float* out_vals, int32_t* out_ids,
+                                  cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* S4: candidate assembly                                                    */

@@ -26,7 +26,7 @@ if not os.path.exists(LIB_PATH):
         "`python -m speculative_decoding_heads_b200._build` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
-ABI_VERSION = 2   # layout of medusa_step_args_t (StepArgs below) and of every signature
+ABI_VERSION = 3   # layout of medusa_step_args_t (StepArgs below) and of every signature
 _lib.medusa_abi_version.restype = ctypes.c_int
 if _lib.medusa_abi_version() != ABI_VERSION:
     raise ImportError(f"{LIB_PATH} has ABI version {_lib.medusa_abi_version()}, this binding needs "
@@ -42,7 +42,7 @@ MEDUSA_F32 = 0
 MEDUSA_BF16 = 1
 MEDUSA_GREEDY = 0
 MEDUSA_TYPICAL = 1
-MAX_T, MAX_K, MAX_TOPK, MAX_B = 256, 16, 32, 64
+MAX_T, MAX_K, MAX_TOPK, MAX_B, MAX_SHARDS = 256, 16, 32, 64, 64
 
 # Every symbol the header declares (checked by the CPU tests).
 EXPORTED = [
@@ -50,7 +50,7 @@ EXPORTED = [
     "medusa_tree_choices_ranksum", "medusa_tree_create", "medusa_tree_destroy",
     "medusa_tree_info", "medusa_tree_tables",
     "medusa_heads_workspace_size", "medusa_heads_topk", "medusa_heads_topk_noalloc",
-    "medusa_build_tree",
+    "medusa_topk_merge", "medusa_build_tree",
     "medusa_attention_workspace_size", "medusa_tree_attention",
     "medusa_posterior_workspace_size", "medusa_evaluate_posterior",
     "medusa_accept_kv",
@@ -106,6 +106,7 @@ _sig("medusa_tree_tables", _i32, [_vp, _pi32, _pi32, _pi32, _pi32, _pu64])
 _sig("medusa_heads_workspace_size", _sz, [_i32] * 5)
 _sig("medusa_heads_topk", _i32, [_vp, _vp, _vp, _vp] + [_i32] * 5 + [_i32, _vp, _vp, _vp, _vp, _sz, _vp])
 _sig("medusa_heads_topk_noalloc", _i32, [_vp, _vp, _vp, _vp] + [_i32] * 5 + [_i32, _vp, _vp, _vp, _vp])
+_sig("medusa_topk_merge", _i32, [_vp, _vp, _pi32] + [_i32] * 5 + [_vp, _vp, _vp])
 _sig("medusa_build_tree", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp])
 _sig("medusa_attention_workspace_size", _sz, [_vp, _i32, _i32, _i32, _i32, _i32])
 _sig("medusa_tree_attention", _i32,
@@ -251,6 +252,17 @@ def medusa_heads_topk_noalloc(h, W1, b1, Wout, topk, topk_ids, topk_vals, head_l
     K, V = Wout.shape[0], Wout.shape[1]
     _check(_lib.medusa_heads_topk_noalloc(_p(h), _p(W1), _p(b1), _p(Wout), B, d, V, K, topk, _dtype(h),
                                           _p(head_logits), _p(topk_ids), _p(topk_vals), _stream(stream)))
+
+
+def medusa_topk_merge(vals, ids, row0: Sequence[int], V: int, out_vals, out_ids, stream=None):
+    """Global top-k from gathered per-shard lists: vals/ids [G, B, K, topk] (shard-local ids),
+    row0[g] the first vocabulary row of shard g; writes out_vals/out_ids [B, K, topk]."""
+    G, B, K, topk = vals.shape
+    if len(row0) != G:
+        raise ValueError(f"row0 has {len(row0)} entries for {G} shards")
+    r0 = (ctypes.c_int32 * G)(*[int(x) for x in row0])
+    _check(_lib.medusa_topk_merge(_p(vals), _p(ids), r0, G, V, B, K, topk, _p(out_vals), _p(out_ids),
+                                  _stream(stream)))
 
 
 def medusa_build_tree(tree: Tree, root_tokens, topk_ids, seq_lens, tree_tokens, candidates,

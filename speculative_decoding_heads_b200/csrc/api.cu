@@ -152,6 +152,24 @@ extern "C" medusa_status_t medusa_heads_topk(const void* h, const void* W1, cons
                       stream);
 }
 
+extern "C" medusa_status_t medusa_topk_merge(const float* vals, const int32_t* ids, const int32_t* row0, int G,
+                                             int V, int B, int K, int topk, float* out_vals, int32_t* out_ids,
+                                             cudaStream_t stream) {
+  const char* fn = "medusa_topk_merge";
+  if (!vals || !ids || !row0 || !out_vals || !out_ids) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (G < 1 || G > MEDUSA_MAX_SHARDS || B < 1 || B > MEDUSA_MAX_B || K < 1 || K > MEDUSA_MAX_K)
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": G, B or K out of range");
+  if (topk < 1 || topk > MEDUSA_MAX_TOPK) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": topk out of range");
+  if (row0[0] != 0) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": row0[0] must be 0");
+  for (int g = 0; g < G; ++g) {
+    const long long end = g + 1 < G ? row0[g + 1] : V;
+    if (end - row0[g] < topk)
+      return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": shard " + std::to_string(g) + " holds fewer than topk rows");
+  }
+  if (sm_count() <= 0) return fail(MEDUSA_ERR_CUDA, std::string(fn) + ": no usable CUDA device");
+  return launch_topk_merge(vals, ids, row0, G, B, K, topk, out_vals, out_ids, stream);
+}
+
 extern "C" medusa_status_t medusa_build_tree(const medusa_tree_t* tree, int B, const int32_t* root_tokens,
                                              const int32_t* topk_ids, const int32_t* seq_lens,
                                              int32_t* tree_tokens, int32_t* candidates, int32_t* position_ids,

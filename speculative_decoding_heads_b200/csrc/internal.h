@@ -90,6 +90,9 @@ medusa_status_t launch_accept_kv(const TreeDev& t, int layers, int B, int H, int
                                  int32_t* seq_lens, const int32_t* best_path,
                                  const int32_t* accept_len, cudaStream_t stream, bool pdl = false);
 
+medusa_status_t launch_topk_merge(const float* vals, const int32_t* ids, const int32_t* row0, int G, int B,
+                                  int K, int topk, float* out_vals, int32_t* out_ids, cudaStream_t stream);
+
 // cuTensorMapEncodeTiled (PFN_cuTensorMapEncodeTiled_v12000), or null.
 void* tensor_map_encoder();
 
