@@ -344,7 +344,6 @@ __device__ __forceinline__ uint64_t anc_window(const uint64_t (&a)[4], int o) {
 // more than 2^8, so P stays below 2^8 and O is rarely touched.
 __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem, Bars* bar, int warp, int lane) {
   const int q = warp & 3, h = lane >> 4, i = lane & 15;
-  const int T = p.t.T;
   const uint32_t la = static_cast<uint32_t>(32 * q) << 16;
   int g = 0, k = 0;
   for (int kk = 0;; ++kk) {
