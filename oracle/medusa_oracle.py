@@ -239,6 +239,59 @@ def tree_attention(tree, q, k_cache, v_cache, seq_lens, scale):
     return out
 
 
+# S5 split along the cached prefix (several ranks share one slice's keys).
+# The pages have no counterpart: this is the library's multi-GPU option.  Its
+# definition is the restriction of tree_attention_slice to a key subset, and
+# putting the parts back together is the log-sum-exp identity.
+
+
+def attention_window(G: int, r: int, L_b: int):
+    """Prefix rows [lo, hi) of rank r of G: lo = floor(L_b r / G), hi = floor(L_b (r+1) / G).
+    The tree's own rows belong to the last rank only."""
+    return (L_b * r) // G, (L_b * (r + 1)) // G
+
+
+def tree_attention_window_slice(tree, q_slice, k_slice, v_slice, L_b: int, scale: float,
+                                lo: int, hi: int, with_tree: bool):
+    """Attention of the T tree queries over prefix rows lo..hi-1 and, when with_tree, the tree
+    rows each node may see (itself and its ancestors).  Returns (O [T, hd] normalised over that
+    set, lse [T] = ln sum exp(scale q.k) over it); a query with no key gets O = 0, lse = -inf."""
+    T = tree["T"]
+    q = np.asarray(q_slice, dtype=np.float64)
+    kk = np.asarray(k_slice, dtype=np.float64)
+    vv = np.asarray(v_slice, dtype=np.float64)
+    out = np.zeros((T, q.shape[1]), dtype=np.float64)
+    lse = np.full(T, -np.inf)
+    for i in range(T):
+        rows = list(range(lo, hi))
+        if with_tree:
+            rows += [L_b + j for j in range(T) if tree["anc"][i, j]]
+        if not rows:
+            continue
+        s = (kk[rows] @ q[i]) * scale
+        m = s.max()
+        w = np.exp(s - m)
+        lse[i] = m + np.log(w.sum())
+        out[i] = (w / w.sum()) @ vv[rows]
+    return out, lse
+
+
+def combine_partials(outs, lses):
+    """Attention over the union of G disjoint key sets from each set's (O_r, lse_r):
+    lse = ln sum_r exp(lse_r) and O = sum_r exp(lse_r - lse) O_r.
+    outs [G, ..., hd], lses [G, ...]; entries with lse_r = -inf contribute nothing."""
+    outs = np.asarray(outs, dtype=np.float64)
+    lses = np.asarray(lses, dtype=np.float64)
+    m = lses.max(axis=0)
+    safe = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lses - safe)                      # exp(-inf) = 0
+    tot = w.sum(axis=0)
+    with np.errstate(divide="ignore"):
+        lse = np.where(tot > 0, safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    wn = np.where(tot > 0, w / np.where(tot > 0, tot, 1.0), 0.0)
+    return (wn[..., None] * outs).sum(axis=0), lse
+
+
 # ----------------------------------------------------------------------------
 # S6: posterior  [P3 evaluate_posterior (posterior_threshold, posterior_alpha);
 #     P4 key points (typical acceptance), case 1 step 4 (longest acceptable

@@ -1,0 +1,75 @@
+"""Pins for the oracle of tree attention split along the cached prefix.
+
+The split is the library's multi-GPU option (no counterpart on the pages):
+rank r of G attends to its window of prefix rows (the last rank also to the
+tree's own rows) and returns (O_r, lse_r); the log-sum-exp identity puts the
+parts back together.  Pinned here against the already pinned unsplit oracle
+(the identity must reproduce it for any G), closed forms (equal scores give
+the mean of V and ln(n); a single key gives its own V and score), and the
+window bookkeeping."""
+
+import numpy as np
+import pytest
+
+import oracle.medusa_oracle as O
+
+WORKED = [(0,), (1,), (0, 0), (0, 1), (1, 0), (1, 1)]
+
+
+def _inputs(T, L, hd, seed=0):
+    rng = np.random.default_rng(seed)
+    return (rng.normal(size=(T, hd)), rng.normal(size=(L + T + 5, hd)), rng.normal(size=(L + T + 5, hd)))
+
+
+@pytest.mark.parametrize("L,G", [(1024, 1), (1024, 8), (200, 3), (7, 7), (5, 3), (0, 1)])
+def test_windows_partition_the_prefix(L, G):
+    wins = [O.attention_window(G, r, L) for r in range(G)]
+    assert wins[0][0] == 0 and wins[-1][1] == L
+    for (a, b), (c, _) in zip(wins, wins[1:]):
+        assert b == c and a <= b
+    sizes = [b - a for a, b in wins]
+    assert max(sizes) - min(sizes) <= 1
+
+
+@pytest.mark.parametrize("choices,K,topk,L", [(WORKED, 2, 2, 37), (O.ranksum_choices(5, 10, 40), 5, 10, 300),
+                                              (O.ranksum_choices(5, 10, 40), 5, 10, 3), ([], 3, 2, 64)])
+@pytest.mark.parametrize("G", [1, 2, 3, 7])
+def test_combined_windows_equal_the_unsplit_attention(choices, K, topk, L, G):
+    tr = O.tree_tables(choices, K, topk)
+    hd = 32
+    q, k, v = _inputs(tr["T"], L, hd, seed=G)
+    scale = O.attention_scale(hd)
+    ref = O.tree_attention_slice(tr, q, k, v, L, scale)
+    outs, lses = [], []
+    for r in range(G):
+        lo, hi = O.attention_window(G, r, L)
+        o, l = O.tree_attention_window_slice(tr, q, k, v, L, scale, lo, hi, with_tree=(r == G - 1))
+        outs.append(o)
+        lses.append(l)
+    got, lse = O.combine_partials(np.stack(outs), np.stack(lses))
+    assert np.allclose(got, ref, atol=1e-12, rtol=1e-12)
+    o1, l1 = O.tree_attention_window_slice(tr, q, k, v, L, scale, 0, L, with_tree=True)
+    assert np.allclose(lse, l1, atol=1e-12) and np.allclose(o1, ref, atol=1e-12)
+
+
+def test_window_closed_forms():
+    tr = O.tree_tables(O.ranksum_choices(3, 2, 6), 3, 2)
+    T, L, hd = tr["T"], 20, 16
+    _, k, v = _inputs(T, L, hd, seed=5)
+    # q = 0: every score is 0, so lse = ln(number of keys) and O is the mean of their V rows
+    q0 = np.zeros((T, hd))
+    o, lse = O.tree_attention_window_slice(tr, q0, k, v, L, 0.25, 4, 13, with_tree=True)
+    for i in range(T):
+        rows = list(range(4, 13)) + [L + j for j in range(T) if tr["anc"][i, j]]
+        assert np.isclose(lse[i], np.log(len(rows)), atol=1e-14)
+        assert np.allclose(o[i], v[rows].mean(axis=0), atol=1e-14)
+    # one prefix key and no tree rows: O is that key's V row, lse its scaled score
+    q = np.random.default_rng(9).normal(size=(T, hd))
+    o, lse = O.tree_attention_window_slice(tr, q, k, v, L, 0.3, 7, 8, with_tree=False)
+    assert np.allclose(o, np.broadcast_to(v[7], o.shape), atol=0)
+    assert np.allclose(lse, 0.3 * (q @ k[7]), atol=1e-14)
+    # an empty window: O = 0, lse = -inf, and it contributes nothing when combined
+    o_e, l_e = O.tree_attention_window_slice(tr, q, k, v, L, 0.3, 5, 5, with_tree=False)
+    assert not o_e.any() and np.all(l_e == -np.inf)
+    got, l2 = O.combine_partials(np.stack([o_e, o]), np.stack([l_e, lse]))
+    assert np.allclose(got, o, atol=0) and np.allclose(l2, lse, atol=0)
