@@ -24,6 +24,10 @@
  *   S3 over G ranks  medusa_topk_merge  the global top-k from the top-k lists
  *                                   of G vocabulary shards (rows of Wout
  *                                   split across ranks, lists all-gathered).
+ *   S5 over G ranks  medusa_tree_attention_split, medusa_attention_combine
+ *                                   attention over one window of the cached
+ *                                   prefix per rank, then the log-sum-exp
+ *                                   combine of the gathered partials.
  *   medusa_step                     S1..S7 in order on one stream.
  *
  * Conventions shared by every call:
@@ -243,6 +247,41 @@ medusa_status_t medusa_tree_attention(const medusa_tree_t* tree, int layers, int
                                       const int32_t* seq_lens, float scale, void* out,
                                       void* workspace, size_t workspace_bytes,
                                       cudaStream_t stream);
+
+/* S5 split along the cached prefix over G ranks.  Caches keep the layout of
+ * medusa_tree_attention ([layers, B, H, Lcap, hd]); a rank's call uses only
+ * the rows of its own window, so the other rows may hold anything (they are
+ * read past a window's end only to fill a tile, and masked).  Rank `rank` attends to
+ * prefix rows [lo, hi) = [floor(L r / G), floor(L (r+1) / G)) of every slice
+ * (L = seq_lens[b]) and, when rank = G - 1, to the tree rows node i may see
+ * (as medusa_tree_attention), and writes
+ *   out [layers, B, T, H, hd] fp32: attention over that window (normalised
+ *                over the window alone)
+ *   lse [layers, B, T, H] fp32: ln sum exp(scale q.k) over the window.
+ * medusa_attention_combine over the G ranks' (out, lse), gathered in rank
+ * order, gives medusa_tree_attention's output.  Supported: bf16, hd = 128,
+ * trees of at most 64 tokens (else MEDUSA_ERR_UNSUPPORTED).  Every
+ * seq_lens[b] must be >= G (an empty window sets MEDUSA_ERR_DEVICE_CHECK and
+ * leaves that slice unwritten), as must seq_lens[b] + T <= Lcap.
+ * 1 <= G <= MEDUSA_MAX_SHARDS, 0 <= rank < G.  No workspace.
+ * The pages have no counterpart: the split is this library's multi-GPU
+ * option; the combine is the log-sum-exp identity. */
+medusa_status_t medusa_tree_attention_split(const medusa_tree_t* tree, int layers, int B, int H, int hd,
+                                            medusa_dtype_t dtype, const void* q, const void* k_cache,
+                                            const void* v_cache, int Lcap, const int32_t* seq_lens,
+                                            float scale, int rank, int G, float* out, float* lse,
+                                            cudaStream_t stream);
+
+/* Attention over the union of G disjoint key windows from each window's
+ * normalised output and lse:
+ *   outs [G, rows, hd] fp32, lses [G, rows] fp32 (rows = layers*B*T*H)
+ *   out [rows, hd] = sum_g exp(lse_g - lse) outs[g],  lse = ln sum_g exp(lse_g)
+ *   lse_out [rows] (may be NULL) receives lse.
+ * A row whose every lse_g is -inf gets out = 0, lse = -inf.  hd a multiple
+ * of 4 in [4, 1024]; outs and out 16-byte aligned; out must not overlap
+ * outs.  1 <= G <= MEDUSA_MAX_SHARDS. */
+medusa_status_t medusa_attention_combine(int G, int64_t rows, int hd, const float* outs, const float* lses,
+                                         float* out, float* lse_out, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* S6: posterior                                                             */

@@ -52,6 +52,7 @@ EXPORTED = [
     "medusa_heads_workspace_size", "medusa_heads_topk", "medusa_heads_topk_noalloc",
     "medusa_topk_merge", "medusa_build_tree",
     "medusa_attention_workspace_size", "medusa_tree_attention",
+    "medusa_tree_attention_split", "medusa_attention_combine",
     "medusa_posterior_workspace_size", "medusa_evaluate_posterior",
     "medusa_accept_kv",
     "medusa_step_workspace_size", "medusa_step",
@@ -111,6 +112,9 @@ _sig("medusa_build_tree", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp])
 _sig("medusa_attention_workspace_size", _sz, [_vp, _i32, _i32, _i32, _i32, _i32])
 _sig("medusa_tree_attention", _i32,
      [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _f32, _vp, _vp, _sz, _vp])
+_sig("medusa_tree_attention_split", _i32,
+     [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _f32, _i32, _i32, _vp, _vp, _vp])
+_sig("medusa_attention_combine", _i32, [_i32, ctypes.c_int64, _i32, _vp, _vp, _vp, _vp, _vp])
 _sig("medusa_posterior_workspace_size", _sz, [_vp, _i32])
 _sig("medusa_evaluate_posterior", _i32,
      [_vp, _i32, _i32, _vp, _vp, _i32, _f32, _f32, _f32, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
@@ -282,6 +286,25 @@ def medusa_tree_attention(tree: Tree, q, k_cache, v_cache, seq_lens, scale, out,
     _check(_lib.medusa_tree_attention(tree.handle, layers, B, H, hd, _dtype(q), _p(q), _p(k_cache),
                                       _p(v_cache), Lcap, _p(seq_lens), float(scale), _p(out), _p(ws),
                                       0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def medusa_tree_attention_split(tree: Tree, q, k_cache, v_cache, seq_lens, scale, rank: int, G: int, out, lse,
+                                stream=None):
+    """Attention over window `rank` of G of each slice's cached prefix (the tree rows with the last
+    window): out [layers, B, T, H, hd] normalised over the window, lse [layers, B, T, H]."""
+    layers, B, T, H, hd = q.shape
+    Lcap = k_cache.shape[3]
+    _check(_lib.medusa_tree_attention_split(tree.handle, layers, B, H, hd, _dtype(q), _p(q), _p(k_cache),
+                                            _p(v_cache), Lcap, _p(seq_lens), float(scale), int(rank), int(G),
+                                            _p(out), _p(lse), _stream(stream)))
+
+
+def medusa_attention_combine(outs, lses, out, lse_out=None, stream=None):
+    """outs [G, ..., hd], lses [G, ...] (the same leading shape) -> out [..., hd], lse_out [...]."""
+    G, hd = outs.shape[0], outs.shape[-1]
+    rows = lses[0].numel()
+    _check(_lib.medusa_attention_combine(G, rows, hd, _p(outs), _p(lses), _p(out), _p(lse_out),
+                                         _stream(stream)))
 
 
 def medusa_posterior_workspace_size(tree: Tree, B) -> int:

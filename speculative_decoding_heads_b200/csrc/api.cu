@@ -224,6 +224,37 @@ extern "C" medusa_status_t medusa_tree_attention(const medusa_tree_t* tree, int 
                           workspace, stream);
 }
 
+extern "C" medusa_status_t medusa_tree_attention_split(const medusa_tree_t* tree, int layers, int B, int H,
+                                                       int hd, medusa_dtype_t dtype, const void* q,
+                                                       const void* k_cache, const void* v_cache, int Lcap,
+                                                       const int32_t* seq_lens, float scale, int rank, int G,
+                                                       float* out, float* lse, cudaStream_t stream) {
+  const char* fn = "medusa_tree_attention_split";
+  medusa_status_t st =
+      check_attention(tree, layers, B, H, hd, dtype, q, k_cache, v_cache, Lcap, seq_lens, scale, out);
+  if (st != MEDUSA_OK) return st;
+  if (!lse) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (G < 1 || G > MEDUSA_MAX_SHARDS || rank < 0 || rank >= G)
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": rank or G out of range");
+  return launch_attention_split(tree->dev, layers, B, H, hd, dtype, q, k_cache, v_cache, Lcap, seq_lens, scale, rank,
+                                G, out, lse, stream);
+}
+
+extern "C" medusa_status_t medusa_attention_combine(int G, int64_t rows, int hd, const float* outs,
+                                                    const float* lses, float* out, float* lse_out,
+                                                    cudaStream_t stream) {
+  const char* fn = "medusa_attention_combine";
+  if (!outs || !lses || !out) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (G < 1 || G > MEDUSA_MAX_SHARDS || rows < 1 || hd < 4 || hd > 1024 || hd % 4 != 0)
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": G, rows or hd out of range");
+  if (!aligned16(outs) || !aligned16(out)) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": misaligned pointer");
+  const uintptr_t o0 = reinterpret_cast<uintptr_t>(out), o1 = o0 + static_cast<uintptr_t>(rows) * hd * 4;
+  const uintptr_t i0 = reinterpret_cast<uintptr_t>(outs), i1 = i0 + static_cast<uintptr_t>(rows) * hd * 4 * G;
+  if (o0 < i1 && i0 < o1) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": out overlaps outs");
+  if (sm_count() <= 0) return fail(MEDUSA_ERR_CUDA, std::string(fn) + ": no usable CUDA device");
+  return launch_attention_combine(G, static_cast<size_t>(rows), hd, outs, lses, out, lse_out, stream);
+}
+
 extern "C" size_t medusa_posterior_workspace_size(const medusa_tree_t* tree, int B) {
   if (!tree || B < 1) return 0;
   medusa::TreeDev t{};

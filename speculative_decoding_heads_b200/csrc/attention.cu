@@ -102,7 +102,65 @@ constexpr int kHd = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
 
+// The log-sum-exp identity: attention over a union of disjoint key sets from
+// each set's normalised output O_g and lse_g = ln sum exp(scale q.k):
+// out = sum_g exp(lse_g - lse) O_g with lse = ln sum_g exp(lse_g).  One thread
+// per 4 output values; every O_g is read once.
+__global__ void attention_combine_kernel(int G, size_t rows, int hd4, const float4* outs, const float* lses,
+                                         float4* out, float* lse_out) {
+  const size_t n = rows * static_cast<size_t>(hd4);
+  for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < n;
+       idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t row = idx / hd4;
+    float m = -INFINITY;
+    for (int g = 0; g < G; ++g) m = fmaxf(m, lses[g * rows + row]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float tot = 0.f;
+    if (m > -INFINITY) {                 // otherwise no window held a key: O = 0
+      for (int g = 0; g < G; ++g) {
+        const float w = expf(lses[g * rows + row] - m);
+        const float4 o = outs[g * n + idx];
+        tot += w;
+        acc.x += w * o.x;
+        acc.y += w * o.y;
+        acc.z += w * o.z;
+        acc.w += w * o.w;
+      }
+      const float inv = 1.f / tot;
+      acc.x *= inv;
+      acc.y *= inv;
+      acc.z *= inv;
+      acc.w *= inv;
+    }
+    out[idx] = acc;
+    if (lse_out != nullptr && idx % hd4 == 0) lse_out[row] = m > -INFINITY ? m + logf(tot) : -INFINITY;
+  }
+}
+
 }  // namespace
+
+medusa_status_t launch_attention_split(const TreeDev& t, int layers, int B, int H, int hd, medusa_dtype_t dtype,
+                                       const void* q, const void* k_cache, const void* v_cache, int Lcap,
+                                       const int32_t* seq_lens, float scale, int rank, int G, float* out,
+                                       float* lse, cudaStream_t stream) {
+  if (dtype != MEDUSA_BF16 || hd != kHd || t.T > 64)
+    return fail(MEDUSA_ERR_UNSUPPORTED,
+                "medusa_tree_attention_split: the split runs on the bf16, hd 128 kernel for trees of at most 64 tokens");
+  return launch_attention_tc64(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, scale * kLog2e, out,
+                               device_status_ptr(), stream, false, 0, t.T, rank, G, lse);
+}
+
+medusa_status_t launch_attention_combine(int G, size_t rows, int hd, const float* outs, const float* lses,
+                                         float* out, float* lse_out, cudaStream_t stream) {
+  const size_t n = rows * static_cast<size_t>(hd / 4);
+  const size_t want = (n + 255) / 256;
+  const size_t cap = static_cast<size_t>(sm_count() > 0 ? sm_count() : 1) * 16;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  attention_combine_kernel<<<grid, 256, 0, stream>>>(G, rows, hd / 4, reinterpret_cast<const float4*>(outs), lses,
+                                                     reinterpret_cast<float4*>(out), lse_out);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_attention_combine", e);
+}
 
 size_t attention_workspace_bytes(const TreeDev& t, int layers, int B, int H, int hd, medusa_dtype_t dtype) {
   (void)t;

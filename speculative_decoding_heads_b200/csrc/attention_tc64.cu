@@ -59,6 +59,7 @@ __device__ __forceinline__ uint32_t col_p(int buf) { return 128u + 64u * buf; } 
 __device__ __forceinline__ uint32_t col_o(int buf) { return 256u + 128u * buf; }  // 128 fp32 columns
 constexpr uint32_t kLaneHalf = 16u << 16;      // TMEM address offset of lane 16
 constexpr float kRescaleLog2 = 8.0f;
+constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kLenTab = 160;                   // prefix lengths of a CTA's first slices, in shared memory
 // The polling loops of the producer and the MMA issuer give up after this
 // many SM cycles without progress (about 2 s at 2 GHz); the SM cycle counter
@@ -90,6 +91,9 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 struct Slice {
   int slice, lb, e, L, n, steps;
   int item, grp;   // work item index; query rows 64 grp .. 64 grp + 63
+  int k0;          // first key row of this launch's window (0 unless split along L)
+  int plim;        // prefix keys below plim are visible
+  int last;        // the window holds the tree's own rows (the last rank of a split)
 };
 
 struct Params {
@@ -102,12 +106,15 @@ struct Params {
   float* out;
   int* status;
   int kv_one_box;   // 1: one 32 KB TMA box per tile (4-D map), 0: two 16 KB boxes
+  int split_r, split_G;   // this launch is window split_r of split_G along the prefix (0, 1: all of it)
+  float* lse;             // [layers, B, T, H] natural-log sum of exp(scale q.k) over the window, or null
 };
 
 // Work item kk of this CTA; steps = 0 when it does not exist or fails its
 // check (slice >= total marks the end).  The prefix length comes from the
 // shared table for the first kLenTab items (no global load on any role's
 // critical path at an item boundary).
+template <bool kSplit>
 __device__ __forceinline__ Slice slice_info(int kk, const Params& p, const int* lens) {
   Slice s{};
   s.item = blockIdx.x + kk * gridDim.x;
@@ -120,15 +127,31 @@ __device__ __forceinline__ Slice slice_info(int kk, const Params& p, const int* 
   s.e = s.slice % p.H;
   s.lb = s.slice / p.H;
   s.L = kk < kLenTab ? lens[kk] : p.seq_lens[s.lb % p.B];
-  s.n = s.L + p.t.T;
-  s.steps = (s.L >= 0 && s.n <= p.Lcap) ? (s.n + kStep - 1) / kStep : 0;
+  if constexpr (kSplit) {
+    // Window split_r of split_G: prefix rows [L r / G, L (r+1) / G), and the
+    // tree's own rows with the last window (contiguous with its prefix rows).
+    const int r = p.split_r, G = p.split_G;
+    const long long L = s.L;
+    s.last = r == G - 1;
+    s.k0 = static_cast<int>(L * r / G);
+    const int hi = static_cast<int>(L * (r + 1) / G);
+    s.plim = s.last ? s.L : hi;
+    s.n = s.last ? s.L + p.t.T - s.k0 : hi - s.k0;
+  } else {
+    s.last = 1;
+    s.k0 = 0;
+    s.plim = s.L;
+    s.n = s.L + p.t.T;
+  }
+  s.steps = (s.L >= 0 && s.L + p.t.T <= p.Lcap && s.n > 0) ? (s.n + kStep - 1) / kStep : 0;
   return s;
 }
 
 // First slice at or after kk that passes its check (kk is advanced to it).
+template <bool kSplit>
 __device__ __forceinline__ Slice seek(int& kk, const Params& p, const int* lens) {
-  Slice s = slice_info(kk, p, lens);
-  while (s.slice < p.total && s.steps == 0) s = slice_info(++kk, p, lens);
+  Slice s = slice_info<kSplit>(kk, p, lens);
+  while (s.slice < p.total && s.steps == 0) s = slice_info<kSplit>(++kk, p, lens);
   return s;
 }
 
@@ -171,13 +194,14 @@ __device__ __forceinline__ int step_keys(const Slice& s, int t) {
 // ---- TMA producer (one thread) ----------------------------------------------
 // Three streams, each issued as soon as its buffer is free: Q rows of every
 // slice, K tiles and V tiles of every step.
+template <bool kSplit>
 __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map, const CUtensorMap* v_map,
                              const Params& p, unsigned char* smem, Bars* bar) {
   tc::prefetch_tensormap(q_map);
   tc::prefetch_tensormap(k_map);
   tc::prefetch_tensormap(v_map);
   int kkq = 0, kkk = 0, kkv = 0;
-  Slice sq = seek(kkq, p, bar->lens), sk = seek(kkk, p, bar->lens), sv = seek(kkv, p, bar->lens);
+  Slice sq = seek<kSplit>(kkq, p, bar->lens), sk = seek<kSplit>(kkk, p, bar->lens), sv = seek<kSplit>(kkv, p, bar->lens);
   int nq = 0, gk = 0, gv = 0, tk = 0, tv = 0;     // loads issued; step within slice
   long long last = clock64();
   while ((sq.slice < p.total || sk.slice < p.total || sv.slice < p.total) && !bar->abort) {
@@ -190,7 +214,7 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
       tc::tma_load_4d(qd + kQHalf, q_map, 64, sq.e, p.row_lo + kRows * sq.grp, sq.lb, fb);
       ++nq;
       ++kkq;
-      sq = seek(kkq, p, bar->lens);
+      sq = seek<kSplit>(kkq, p, bar->lens);
       progressed = true;
     }
     for (int which = 0; which < 2; ++which) {
@@ -207,16 +231,16 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
       const CUtensorMap* m = which == 0 ? k_map : v_map;
       mbar_arrive_expect_tx(fb, kTile);
       if (p.kv_one_box) {
-        tc::tma_load_4d(d, m, 0, t * kStep, 0, s.slice, fb);
+        tc::tma_load_4d(d, m, 0, s.k0 + t * kStep, 0, s.slice, fb);
       } else {
-        tc::tma_load_3d(d, m, 0, t * kStep, s.slice, fb);
-        tc::tma_load_3d(d + kHalfTile, m, 64, t * kStep, s.slice, fb);
+        tc::tma_load_3d(d, m, 0, s.k0 + t * kStep, s.slice, fb);
+        tc::tma_load_3d(d + kHalfTile, m, 64, s.k0 + t * kStep, s.slice, fb);
       }
       ++g;
       if (++t == s.steps) {
         t = 0;
         ++kk;
-        s = seek(kk, p, bar->lens);
+        s = seek<kSplit>(kk, p, bar->lens);
       }
       progressed = true;
     }
@@ -254,11 +278,12 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
 // issued as soon as their inputs are ready: S(g) needs K(g) and its TMEM lane
 // half back from the softmax of step g - 2, not P V(g - 1), so the products
 // of later steps run while the softmax of this one computes.
+template <bool kSplit>
 __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* bar) {
   constexpr uint32_t idS = tc::idesc_bf16_f32(64, kStep, 0);
   constexpr uint32_t idO = tc::idesc_bf16_f32(128, kHd, 1);
   int kks = 0, kkp = 0;
-  Slice ss = seek(kks, p, bar->lens), sp = seek(kkp, p, bar->lens);
+  Slice ss = seek<kSplit>(kks, p, bar->lens), sp = seek<kSplit>(kkp, p, bar->lens);
   int gs = 0, ts = 0, ks = 0;     // S cursor: global step, step in slice, slice count
   int gp = 0, tp = 0, kp = 0;     // P V cursor
   long long last = clock64();
@@ -285,7 +310,7 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
         ts = 0;
         ++ks;
         ++kks;
-        ss = seek(kks, p, bar->lens);
+        ss = seek<kSplit>(kks, p, bar->lens);
       }
       progressed = true;
     }
@@ -311,7 +336,7 @@ __device__ void run_mma(const Params& p, uint32_t sbase, uint32_t tmem, Bars* ba
         tp = 0;
         ++kp;
         ++kkp;
-        sp = seek(kkp, p, bar->lens);
+        sp = seek<kSplit>(kkp, p, bar->lens);
       }
       progressed = true;
     }
@@ -342,12 +367,13 @@ __device__ __forceinline__ uint64_t anc_window(const uint64_t (&a)[4], int o) {
 // Online softmax in the log2 domain with a lazy reference: the running
 // maximum moves (and O is rescaled) only when a step's maximum exceeds it by
 // more than 2^8, so P stays below 2^8 and O is rarely touched.
+template <bool kSplit>
 __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem, Bars* bar, int warp, int lane) {
   const int q = warp & 3, h = lane >> 4, i = lane & 15;
   const uint32_t la = static_cast<uint32_t>(32 * q) << 16;
   int g = 0, k = 0;
   for (int kk = 0;; ++kk) {
-    const Slice s = slice_info(kk, p, bar->lens);
+    const Slice s = slice_info<kSplit>(kk, p, bar->lens);
     if (s.slice >= p.total) break;
     if (s.steps == 0) {
       if (lane == 0 && q == 0) set_device_status(p.status, MEDUSA_ERR_DEVICE_CHECK, kDetailAttnSeqLen);
@@ -374,18 +400,19 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&bar->s_free[g & 1]);
 
-      const int key0 = t * kStep + h * 64;
+      const int key0 = s.k0 + t * kStep + h * 64;      // key row of sv[0]
       // Eight independent partial maxima (the maximum does not depend on the
       // order; the short chains keep the one warp per scheduler busy).
       float mx[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) mx[j] = -INFINITY;
-      if (key0 + 64 > s.L) {
-        // Allowed keys of this window as a bit mask: the cached prefix, then
-        // the tree tokens that are ancestors of (or equal to) row r.
-        const int d = s.L - key0;                    // prefix keys in the window (< 64)
+      if (key0 + 64 > s.plim) {
+        // Allowed keys of these 64 as a bit mask: the visible prefix, then
+        // (last window only) the tree tokens that are ancestors of (or equal
+        // to) row r.
+        const int d = s.plim - key0;                 // visible prefix keys among them (< 64)
         uint64_t m = d > 0 ? (1ull << d) - 1ull : 0ull;
-        m |= d >= 0 ? (anc[0] << d) : anc_window(anc, -d);
+        if (s.last) m |= d >= 0 ? (anc[0] << d) : anc_window(anc, -d);
         const uint32_t mlo = static_cast<uint32_t>(m), mhi = static_cast<uint32_t>(m >> 32);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -483,6 +510,9 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
         if (k >= 2 && !wait_bar(&bar->o_free[k & 1], ((k >> 1) - 1) & 1, bar, p.status)) return;
         const float total = lsum + __shfl_xor_sync(0xffffffffu, lsum, 16);
         if (h == 0) bar->lsum[k & 1][16 * q + i] = total;
+        // ln sum exp(scale q.k) = ln 2 (m + log2 total), m the log2-domain reference.
+        if (kSplit && p.lse != nullptr && h == 0 && r < p.row_hi)
+          p.lse[(static_cast<size_t>(s.lb) * p.t.T + r) * p.H + s.e] = (mref + log2f(total)) * kLn2;
         tc::mbar_arrive(&bar->l_ready[k & 1]);
       }
     }
@@ -492,13 +522,14 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
 
 // ---- epilogue (warps 2, 3, 8, 9) ------------------------------------------------
 // out[query] = (O(high-part lanes) + O(remainder lanes)) / row sum, in fp32.
+template <bool kSplit>
 __device__ void run_epilogue(const Params& p, uint32_t tmem, Bars* bar, int warp, int lane) {
   const int q = warp & 3, h = lane >> 4, i = lane & 15;
   const int T = p.t.T;
   const uint32_t la = static_cast<uint32_t>(32 * q) << 16;
   int k = 0;
   for (int kk = 0;; ++kk) {
-    const Slice s = seek(kk, p, bar->lens);
+    const Slice s = seek<kSplit>(kk, p, bar->lens);
     if (s.slice >= p.total) break;
     if (!wait_bar(&bar->l_ready[k & 1], (k >> 1) & 1, bar, p.status)) return;
     if (!wait_bar(&bar->o_full[k & 1], (k >> 1) & 1, bar, p.status)) return;
@@ -528,6 +559,7 @@ __device__ void run_epilogue(const Params& p, uint32_t tmem, Bars* bar, int warp
   }
 }
 
+template <bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     tree_attn_tc64(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                    const __grid_constant__ CUtensorMap v_map, const Params p) {
@@ -573,13 +605,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   allow_dependents();
 
   if (warp == 0) {
-    if (lane == 0) run_producer(&q_map, &k_map, &v_map, p, smem, bar);
+    if (lane == 0) run_producer<kSplit>(&q_map, &k_map, &v_map, p, smem, bar);
   } else if (warp == 1) {
-    if (lane == 0) run_mma(p, smem_u32(smem), tmem, bar);
+    if (lane == 0) run_mma<kSplit>(p, smem_u32(smem), tmem, bar);
   } else if (warp >= 4 && warp < 8) {
-    run_softmax(p, smem, tmem, bar, warp, lane);
+    run_softmax<kSplit>(p, smem, tmem, bar, warp, lane);
   } else {
-    run_epilogue(p, tmem, bar, warp, lane);
+    run_epilogue<kSplit>(p, tmem, bar, warp, lane);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -616,7 +648,7 @@ void* tensor_map_encoder() {
 medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H, const void* q,
                                       const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
                                       float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl,
-                                      int row_lo, int row_hi) {
+                                      int row_lo, int row_hi, int split_r, int split_G, float* lse) {
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!enc) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: cuTensorMapEncodeTiled unavailable");
   if (t.T > 4 * kRows || t.W > 4) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: more than 256 tree tokens");
@@ -681,9 +713,16 @@ medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H
   prm.out = out;
   prm.status = status;
   prm.kv_one_box = one_box;
+  prm.split_r = split_r;
+  prm.split_G = split_G;
+  prm.lse = lse;
   const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
-  cudaError_t e = cudaFuncSetAttribute(tree_attn_tc64, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e == cudaSuccess) e = launch_kernel(tree_attn_tc64, dim3(grid), dim3(kThreads), kSmemBytes, stream, pdl, qm, km, vm, prm);
+  // The split instantiation (window bookkeeping, lse store) only when asked
+  // for: the whole-prefix kernel keeps the plain bookkeeping.
+  const bool split = split_G > 1 || lse != nullptr;
+  auto kernel = split ? tree_attn_tc64<true> : tree_attn_tc64<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e == cudaSuccess) e = launch_kernel(kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, pdl, qm, km, vm, prm);
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_tree_attention: tcgen05 launch", e);
 }
 

@@ -90,16 +90,30 @@ medusa_status_t launch_accept_kv(const TreeDev& t, int layers, int B, int H, int
                                  int32_t* seq_lens, const int32_t* best_path,
                                  const int32_t* accept_len, cudaStream_t stream, bool pdl = false);
 
+// Tree attention over window `rank` of G of each slice's cached prefix (the
+// tree's rows with the last window), writing the window's normalised output
+// and its lse; then the combine of G such partials.
+medusa_status_t launch_attention_split(const TreeDev& t, int layers, int B, int H, int hd, medusa_dtype_t dtype,
+                                       const void* q, const void* k_cache, const void* v_cache, int Lcap,
+                                       const int32_t* seq_lens, float scale, int rank, int G, float* out,
+                                       float* lse, cudaStream_t stream);
+medusa_status_t launch_attention_combine(int G, size_t rows, int hd, const float* outs, const float* lses,
+                                         float* out, float* lse_out, cudaStream_t stream);
+
 medusa_status_t launch_topk_merge(const float* vals, const int32_t* ids, const int32_t* row0, int G, int B,
                                   int K, int topk, float* out_vals, int32_t* out_ids, cudaStream_t stream);
 
 // cuTensorMapEncodeTiled (PFN_cuTensorMapEncodeTiled_v12000), or null.
 void* tensor_map_encoder();
 
+// split_r / split_G: attend only to window split_r of split_G of each slice's
+// cached prefix (the tree's own rows with the last window); lse, if not null,
+// receives ln sum exp(scale q.k) over the window per (layer, seq, node, head).
 medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H, const void* q,
                                       const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
                                       float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl,
-                                      int row_lo, int row_hi);
+                                      int row_lo, int row_hi, int split_r = 0, int split_G = 1,
+                                      float* lse = nullptr);
 
 medusa_status_t launch_attention_tc128(const TreeDev& t, int layers, int B, int H, const void* q,
                                        const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,

@@ -10,6 +10,11 @@ the merge kernel selects the global top-k from the G·k candidates of each
 (sequence, head).  The heads kernel computes each logit the same way for any
 V, so the merged lists are those of the unsplit call bit for bit.
 
+Tree attention can split the same way along each slice's cached prefix:
+rank r attends to its window of prefix rows (the last rank also to the tree
+rows), the ranks all-gather their (output, lse) partials, and the log-sum-exp
+combine gives the unsplit result (tree_attention_sharded).
+
 Every step runs in the library's kernels; torch.distributed only moves the
 gathered lists (NCCL between GPUs, gloo on the host for the tests).
 """
@@ -19,8 +24,8 @@ from typing import List, Optional, Tuple
 import torch
 import torch.distributed as dist
 
-from . import (MAX_SHARDS, medusa_heads_topk, medusa_heads_workspace_size, medusa_topk_merge,
-               workspace)
+from . import (MAX_SHARDS, medusa_attention_combine, medusa_heads_topk, medusa_heads_workspace_size,
+               medusa_topk_merge, medusa_tree_attention, medusa_tree_attention_split, workspace)
 
 
 def shard_bounds(V: int, G: int) -> List[Tuple[int, int]]:
@@ -84,3 +89,31 @@ def heads_topk_sharded(h: torch.Tensor, W1: torch.Tensor, b1: torch.Tensor, Wout
     out_vals = torch.empty_like(vals)
     medusa_topk_merge(all_vals, all_ids, [b[0] for b in bounds], V, out_vals, out_ids, stream=stream)
     return out_ids, out_vals
+
+
+def tree_attention_sharded(tree, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                           seq_lens: torch.Tensor, scale: float, out: torch.Tensor, group=None, stream=None):
+    """S5 with every slice's cached prefix split over the ranks of `group`: this rank's window
+    (medusa_tree_attention_split), an all-gather of the G partial outputs and lse values, and the
+    combine.  `out` [layers, B, T, H, hd] receives medusa_tree_attention's result on every rank;
+    with one rank (or no process group) it is that call.  Each rank needs only its window's rows
+    of the caches (and the last rank the tree rows), in the full [.., Lcap, hd] layout."""
+    G = dist.get_world_size(group) if dist.is_initialized() else 1
+    if G == 1:
+        medusa_tree_attention(tree, q, k_cache, v_cache, seq_lens, scale, out, stream=stream)
+        return out
+    rank = dist.get_rank(group)
+    dev = out.device
+    part = torch.empty_like(out)
+    lse = torch.empty(tuple(out.shape[:-1]), dtype=torch.float32, device=dev)
+    medusa_tree_attention_split(tree, q, k_cache, v_cache, seq_lens, scale, rank, G, part, lse, stream=stream)
+    if stream is not None:
+        torch.cuda.current_stream(dev).wait_stream(stream)
+    all_o = torch.empty((G,) + tuple(out.shape), dtype=torch.float32, device=dev)
+    all_l = torch.empty((G,) + tuple(lse.shape), dtype=torch.float32, device=dev)
+    dist.all_gather(list(all_o.unbind(0)), part, group=group)
+    dist.all_gather(list(all_l.unbind(0)), lse, group=group)
+    if stream is not None:
+        stream.wait_stream(torch.cuda.current_stream(dev))
+    medusa_attention_combine(all_o, all_l, out, stream=stream)
+    return out
