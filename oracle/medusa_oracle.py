@@ -27,7 +27,7 @@ Sources (page title, then section):
   [P5] "基于 Medusa 头的投机解码架构" -- section "技术深度解析" (a chain draft
        that falls back on the first rejected token).
 
-Readings where the pages are silent or disagree (each listed in the design doc):
+Readings where the pages are silent or disagree:
   * one residual block per head, u = h + SiLU(W1 h + b1), then a bias-free
     V x d projection;  Medusa head k (1-based) fills tree depth k;
   * the tree is a set of rank tuples; node (r1..rj) takes head j's

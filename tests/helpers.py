@@ -15,8 +15,9 @@ from synth import inputs as I, workloads as W
 HERE = os.path.dirname(os.path.abspath(__file__))
 SUBSEEDS = os.path.join(HERE, "golden", "subseeds.json")
 
-# Tolerances (BASELINE: head logits 1e-2 relative; attention 2e-3 max-abs for
-# bf16 inputs, 1e-5 for fp32; ids, paths and lengths bit-exact).
+# Tolerances of the verification step's stated accuracy: head logits 1e-2
+# relative; attention 2e-3 max-abs for bf16 inputs, 1e-5 for fp32; ids, paths
+# and lengths bit-exact.
 LOGIT_RTOL = 1e-2
 ATTN_ATOL = {"bf16": 2e-3, "f32": 1e-5}
 
