@@ -1,0 +1,52 @@
+"""The benchmark's JSON line on the host: the reference arm (the oracle,
+timed on the CPU) carries every key the driver reads, with the types and
+the fixed values the contract gives it."""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+REPO = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def line():
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    env.pop("RANK", None)
+    env.pop("WORLD_SIZE", None)
+    r = subprocess.run([sys.executable, os.path.join(REPO, "bench.py"), "--impl", "reference", "--workload",
+                        "tiny_f32", "--steps", "2", "--warmup", "1"], capture_output=True, text=True, env=env,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    return json.loads(lines[0])
+
+
+def test_reference_line_has_every_contract_key(line):
+    for key, typ in [("metric", str), ("value", float), ("unit", str), ("n_gpus", int), ("steps", int),
+                     ("warmup", int), ("ms_per_step", float), ("higher_is_better", bool), ("scaling", str),
+                     ("dtype", str), ("data", str), ("config", dict), ("impl", str), ("cpu_baseline", dict),
+                     ("e2e", dict)]:
+        assert isinstance(line[key], typ), key
+    assert "vs_baseline" in line
+    assert line["impl"] == "reference" and line["n_gpus"] == 1 and line["steps"] == 2 and line["warmup"] == 1
+    assert line["higher_is_better"] is False and line["scaling"] in ("weak", "strong")
+    assert abs(line["ms_per_step"] * 1e3 - line["value"]) <= 1e-6 * line["value"]
+
+
+def test_reference_line_baseline_and_e2e(line):
+    cb, e2e = line["cpu_baseline"], line["e2e"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["unit"] == line["unit"]
+    assert isinstance(cb["sample"], str) and cb["sample"]
+    assert e2e == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_line_config_names_the_workload(line):
+    cfg = line["config"]
+    assert cfg["workload"] == "tiny_f32"
+    assert "model" not in cfg
+    assert "fit in L2" in cfg["l2"]        # 4 MB of inputs: said plainly, not claimed to exceed L2
