@@ -1,0 +1,138 @@
+"""Pins for the oracle of the base model's forward over the tree tokens.
+
+The decisive pin: under the tree mask, every node's output equals an ordinary
+causal forward over the cached prefix plus that node's root-to-leaf path at
+positions L, L+1, ... -- the definition of verifying all candidates in one
+forward.  The causal forward here is written separately, from torch's fp64
+scaled-dot-product attention with a causal mask, so that a wrong mask, a
+wrong position or a wrong cache row fails it.  Closed forms pin RMSNorm,
+RoPE and the SwiGLU feed-forward."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.decoder_oracle as D
+import oracle.medusa_oracle as O
+
+WORKED = [(0,), (1,), (0, 0), (0, 1), (1, 0), (1, 1)]
+
+
+def _layer(rng, Dm, F, s=0.2):
+    return {"attn_norm": 1.0 + 0.1 * rng.normal(size=Dm), "Wq": s * rng.normal(size=(Dm, Dm)),
+            "Wk": s * rng.normal(size=(Dm, Dm)), "Wv": s * rng.normal(size=(Dm, Dm)),
+            "Wo": s * rng.normal(size=(Dm, Dm)), "mlp_norm": 1.0 + 0.1 * rng.normal(size=Dm),
+            "W_gate": s * rng.normal(size=(F, Dm)), "W_up": s * rng.normal(size=(F, Dm)),
+            "W_down": s * rng.normal(size=(Dm, F))}
+
+
+def _rope_ref(x, pos, base=D.ROPE_BASE):
+    """RoPE as complex multiplication: pair (x[i], x[i+hd/2]) times exp(1j pos theta_i)."""
+    hd = x.shape[-1]
+    half = hd // 2
+    theta = base ** (-np.arange(half) * 2.0 / hd)
+    z = (x[..., :half] + 1j * x[..., half:]) * np.exp(1j * np.asarray(pos)[:, None] * theta[None, :])
+    return np.concatenate([z.real, z.imag], axis=-1)
+
+
+def _causal_forward(tokens, embed, layers, k_caches, v_caches, L, H):
+    """A plain causal decoder over a token sequence at positions L.. with a prefix cache."""
+    x = embed[np.asarray(tokens)].astype(np.float64)
+    n, Dm = x.shape
+    hd = Dm // H
+    pos = L + np.arange(n)
+    for li, ly in enumerate(layers):
+        h = D.rms_norm(x, ly["attn_norm"])
+        q = _rope_ref((h @ ly["Wq"].T).reshape(n, H, hd).transpose(1, 0, 2), pos)
+        k = _rope_ref((h @ ly["Wk"].T).reshape(n, H, hd).transpose(1, 0, 2), pos)
+        v = (h @ ly["Wv"].T).reshape(n, H, hd).transpose(1, 0, 2)
+        K = np.concatenate([k_caches[li][:, :L], k], axis=1)
+        V = np.concatenate([v_caches[li][:, :L], v], axis=1)
+        mask = torch.ones(n, L + n, dtype=torch.bool).tril(L)
+        att = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None],
+            attn_mask=mask[None, None])[0].numpy()
+        x = x + att.transpose(1, 0, 2).reshape(n, Dm) @ ly["Wo"].T
+        hm = D.rms_norm(x, ly["mlp_norm"])
+        x = x + (O.silu(hm @ ly["W_gate"].T) * (hm @ ly["W_up"].T)) @ ly["W_down"].T
+    return x
+
+
+@pytest.mark.parametrize("choices,K,topk,L", [(WORKED, 2, 2, 9), (O.ranksum_choices(4, 3, 20), 4, 3, 17),
+                                              (O.ranksum_choices(3, 2, 8), 3, 2, 0)])
+def test_tree_forward_equals_causal_forward_along_every_path(choices, K, topk, L):
+    rng = np.random.default_rng(L + len(choices))
+    tr = O.tree_tables(choices, K, topk)
+    T, Dm, F, H, Vv, nl = tr["T"], 32, 48, 4, 50, 2
+    hd = Dm // H
+    embed = rng.normal(size=(Vv, Dm))
+    layers = [_layer(rng, Dm, F) for _ in range(nl)]
+    tokens = rng.integers(0, Vv, size=T)
+    kcs = [rng.normal(size=(H, L + T + 3, hd)) for _ in range(nl)]
+    vcs = [rng.normal(size=(H, L + T + 3, hd)) for _ in range(nl)]
+    logits, hid, kc_out, _ = D.tree_forward(tr, tokens, embed, layers, np.ones(Dm), rng.normal(size=(Vv, Dm)),
+                                            kcs, vcs, L, H)
+    for p in range(tr["P"]):
+        path = [n for n in tr["retrieve"][p] if n >= 0]
+        ref = _causal_forward(tokens[path], embed, layers, kcs, vcs, L, H)
+        assert np.allclose(hid[path], ref, atol=1e-10, rtol=1e-10), p
+    # the prefix rows of the caches are untouched; the tree rows now hold the tree's keys
+    for li in range(nl):
+        assert np.array_equal(kc_out[li][:, :L], kcs[li][:, :L])
+        assert not np.allclose(kc_out[li][:, L:L + T], kcs[li][:, L:L + T])
+    assert logits.shape == (T, Vv)
+
+
+def test_rms_norm_closed_forms():
+    rng = np.random.default_rng(1)
+    x = rng.normal(size=(5, 64))
+    y = D.rms_norm(x, np.ones(64), eps=0.0)
+    assert np.allclose(np.sqrt((y * y).mean(axis=-1)), 1.0, atol=1e-14)
+    assert np.allclose(D.rms_norm(7.5 * x, np.ones(64), eps=0.0), y, atol=1e-14)
+    w = rng.normal(size=64)
+    assert np.allclose(D.rms_norm(x, w, eps=0.0), y * w, atol=1e-14)
+    assert np.allclose(D.rms_norm(np.full((1, 4), 3.0), np.ones(4), eps=0.0), 1.0)
+
+
+def test_rope_closed_forms():
+    rng = np.random.default_rng(2)
+    hd, n = 16, 7
+    x = rng.normal(size=(n, hd))
+    pos = np.arange(3, 3 + n)
+    y = D.rope(x, pos)
+    assert np.allclose(y, _rope_ref(x, pos), atol=1e-13)
+    assert np.allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), atol=1e-13)
+    assert np.allclose(D.rope(x, np.zeros(n)), x, atol=0)
+    # scores depend only on the position difference
+    qv, kv = rng.normal(size=(1, hd)), rng.normal(size=(1, hd))
+    s1 = D.rope(qv, [11]) @ D.rope(kv, [4]).T
+    s2 = D.rope(qv, [107]) @ D.rope(kv, [100]).T
+    assert np.allclose(s1, s2, atol=1e-12)
+    # the first pair turns by exactly pos radians (theta_0 = 1)
+    e0 = np.zeros((1, hd))
+    e0[0, 0] = 1.0
+    r = D.rope(e0, [0.5])
+    assert np.isclose(r[0, 0], np.cos(0.5)) and np.isclose(r[0, hd // 2], np.sin(0.5))
+
+
+def test_swiglu_closed_form():
+    h = np.array([[2.0, -1.0]])
+    Wg = np.array([[1.0, 0.0]])          # gate = 2
+    Wu = np.array([[0.0, -3.0]])         # up = 3
+    Wd = np.array([[1.0], [0.5]])
+    out = D.swiglu_mlp(h, Wg, Wu, Wd)
+    silu2 = 2.0 / (1.0 + np.exp(-2.0))
+    assert np.allclose(out, [[3.0 * silu2, 1.5 * silu2]], atol=1e-15)
+
+
+def test_root_only_tree_is_one_decode_step():
+    rng = np.random.default_rng(4)
+    tr = O.tree_tables([], 3, 2)         # T = 1: the root
+    Dm, F, H, Vv, L = 16, 24, 2, 20, 6
+    embed = rng.normal(size=(Vv, Dm))
+    layers = [_layer(rng, Dm, F)]
+    kcs = [rng.normal(size=(H, L + 2, Dm // H))]
+    vcs = [rng.normal(size=(H, L + 2, Dm // H))]
+    _, hid, _, _ = D.tree_forward(tr, np.array([5]), embed, layers, np.ones(Dm), np.eye(Vv, Dm), kcs, vcs, L, H)
+    ref = _causal_forward(np.array([5]), embed, layers, kcs, vcs, L, H)
+    assert np.allclose(hid, ref, atol=1e-12)
