@@ -6,7 +6,8 @@ tree's own rows) and returns (O_r, lse_r); the log-sum-exp identity puts the
 parts back together.  Pinned here against the already pinned unsplit oracle
 (the identity must reproduce it for any G), closed forms (equal scores give
 the mean of V and ln(n); a single key gives its own V and score), and the
-window bookkeeping."""
+window bookkeeping.  The host-side argument checks of medusa_attention_combine
+are exercised at the end (nothing reaches a device)."""
 
 import numpy as np
 import pytest
@@ -73,3 +74,46 @@ def test_window_closed_forms():
     assert not o_e.any() and np.all(l_e == -np.inf)
     got, l2 = O.combine_partials(np.stack([o_e, o]), np.stack([l_e, lse]))
     assert np.allclose(got, o, atol=0) and np.allclose(l2, lse, atol=0)
+
+
+# ---------------------------------------------------------------------------
+# medusa_attention_combine: host-side checks (nothing reaches a device)
+
+
+@pytest.fixture(scope="module")
+def mb(built):
+    import speculative_decoding_heads_b200 as mb
+    return mb
+
+
+class _NoStream:
+    cuda_stream = 0
+
+
+def _combine_args(G, rows, hd):
+    import torch
+    return torch.zeros(G, rows, hd), torch.zeros(G, rows), torch.zeros(rows, hd)
+
+
+@pytest.mark.parametrize("G,rows,hd,what", [(65, 4, 8, "G, rows or hd"), (0, 4, 8, "G, rows or hd"),
+                                            (2, 4, 6, "G, rows or hd"), (2, 4, 2048, "G, rows or hd")])
+def test_combine_rejects_shapes(mb, G, rows, hd, what):
+    outs, lses, out = _combine_args(max(G, 1), rows, hd)
+    with pytest.raises(mb.MedusaError) as e:
+        mb._check(mb._lib.medusa_attention_combine(G, rows, hd, mb._p(outs), mb._p(lses), mb._p(out), None, 0))
+    assert e.value.code == mb.MEDUSA_ERR_INVALID_ARG and what in str(e.value)
+
+
+def test_combine_rejects_overlap_and_misalignment(mb):
+    import torch
+    outs, lses, _ = _combine_args(2, 4, 8)
+    with pytest.raises(mb.MedusaError) as e:
+        mb.medusa_attention_combine(outs, lses, outs[1], stream=_NoStream())
+    assert "overlaps" in str(e.value)
+    odd = torch.zeros(4 * 8 + 1)[1:].view(4, 8)          # 4 bytes past a 16-byte boundary
+    with pytest.raises(mb.MedusaError) as e:
+        mb.medusa_attention_combine(outs, lses, odd, stream=_NoStream())
+    assert "misaligned" in str(e.value)
+    with pytest.raises(mb.MedusaError) as e:
+        mb._check(mb._lib.medusa_attention_combine(2, 4, 8, None, mb._p(lses), mb._p(odd), None, 0))
+    assert "null pointer" in str(e.value)
