@@ -271,7 +271,6 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
   }
 }
 
-// PART3
 // ---- MMA issuer (one thread) ------------------------------------------------
 // S(g) = Q K^T of step g (M = 64, N = 128, 8 products over the head dim) and
 // O += P(g) V (M = 128, N = 128, one product per 16 valid keys).  Both are
