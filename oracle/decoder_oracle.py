@@ -104,3 +104,76 @@ def tree_forward(tree, tokens, embed, layers, final_norm, lm_head, k_caches, v_c
         vcs.append(vc)
     hid = rms_norm(x, final_norm)
     return hid @ np.asarray(lm_head, dtype=np.float64).T, x, kcs, vcs
+
+
+# ----------------------------------------------------------------------------
+# The generation loop  [P3 MedusaModelABC.medusa_generate: repeat the step;
+#     P4 实践案例 case 1 (guess, verify, keep the accepted prefix) and 学到什么
+#     (each step also yields the base model's own token)]
+# ----------------------------------------------------------------------------
+
+
+def chain_tree(n: int):
+    """The tree of n tokens in a row (node i at depth i, seeing nodes 0..i): a causal forward."""
+    return {"T": n, "depth": np.arange(n), "anc": np.tril(np.ones((n, n), dtype=bool))}
+
+
+def _empty_caches(model, Lcap):
+    D = model["embed"].shape[1]
+    H = model["H"]
+    shape = (H, Lcap, D // H)
+    return [np.zeros(shape) for _ in model["layers"]], [np.zeros(shape) for _ in model["layers"]]
+
+
+def _forward(model, tree, tokens, kcs, vcs, L):
+    return tree_forward(tree, tokens, model["embed"], model["layers"], model["final_norm"], model["lm_head"],
+                        kcs, vcs, L, model["H"])
+
+
+def greedy_decode(model, prompt, n_new: int, Lcap: int):
+    """Plain greedy decoding with the base model: n_new tokens after the prompt, one forward each."""
+    kcs, vcs = _empty_caches(model, Lcap)
+    logits, _, kcs, vcs = _forward(model, chain_tree(len(prompt)), np.asarray(prompt), kcs, vcs, 0)
+    L = len(prompt)
+    out = [int(np.argmax(logits[-1]))]
+    while len(out) < n_new:
+        logits, _, kcs, vcs = _forward(model, chain_tree(1), np.asarray(out[-1:]), kcs, vcs, L)
+        L += 1
+        out.append(int(np.argmax(logits[-1])))
+    return out
+
+
+def medusa_generate_greedy(model, heads, choices, K: int, topk: int, prompt, n_new: int, Lcap: int):
+    """Greedy Medusa decoding of one sequence, built from the step's oracle functions.
+
+    After the prompt's forward, each step: the heads on the last accepted token's final hidden
+    state (after the final RMSNorm), their top-k, the candidate tree rooted at the base model's own
+    next token, the base model's forward over the tree at the cache length (S5 inside it), greedy
+    acceptance, and the KV compaction.  The step emits the root and the a accepted tokens.
+    Returns (tokens [n_new], accept length of every step)."""
+    tr = O.tree_tables(choices, K, topk)
+    kcs, vcs = _empty_caches(model, Lcap)
+    logits, x, kcs, vcs = _forward(model, chain_tree(len(prompt)), np.asarray(prompt), kcs, vcs, 0)
+    L = len(prompt)
+    h = rms_norm(x[-1:], model["final_norm"])
+    root = int(np.argmax(logits[-1]))
+    out, accepts = [], []
+    while len(out) < n_new:
+        if L + tr["T"] > Lcap:
+            raise ValueError("cache capacity too small for the next tree")
+        _, z = O.medusa_heads(h, heads["W1"], heads["b1"], heads["Wout"])
+        ids, _ = O.topk_desc(z, topk)
+        toks, cand, _ = O.build_tree(tr, [root], ids, [L])
+        logits, x, kcs, vcs = _forward(model, tr, toks[0], kcs, vcs, L)
+        post = O.evaluate_posterior(tr, logits[None], cand, "greedy")
+        a, best = int(post["accept_len"][0]), int(post["best_path"][0])
+        k_new, v_new, _ = O.accept_kv(tr, np.stack(kcs)[:, None], np.stack(vcs)[:, None], [L], [best], [a])
+        kcs = [k_new[l, 0] for l in range(len(kcs))]
+        vcs = [v_new[l, 0] for l in range(len(vcs))]
+        out.extend(int(t) for t in post["accepted_tokens"][0, :a + 1])
+        node = int(tr["retrieve"][best, a])
+        h = rms_norm(x[node:node + 1], model["final_norm"])
+        root = int(post["next_token"][0])
+        L += a + 1
+        accepts.append(a)
+    return out[:n_new], accepts

@@ -6,7 +6,8 @@ positions L, L+1, ... -- the definition of verifying all candidates in one
 forward.  The causal forward here is written separately, from torch's fp64
 scaled-dot-product attention with a causal mask, so that a wrong mask, a
 wrong position or a wrong cache row fails it.  Closed forms pin RMSNorm,
-RoPE and the SwiGLU feed-forward."""
+RoPE and the SwiGLU feed-forward.  The generation loop is pinned by
+losslessness: greedy Medusa decoding emits the base model's greedy tokens."""
 
 import numpy as np
 import pytest
@@ -136,3 +137,42 @@ def test_root_only_tree_is_one_decode_step():
     _, hid, _, _ = D.tree_forward(tr, np.array([5]), embed, layers, np.ones(Dm), np.eye(Vv, Dm), kcs, vcs, L, H)
     ref = _causal_forward(np.array([5]), embed, layers, kcs, vcs, L, H)
     assert np.allclose(hid, ref, atol=1e-12)
+
+
+def _model(rng, V, Dm=16, F=24, H=2, nl=2, s=0.3):
+    return {"embed": rng.normal(size=(V, Dm)), "layers": [_layer(rng, Dm, F, s) for _ in range(nl)],
+            "final_norm": np.ones(Dm), "lm_head": rng.normal(size=(V, Dm)), "H": H}
+
+
+def _heads(rng, K, V, Dm=16, s=0.5):
+    return {"W1": s * rng.normal(size=(K, Dm, Dm)), "b1": s * rng.normal(size=(K, Dm)),
+            "Wout": rng.normal(size=(K, V, Dm))}
+
+
+def _copy_heads(model, K):
+    """Heads that propose the base model's current prediction at every depth (u = h, Wout = LM head)."""
+    Dm = model["embed"].shape[1]
+    return {"W1": np.zeros((K, Dm, Dm)), "b1": np.zeros((K, Dm)),
+            "Wout": np.repeat(model["lm_head"][None], K, axis=0)}
+
+
+@pytest.mark.parametrize("seed,V,K,topk,n_nodes,kind", [
+    (0, 4, 3, 2, 10, "random"), (1, 5, 4, 3, 20, "random"), (3, 50, 3, 2, 8, "random"),
+    (0, 4, 3, 2, 10, "copy"), (1, 5, 4, 3, 20, "copy"), (2, 6, 2, 2, 6, "copy"), (4, 8, 5, 2, 16, "copy")])
+def test_greedy_medusa_generation_is_lossless(seed, V, K, topk, n_nodes, kind):
+    """Greedy Medusa decoding emits exactly the base model's greedy tokens, whatever the heads
+    propose: the base model decides.  Random heads are mostly rejected; heads that repeat the base
+    model's current prediction are accepted whenever the base model repeats itself, so accepted
+    paths, the KV compaction and the positions of later steps are exercised."""
+    rng = np.random.default_rng(seed)
+    model = _model(rng, V)
+    heads = _heads(rng, K, V) if kind == "random" else _copy_heads(model, K)
+    prompt = rng.integers(0, V, size=5)
+    n_new = 24
+    ref = D.greedy_decode(model, prompt, n_new, Lcap=64)
+    choices = O.ranksum_choices(K, topk, n_nodes)
+    got, accepts = D.medusa_generate_greedy(model, heads, choices, K, topk, prompt, n_new, Lcap=160)
+    assert got == ref
+    assert len(accepts) <= n_new and all(0 <= a <= K for a in accepts)
+    if kind == "copy":
+        assert sum(accepts) > 0, "no proposal was ever accepted: the case would not exercise acceptance"
