@@ -382,7 +382,9 @@ def run_ours(a, w):
     esz = 2 if w.dtype == "bf16" else 4
     head_bytes = w.K * (w.d * w.d + w.d + w.V * w.d) * esz
     kv_bytes = w.metric_bytes() - head_bytes
-    heads_gbs = head_bytes / (stage["heads_topk"] * 1e-6) / 1e9
+    # The heads kernel reads the weights once per group of up to four sequences, one launch each.
+    head_launches = (w.B + 3) // 4
+    heads_gbs = head_bytes * head_launches / (stage["heads_topk"] * 1e-6) / 1e9
     attn_gbs = kv_bytes / (stage["tree_attention"] * 1e-6) / 1e9
     traffic = None
     tpath = os.path.join(REPO, "profiles", "heads_topk_traffic.json")
