@@ -135,7 +135,13 @@ def _check(st: int):
 
 
 def _p(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device pointer of a tensor argument (None stays NULL).  Every tensor the C ABI takes is
+    device memory: a host tensor is refused here, before anything is enqueued."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmedusa_b200 tensor arguments must be CUDA tensors (got one on the host)")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -343,8 +349,8 @@ def make_step_args(tree: Tree, t: dict, mode: int, temperature=0.0, eps=0.09, al
                  "base_logits", "topk_ids", "topk_vals", "tree_tokens", "candidates",
                  "position_ids", "attn_out", "best_path", "accept_len", "accepted_tokens",
                  "next_token"):
-        setattr(a, name, t[name].data_ptr())
-    a.head_logits = t["head_logits"].data_ptr() if t.get("head_logits") is not None else None
+        setattr(a, name, _p(t[name]).value)
+    a.head_logits = _p(t["head_logits"]).value if t.get("head_logits") is not None else None
     a.scale = float(scale if scale is not None else hd ** -0.5)
     a.mode = int(mode)
     a.temperature, a.eps, a.alpha = float(temperature), float(eps), float(alpha)

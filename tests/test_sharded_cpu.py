@@ -3,6 +3,7 @@ merge relies on (pinned with the oracle's own top-k), the all-gather between
 two gloo ranks, and the host-side argument checks of medusa_topk_merge.  No
 compute call is made here."""
 
+import ctypes
 import os
 import socket
 import sys
@@ -137,9 +138,19 @@ def test_merge_rejects_bad_arguments_before_launch(mb, G, topk, row0, V, what):
     ids = torch.zeros(G, 1, 1, topk, dtype=torch.int32)
     out_vals = torch.zeros(1, 1, topk)
     out_ids = torch.zeros(1, 1, topk, dtype=torch.int32)
+    raw = lambda t: ctypes.c_void_p(t.data_ptr())      # host memory: the checks fail before any use
+    r0 = (ctypes.c_int32 * len(row0))(*row0)
     with pytest.raises(mb.MedusaError) as e:
-        mb.medusa_topk_merge(vals, ids, row0, V, out_vals, out_ids, stream=_NoStream())
+        mb._check(mb._lib.medusa_topk_merge(raw(vals), raw(ids), r0, G, V, 1, 1, topk, raw(out_vals), raw(out_ids),
+                                            None))
     assert e.value.code == mb.MEDUSA_ERR_INVALID_ARG and what in str(e.value)
+
+
+def test_binding_refuses_host_tensors(mb):
+    vals, ids = torch.zeros(2, 1, 1, 4), torch.zeros(2, 1, 1, 4, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        mb.medusa_topk_merge(vals, ids, [0, 50], 100, torch.zeros(1, 1, 4), torch.zeros(1, 1, 4, dtype=torch.int32),
+                             stream=_NoStream())
 
 
 class _NoStream:

@@ -86,8 +86,15 @@ def mb(built):
     return mb
 
 
-class _NoStream:
-    cuda_stream = 0
+def _raw(t):
+    """A host tensor's address: these calls fail their checks before any use of it."""
+    import ctypes
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _combine(mb, G, rows, hd, outs, lses, out):
+    mb._check(mb._lib.medusa_attention_combine(G, rows, hd, outs if outs is None else _raw(outs), _raw(lses),
+                                               _raw(out), None, 0))
 
 
 def _combine_args(G, rows, hd):
@@ -100,7 +107,7 @@ def _combine_args(G, rows, hd):
 def test_combine_rejects_shapes(mb, G, rows, hd, what):
     outs, lses, out = _combine_args(max(G, 1), rows, hd)
     with pytest.raises(mb.MedusaError) as e:
-        mb._check(mb._lib.medusa_attention_combine(G, rows, hd, mb._p(outs), mb._p(lses), mb._p(out), None, 0))
+        _combine(mb, G, rows, hd, outs, lses, out)
     assert e.value.code == mb.MEDUSA_ERR_INVALID_ARG and what in str(e.value)
 
 
@@ -108,12 +115,14 @@ def test_combine_rejects_overlap_and_misalignment(mb):
     import torch
     outs, lses, _ = _combine_args(2, 4, 8)
     with pytest.raises(mb.MedusaError) as e:
-        mb.medusa_attention_combine(outs, lses, outs[1], stream=_NoStream())
+        _combine(mb, 2, 4, 8, outs, lses, outs[1])
     assert "overlaps" in str(e.value)
     odd = torch.zeros(4 * 8 + 1)[1:].view(4, 8)          # 4 bytes past a 16-byte boundary
     with pytest.raises(mb.MedusaError) as e:
-        mb.medusa_attention_combine(outs, lses, odd, stream=_NoStream())
+        _combine(mb, 2, 4, 8, outs, lses, odd)
     assert "misaligned" in str(e.value)
     with pytest.raises(mb.MedusaError) as e:
-        mb._check(mb._lib.medusa_attention_combine(2, 4, 8, None, mb._p(lses), mb._p(odd), None, 0))
+        _combine(mb, 2, 4, 8, None, lses, odd)
     assert "null pointer" in str(e.value)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        mb.medusa_attention_combine(outs, lses, torch.zeros(4, 8))
