@@ -141,6 +141,9 @@ def _p(t: Optional[torch.Tensor]):
         return None
     if not t.is_cuda:
         raise ValueError("libmedusa_b200 tensor arguments must be CUDA tensors (got one on the host)")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"libmedusa_b200 tensor argument on {t.device}, but the current device is "
+                         f"cuda:{torch.cuda.current_device()} (the kernels run there)")
     return ctypes.c_void_p(t.data_ptr())
 
 
