@@ -20,8 +20,12 @@ from helpers import ATTN_ATOL, check_logits, oracle_heads, oracle_tree, stored_s
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["vicuna7b_bs1_L1024", "vicuna7b_bs1_L4096_typical", "vicuna13b_bs8_ragged",
-        "vicuna33b_bs4_L8192_N16", "vicuna33b_bs4_L8192_N128"]
+# Every full workload in every acceptance mode it names (config 3 runs greedy
+# and typical; config 4 sweeps trees of 16, 32, 64 and 128 nodes).
+FULL = [(name, mode) for name in ("vicuna7b_bs1_L1024", "vicuna7b_bs1_L4096_typical", "vicuna13b_bs8_ragged",
+                                  "vicuna33b_bs4_L8192_N16", "vicuna33b_bs4_L8192_N32",
+                                  "vicuna33b_bs4_L8192_N64", "vicuna33b_bs4_L8192_N128")
+        for mode in W.get(name).modes]
 
 
 @pytest.fixture(scope="module")
@@ -44,14 +48,13 @@ def _sample_slices(w, n_random=6):
     return sorted(picks)
 
 
-@pytest.mark.parametrize("name", FULL)
-def test_full_step(mb, name):
+@pytest.mark.parametrize("name,mode", FULL, ids=[f"{n}-{m}" for n, m in FULL])
+def test_full_step(mb, name, mode):
     from synth import device
     w = W.get(name)
     sub = stored_subseeds(w)
     assert sub is not None, "full workloads carry stored sub-seeds"
     sub_h, sub_l = sub
-    mode = w.modes[0]
     tr = oracle_tree(w)
 
     # ---- oracle: S1-S4 in full, S6 in full

@@ -444,6 +444,94 @@ def test_accept_kv_invariants():
 
 
 # ---------------------------------------------------------------------------
+# margin guards (they choose the sub-seeds that make bit-exact ids a fair
+# demand: every top-k gap and every typical-acceptance margin >= 1e-4 relative)
+# ---------------------------------------------------------------------------
+
+
+def check_topk_gap_guard(O):
+    # Well separated: fine at every k up to the row length.
+    z = np.array([[10.0, 9.0, 8.0, 7.0, -3.0, 0.5]])
+    assert all(O.topk_gap_ok(z, k) for k in range(1, 6))
+    # The 3rd and 4th largest values are 5e-5 apart (relative): the top-3 set
+    # depends on that pair, so k = 3 must be refused; k = 2 never looks at it.
+    z = np.array([[10.0, 9.0, 8.0, 8.0 * (1 - 5e-5), 1.0]])
+    assert O.topk_gap_ok(z, 2)
+    assert not O.topk_gap_ok(z, 3)
+    # A tie right after the k-th value (k = 4) decides membership; ties further
+    # down the row do not.
+    z = np.array([[5.0, 4.0, 3.0, 1.0, 1.0, 1.0]])
+    assert O.topk_gap_ok(z, 3)
+    assert not O.topk_gap_ok(z, 4)
+    # Gap just under and just over 1e-4 of the larger magnitude (1.0).  The
+    # first gap is above 1e-4 of the smaller value, so only a guard relative to
+    # the larger one refuses it.
+    g_in, g_out = 1e-4 * (1 - 5e-5), 1e-4 * (1 + 5e-5)
+    assert not O.topk_gap_ok(np.array([[1.0, 1.0 - g_in, -5.0]]), 1)
+    assert O.topk_gap_ok(np.array([[1.0, 1.0 - g_out, -5.0]]), 1)
+    # Negative values: the magnitude counts, not the signed value.
+    assert not O.topk_gap_ok(np.array([[-2.0, -2.0 * (1 + 5e-5), -9.0]]), 1)
+    assert O.topk_gap_ok(np.array([[-2.0, -2.0 * (1 + 5e-4), -9.0]]), 1)
+    # Every row of a batch is checked, whatever its position.
+    ok_row, bad_row = [7.0, 3.0, 1.0, 0.0], [7.0, 3.0, 3.0 * (1 + 1e-5), 0.0]
+    assert O.topk_gap_ok(np.array([[ok_row, ok_row], [ok_row, ok_row]]), 2)
+    assert not O.topk_gap_ok(np.array([[ok_row, ok_row], [ok_row, bad_row]]), 2)
+
+
+def test_topk_gap_guard():
+    check_topk_gap_guard(O)
+
+
+def _two_level_margin(a, V, temp, eps, alpha):
+    """(p - thr) / max(p, thr) for the token with logit a in a row [a, 0, ..., 0] (closed form)."""
+    e = math.exp(a / temp)
+    p, r = e / (e + V - 1), 1.0 / (e + V - 1)
+    H = -(p * math.log(p) + (V - 1) * r * math.log(r))
+    thr = min(eps, alpha * math.exp(-H))
+    return (p - thr) / max(p, thr)
+
+
+def _logit_for_margin(target, V, temp, eps, alpha, lo=-3.0, hi=1.0):
+    """Bisection for the logit a whose two-level margin is `target` (it grows with a here)."""
+    assert _two_level_margin(lo, V, temp, eps, alpha) < target < _two_level_margin(hi, V, temp, eps, alpha)
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        if _two_level_margin(mid, V, temp, eps, alpha) < target:
+            lo = mid
+        else:
+            hi = mid
+    return 0.5 * (lo + hi)
+
+
+def check_typical_margin_guard(O):
+    V, temp, eps, alpha = 8, 1.0, 0.09, 0.3
+    # One-edge tree: root -> its head-1 top-1 token (token 0 of the vocabulary).
+    tr = O.tree_tables([(0,)], 1, 1)
+    _, cand, _ = O.build_tree(tr, np.array([3]), np.array([[[0]]]), np.array([0]))
+
+    def ok(target, child_row=None):
+        z = np.zeros((1, 2, V))
+        z[0, 0, 0] = _logit_for_margin(target, V, temp, eps, alpha)
+        if child_row is not None:
+            z[0, 1] = child_row
+        return O.typical_margin_ok(tr, z, cand, temp, eps, alpha)
+
+    assert ok(2e-4) and ok(-2e-4)
+    assert not ok(5e-5) and not ok(-5e-5)
+    # Just inside 1e-4 of the larger of p and thr (but not of the smaller).
+    assert not ok(1e-4 * (1 - 2e-5)) and not ok(-1e-4 * (1 - 2e-5))
+    assert ok(1e-4 * (1 + 2e-5)) and ok(-1e-4 * (1 + 2e-5))
+    # A leaf's own row is no edge's parent: its values never matter.
+    leaf = np.zeros(V)
+    leaf[5] = _logit_for_margin(0.0, V, temp, eps, alpha)
+    assert ok(2e-4, leaf)
+
+
+def test_typical_margin_guard():
+    check_typical_margin_guard(O)
+
+
+# ---------------------------------------------------------------------------
 # planted mistakes must be caught
 # ---------------------------------------------------------------------------
 
@@ -499,6 +587,35 @@ def _stats_log2(logits_b, temperature, eps, alpha):
     return st
 
 
+def _gap_top_k_only(z, k, rel=1e-4):
+    return O.topk_gap_ok(z, k - 1, rel)     # looks at the k largest values, not k+1
+
+
+def _gap_rel_smaller(z, k, rel=1e-4):
+    flat = np.asarray(z, dtype=np.float64).reshape(-1, z.shape[-1])
+    for r in range(flat.shape[0]):
+        top = np.sort(flat[r])[::-1][:k + 1]
+        for j in range(len(top) - 1):
+            if abs(top[j] - top[j + 1]) < rel * min(abs(top[j]), abs(top[j + 1])):
+                return False
+    return True
+
+
+def _margin_rel_smaller(tree, logits, candidates, temperature, eps, alpha, rel=1e-4):
+    ret = tree["retrieve"]
+    for b in range(logits.shape[0]):
+        st = O.node_statistics(logits[b], temperature, eps, alpha)
+        for p in range(tree["P"]):
+            for j in range(1, tree["D"] + 1):
+                if ret[p, j] < 0:
+                    break
+                pr = st["prob"][ret[p, j - 1], int(candidates[b, p, j])]
+                th = st["threshold"][ret[p, j - 1]]
+                if abs(pr - th) < rel * min(pr, th):
+                    return False
+    return True
+
+
 def _tables_bad_index(choices, K, topk):
     tr = O.tree_tables(choices, K, topk)
     tr = dict(tr)
@@ -518,6 +635,10 @@ MUTANTS = {
     "entropy in bits": (dict(node_statistics=_stats_log2), [check_typical_closed_forms]),
     "tree index from first rank": (dict(tree_tables=_tables_bad_index),
                                    [check_worked_example, check_tree_tables_random]),
+    "gap guard over the top k only": (dict(topk_gap_ok=_gap_top_k_only), [check_topk_gap_guard]),
+    "gap guard relative to the smaller value": (dict(topk_gap_ok=_gap_rel_smaller), [check_topk_gap_guard]),
+    "margin guard relative to the smaller value": (dict(typical_margin_ok=_margin_rel_smaller),
+                                                   [check_typical_margin_guard]),
 }
 
 
