@@ -180,6 +180,10 @@ medusa_status_t medusa_heads_topk(const void* h, const void* W1, const void* b1,
  *    are rejected with MEDUSA_ERR_UNSUPPORTED before anything is enqueued.
  *  - The first call on a device looks up the array's device address (with
  *    that device current); make that first call before any stream capture.
+ *    The address is kept until the process exits: do not use this call on a
+ *    device after resetting it (cudaDeviceReset).
+ *  - Invalid arguments are refused before anything is enqueued; a refused
+ *    call leaves the array as it was.
  *  - Every call on a device shares the one array and leaves its contents
  *    behind; each call clears the part it uses on `stream` before launching.
  *    Calls whose work overlaps on the GPU (other streams, other threads)
@@ -282,6 +286,22 @@ medusa_status_t medusa_tree_attention_split(const medusa_tree_t* tree, int layer
  * outs.  1 <= G <= MEDUSA_MAX_SHARDS. */
 medusa_status_t medusa_attention_combine(int G, int64_t rows, int hd, const float* outs, const float* lses,
                                          float* out, float* lse_out, cudaStream_t stream);
+
+/* The combine of medusa_attention_combine split across the ranks, so that the
+ * ranks exchange only their lse values and then sum their outputs (an
+ * all-reduce of one output per rank instead of an all-gather of G):
+ *   lses [G, rows] fp32   every rank's lse, gathered in rank order
+ *   part [rows, hd] fp32  rank `rank`'s own window output, scaled in place:
+ *                         part[row] *= exp(lses[rank, row] - lse[row]),
+ *                         lse = ln sum_g exp(lses[g, row])
+ *   lse_out [rows] (may be NULL) receives lse.
+ * The sum over ranks of the scaled parts equals medusa_attention_combine's
+ * out.  A row whose every lse_g is -inf gets part = 0, lse = -inf.  hd a
+ * multiple of 4 in [4, 1024]; part 16-byte aligned; 1 <= G <=
+ * MEDUSA_MAX_SHARDS, 0 <= rank < G.  The pages have no counterpart (this is
+ * the library's multi-GPU option). */
+medusa_status_t medusa_attention_rescale(int G, int rank, int64_t rows, int hd, const float* lses, float* part,
+                                         float* lse_out, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* S6: posterior                                                             */

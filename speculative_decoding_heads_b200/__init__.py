@@ -52,7 +52,7 @@ EXPORTED = [
     "medusa_heads_workspace_size", "medusa_heads_topk", "medusa_heads_topk_noalloc",
     "medusa_topk_merge", "medusa_build_tree",
     "medusa_attention_workspace_size", "medusa_tree_attention",
-    "medusa_tree_attention_split", "medusa_attention_combine",
+    "medusa_tree_attention_split", "medusa_attention_combine", "medusa_attention_rescale",
     "medusa_posterior_workspace_size", "medusa_evaluate_posterior",
     "medusa_accept_kv",
     "medusa_step_workspace_size", "medusa_step",
@@ -115,6 +115,7 @@ _sig("medusa_tree_attention", _i32,
 _sig("medusa_tree_attention_split", _i32,
      [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _f32, _i32, _i32, _vp, _vp, _vp])
 _sig("medusa_attention_combine", _i32, [_i32, ctypes.c_int64, _i32, _vp, _vp, _vp, _vp, _vp])
+_sig("medusa_attention_rescale", _i32, [_i32, _i32, ctypes.c_int64, _i32, _vp, _vp, _vp, _vp])
 _sig("medusa_posterior_workspace_size", _sz, [_vp, _i32])
 _sig("medusa_evaluate_posterior", _i32,
      [_vp, _i32, _i32, _vp, _vp, _i32, _f32, _f32, _f32, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
@@ -159,6 +160,64 @@ def _dtype(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return MEDUSA_F32
     raise MedusaError(MEDUSA_ERR_UNSUPPORTED, f"unsupported dtype {t.dtype}")
+
+
+# Shape, dtype and layout of every tensor argument are checked here, before
+# any call: the C ABI takes bare pointers and sizes, so a tensor smaller than
+# the sizes say (a wrong shape, a 2-byte dtype where 4 bytes are read) would
+# be read or written past its end on the device, and a strided view would be
+# read as if it were dense.
+
+
+def _require(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _spec(name: str, t: Optional[torch.Tensor], shape, dtype: Optional[torch.dtype]):
+    """`t` must have exactly `shape` (and `dtype`, unless None) and be contiguous."""
+    _require(isinstance(t, torch.Tensor), f"{name} must be a tensor")
+    _require(tuple(t.shape) == tuple(int(x) for x in shape),
+             f"{name} has shape {tuple(t.shape)}, expected {tuple(int(x) for x in shape)}")
+    _require(dtype is None or t.dtype == dtype, f"{name} has dtype {t.dtype}, expected {dtype}")
+    _require(t.is_contiguous(), f"{name} must be contiguous")
+
+
+def _nbytes(name: str, t: torch.Tensor) -> int:
+    """Byte size of a contiguous workspace tensor (any element type)."""
+    _require(isinstance(t, torch.Tensor) and t.is_contiguous(), f"{name} must be a contiguous tensor")
+    return t.numel() * t.element_size()
+
+
+def _heads_specs(h, W1, b1, Wout, topk, topk_ids, topk_vals, head_logits):
+    _require(h.dim() == 2 and Wout.dim() == 3, "h must be [B, d] and Wout [K, V, d]")
+    B, d = h.shape
+    K, V = Wout.shape[0], Wout.shape[1]
+    _dtype(h)
+    _spec("h", h, (B, d), h.dtype)
+    _spec("W1", W1, (K, d, d), h.dtype)
+    _spec("b1", b1, (K, d), h.dtype)
+    _spec("Wout", Wout, (K, V, d), h.dtype)
+    _spec("topk_ids", topk_ids, (B, K, topk), torch.int32)
+    _spec("topk_vals", topk_vals, (B, K, topk), torch.float32)
+    if head_logits is not None:
+        _spec("head_logits", head_logits, (B, K, V), torch.float32)
+    return B, d, K, V
+
+
+def _attention_specs(tree, q, k_cache, v_cache, seq_lens, out):
+    _require(q.dim() == 5 and k_cache.dim() == 5,
+             "q must be [layers, B, T, H, hd] and the caches [layers, B, H, Lcap, hd]")
+    layers, B, T, H, hd = q.shape
+    _require(T == tree.T, f"q holds {T} tree tokens per sequence; the tree has {tree.T}")
+    Lcap = k_cache.shape[3]
+    _dtype(q)
+    _spec("q", q, (layers, B, T, H, hd), q.dtype)
+    _spec("k_cache", k_cache, (layers, B, H, Lcap, hd), q.dtype)
+    _spec("v_cache", v_cache, (layers, B, H, Lcap, hd), q.dtype)
+    _spec("seq_lens", seq_lens, (B,), torch.int32)
+    _spec("out", out, (layers, B, T, H, hd), torch.float32)
+    return layers, B, T, H, hd, Lcap
 
 
 def abi_version() -> int:
@@ -252,17 +311,16 @@ def medusa_heads_workspace_size(B, d, V, K, topk) -> int:
 
 
 def medusa_heads_topk(h, W1, b1, Wout, topk, topk_ids, topk_vals, ws, head_logits=None, stream=None):
-    B, d = h.shape
-    K, V = Wout.shape[0], Wout.shape[1]
+    B, d, K, V = _heads_specs(h, W1, b1, Wout, topk, topk_ids, topk_vals, head_logits)
+    nbytes = _nbytes("ws", ws)
     _check(_lib.medusa_heads_topk(_p(h), _p(W1), _p(b1), _p(Wout), B, d, V, K, topk, _dtype(h),
                                   _p(head_logits), _p(topk_ids), _p(topk_vals), _p(ws),
-                                  ws.numel(), _stream(stream)))
+                                  nbytes, _stream(stream)))
 
 
 def medusa_heads_topk_noalloc(h, W1, b1, Wout, topk, topk_ids, topk_vals, head_logits=None, stream=None):
     """medusa_heads_topk without a workspace (the library's fixed scratch array)."""
-    B, d = h.shape
-    K, V = Wout.shape[0], Wout.shape[1]
+    B, d, K, V = _heads_specs(h, W1, b1, Wout, topk, topk_ids, topk_vals, head_logits)
     _check(_lib.medusa_heads_topk_noalloc(_p(h), _p(W1), _p(b1), _p(Wout), B, d, V, K, topk, _dtype(h),
                                           _p(head_logits), _p(topk_ids), _p(topk_vals), _stream(stream)))
 
@@ -270,7 +328,12 @@ def medusa_heads_topk_noalloc(h, W1, b1, Wout, topk, topk_ids, topk_vals, head_l
 def medusa_topk_merge(vals, ids, row0: Sequence[int], V: int, out_vals, out_ids, stream=None):
     """Global top-k from gathered per-shard lists: vals/ids [G, B, K, topk] (shard-local ids),
     row0[g] the first vocabulary row of shard g; writes out_vals/out_ids [B, K, topk]."""
+    _require(vals.dim() == 4, "vals must be [G, B, K, topk]")
     G, B, K, topk = vals.shape
+    _spec("vals", vals, (G, B, K, topk), torch.float32)
+    _spec("ids", ids, (G, B, K, topk), torch.int32)
+    _spec("out_vals", out_vals, (B, K, topk), torch.float32)
+    _spec("out_ids", out_ids, (B, K, topk), torch.int32)
     if len(row0) != G:
         raise ValueError(f"row0 has {len(row0)} entries for {G} shards")
     r0 = (ctypes.c_int32 * G)(*[int(x) for x in row0])
@@ -280,6 +343,14 @@ def medusa_topk_merge(vals, ids, row0: Sequence[int], V: int, out_vals, out_ids,
 
 def medusa_build_tree(tree: Tree, root_tokens, topk_ids, seq_lens, tree_tokens, candidates,
                       position_ids, stream=None):
+    _require(root_tokens.dim() == 1, "root_tokens must be [B]")
+    B = root_tokens.shape[0]
+    _spec("root_tokens", root_tokens, (B,), torch.int32)
+    _spec("topk_ids", topk_ids, (B, tree.K, tree.topk), torch.int32)
+    _spec("seq_lens", seq_lens, (B,), torch.int32)
+    _spec("tree_tokens", tree_tokens, (B, tree.T), torch.int32)
+    _spec("candidates", candidates, (B, tree.P, tree.D + 1), torch.int32)
+    _spec("position_ids", position_ids, (B, tree.T), torch.int32)
     _check(_lib.medusa_build_tree(tree.handle, root_tokens.shape[0], _p(root_tokens), _p(topk_ids),
                                   _p(seq_lens), _p(tree_tokens), _p(candidates), _p(position_ids),
                                   _stream(stream)))
@@ -290,19 +361,19 @@ def medusa_attention_workspace_size(tree: Tree, layers, B, H, hd, dtype) -> int:
 
 
 def medusa_tree_attention(tree: Tree, q, k_cache, v_cache, seq_lens, scale, out, ws=None, stream=None):
-    layers, B, T, H, hd = q.shape
-    Lcap = k_cache.shape[3]
+    layers, B, T, H, hd, Lcap = _attention_specs(tree, q, k_cache, v_cache, seq_lens, out)
+    nbytes = 0 if ws is None else _nbytes("ws", ws)
     _check(_lib.medusa_tree_attention(tree.handle, layers, B, H, hd, _dtype(q), _p(q), _p(k_cache),
                                       _p(v_cache), Lcap, _p(seq_lens), float(scale), _p(out), _p(ws),
-                                      0 if ws is None else ws.numel(), _stream(stream)))
+                                      nbytes, _stream(stream)))
 
 
 def medusa_tree_attention_split(tree: Tree, q, k_cache, v_cache, seq_lens, scale, rank: int, G: int, out, lse,
                                 stream=None):
     """Attention over window `rank` of G of each slice's cached prefix (the tree rows with the last
     window): out [layers, B, T, H, hd] normalised over the window, lse [layers, B, T, H]."""
-    layers, B, T, H, hd = q.shape
-    Lcap = k_cache.shape[3]
+    layers, B, T, H, hd, Lcap = _attention_specs(tree, q, k_cache, v_cache, seq_lens, out)
+    _spec("lse", lse, (layers, B, T, H), torch.float32)
     _check(_lib.medusa_tree_attention_split(tree.handle, layers, B, H, hd, _dtype(q), _p(q), _p(k_cache),
                                             _p(v_cache), Lcap, _p(seq_lens), float(scale), int(rank), int(G),
                                             _p(out), _p(lse), _stream(stream)))
@@ -310,10 +381,30 @@ def medusa_tree_attention_split(tree: Tree, q, k_cache, v_cache, seq_lens, scale
 
 def medusa_attention_combine(outs, lses, out, lse_out=None, stream=None):
     """outs [G, ..., hd], lses [G, ...] (the same leading shape) -> out [..., hd], lse_out [...]."""
+    _require(outs.dim() >= 2 and lses.dim() == outs.dim() - 1, "outs must be [G, ..., hd] and lses [G, ...]")
     G, hd = outs.shape[0], outs.shape[-1]
+    _spec("outs", outs, outs.shape, torch.float32)
+    _spec("lses", lses, tuple(outs.shape[:-1]), torch.float32)
+    _spec("out", out, tuple(outs.shape[1:]), torch.float32)
+    if lse_out is not None:
+        _spec("lse_out", lse_out, tuple(outs.shape[1:-1]), torch.float32)
     rows = lses[0].numel()
     _check(_lib.medusa_attention_combine(G, rows, hd, _p(outs), _p(lses), _p(out), _p(lse_out),
                                          _stream(stream)))
+
+
+def medusa_attention_rescale(lses, rank: int, part, lse_out=None, stream=None):
+    """lses [G, ...] (every rank's lse, rank order), part [..., hd] (this rank's window output,
+    the same leading shape), scaled in place by exp(lse_rank - lse) so that the G ranks' parts sum
+    to the combined output; lse_out [...] receives lse."""
+    _require(lses.dim() >= 1 and part.dim() == lses.dim(), "lses must be [G, ...] and part [..., hd]")
+    G, hd = lses.shape[0], part.shape[-1]
+    _spec("lses", lses, (G,) + tuple(part.shape[:-1]), torch.float32)
+    _spec("part", part, part.shape, torch.float32)
+    if lse_out is not None:
+        _spec("lse_out", lse_out, tuple(part.shape[:-1]), torch.float32)
+    rows = lses[0].numel()
+    _check(_lib.medusa_attention_rescale(G, int(rank), rows, hd, _p(lses), _p(part), _p(lse_out), _stream(stream)))
 
 
 def medusa_posterior_workspace_size(tree: Tree, B) -> int:
@@ -323,15 +414,29 @@ def medusa_posterior_workspace_size(tree: Tree, B) -> int:
 def medusa_evaluate_posterior(tree: Tree, logits, candidates, mode, best_path, accept_len,
                               accepted_tokens, next_token, ws, temperature=0.0, eps=0.09,
                               alpha=0.3, stream=None):
+    _require(logits.dim() == 3, "logits must be [B, T, V]")
     B, T, V = logits.shape
+    _require(T == tree.T, f"logits hold {T} tree nodes per sequence; the tree has {tree.T}")
+    _spec("logits", logits, (B, T, V), torch.float32)
+    _spec("candidates", candidates, (B, tree.P, tree.D + 1), torch.int32)
+    for name, t in (("best_path", best_path), ("accept_len", accept_len), ("next_token", next_token)):
+        _spec(name, t, (B,), torch.int32)
+    _spec("accepted_tokens", accepted_tokens, (B, tree.D + 1), torch.int32)
+    nbytes = _nbytes("ws", ws)
     _check(_lib.medusa_evaluate_posterior(tree.handle, B, V, _p(logits), _p(candidates), int(mode),
                                           float(temperature), float(eps), float(alpha),
                                           _p(best_path), _p(accept_len), _p(accepted_tokens),
-                                          _p(next_token), _p(ws), ws.numel(), _stream(stream)))
+                                          _p(next_token), _p(ws), nbytes, _stream(stream)))
 
 
 def medusa_accept_kv(tree: Tree, k_cache, v_cache, seq_lens, best_path, accept_len, stream=None):
+    _require(k_cache.dim() == 5, "the caches must be [layers, B, H, Lcap, hd]")
     layers, B, H, Lcap, hd = k_cache.shape
+    _dtype(k_cache)
+    _spec("k_cache", k_cache, k_cache.shape, k_cache.dtype)
+    _spec("v_cache", v_cache, k_cache.shape, k_cache.dtype)
+    for name, t in (("seq_lens", seq_lens), ("best_path", best_path), ("accept_len", accept_len)):
+        _spec(name, t, (B,), torch.int32)
     _check(_lib.medusa_accept_kv(tree.handle, layers, B, H, hd, _dtype(k_cache), _p(k_cache),
                                  _p(v_cache), Lcap, _p(seq_lens), _p(best_path), _p(accept_len),
                                  _stream(stream)))
@@ -340,7 +445,19 @@ def medusa_accept_kv(tree: Tree, k_cache, v_cache, seq_lens, best_path, accept_l
 def make_step_args(tree: Tree, t: dict, mode: int, temperature=0.0, eps=0.09, alpha=0.3,
                    scale=None) -> StepArgs:
     """Builds ``medusa_step_args_t`` from a dict of device tensors (see ``StepBuffers``)."""
-    layers, B, T, H, hd = t["q"].shape
+    layers, B, T, H, hd, Lcap = _attention_specs(tree, t["q"], t["k_cache"], t["v_cache"], t["seq_lens"],
+                                                 t["attn_out"])
+    _require(t["q"].dtype == t["h"].dtype, "q and the caches must have the dtype of h and the weights")
+    _heads_specs(t["h"], t["W1"], t["b1"], t["Wout"], tree.topk, t["topk_ids"], t["topk_vals"],
+                 t.get("head_logits"))
+    _require(t["Wout"].shape[0] == tree.K, f"Wout holds {t['Wout'].shape[0]} heads; the tree has {tree.K}")
+    V = t["Wout"].shape[1]
+    _spec("root_tokens", t["root_tokens"], (B,), torch.int32)
+    _spec("base_logits", t["base_logits"], (B, T, V), torch.float32)
+    for name, shape in (("tree_tokens", (B, T)), ("position_ids", (B, T)), ("candidates", (B, tree.P, tree.D + 1)),
+                        ("best_path", (B,)), ("accept_len", (B,)), ("next_token", (B,)),
+                        ("accepted_tokens", (B, tree.D + 1))):
+        _spec(name, t[name], shape, torch.int32)
     a = StepArgs()
     a.tree = tree.handle
     a.B, a.d = t["h"].shape
@@ -365,7 +482,8 @@ def medusa_step_workspace_size(args: StepArgs) -> int:
 
 
 def medusa_step(args: StepArgs, ws, stream=None):
-    _check(_lib.medusa_step(ctypes.byref(args), _p(ws), ws.numel(), _stream(stream)))
+    nbytes = _nbytes("ws", ws)
+    _check(_lib.medusa_step(ctypes.byref(args), _p(ws), nbytes, _stream(stream)))
 
 
 def medusa_step_from_host(args: StepArgs, ws, host_in: dict, dev: dict, host_out: dict, stream=None,

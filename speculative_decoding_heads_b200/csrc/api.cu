@@ -112,10 +112,10 @@ extern "C" size_t medusa_heads_workspace_size(int B, int d, int V, int K, int to
   return heads_workspace_bytes(B, d, V, K, topk);
 }
 
-static medusa_status_t check_heads(const void* h, const void* W1, const void* b1, const void* Wout, int B,
-                                   int d, int V, int K, int topk, medusa_dtype_t dtype, const float* head_logits,
-                                   const int32_t* topk_ids, const float* topk_vals, const void* ws,
-                                   size_t ws_bytes) {
+medusa_status_t medusa::check_heads(const void* h, const void* W1, const void* b1, const void* Wout, int B,
+                                    int d, int V, int K, int topk, medusa_dtype_t dtype, const float* head_logits,
+                                    const int32_t* topk_ids, const float* topk_vals, const void* ws,
+                                    size_t ws_bytes) {
   const char* fn = "medusa_heads_topk";
   if (!h || !W1 || !b1 || !Wout || !topk_ids || !topk_vals || !ws)
     return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
@@ -253,6 +253,17 @@ extern "C" medusa_status_t medusa_attention_combine(int G, int64_t rows, int hd,
   if (o0 < i1 && i0 < o1) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": out overlaps outs");
   if (sm_count() <= 0) return fail(MEDUSA_ERR_CUDA, std::string(fn) + ": no usable CUDA device");
   return launch_attention_combine(G, static_cast<size_t>(rows), hd, outs, lses, out, lse_out, stream);
+}
+
+extern "C" medusa_status_t medusa_attention_rescale(int G, int rank, int64_t rows, int hd, const float* lses,
+                                                    float* part, float* lse_out, cudaStream_t stream) {
+  const char* fn = "medusa_attention_rescale";
+  if (!lses || !part) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (G < 1 || G > MEDUSA_MAX_SHARDS || rank < 0 || rank >= G || rows < 1 || hd < 4 || hd > 1024 || hd % 4 != 0)
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": G, rank, rows or hd out of range");
+  if (!aligned16(part)) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": misaligned pointer");
+  if (sm_count() <= 0) return fail(MEDUSA_ERR_CUDA, std::string(fn) + ": no usable CUDA device");
+  return launch_attention_rescale(G, rank, static_cast<size_t>(rows), hd, lses, part, lse_out, stream);
 }
 
 extern "C" size_t medusa_posterior_workspace_size(const medusa_tree_t* tree, int B) {

@@ -137,7 +137,46 @@ __global__ void attention_combine_kernel(int G, size_t rows, int hd4, const floa
   }
 }
 
+// The same identity split across ranks: rank `rank` scales its own partial
+// by exp(lse_rank - lse) in place, so that the G scaled partials sum to the
+// combined output (an all-reduce then replaces the gather of G outputs).
+// Only the G lse values of a row are read from every rank.
+__global__ void attention_rescale_kernel(int G, int rank, size_t rows, int hd4, const float* lses, float4* part,
+                                         float* lse_out) {
+  const size_t n = rows * static_cast<size_t>(hd4);
+  for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < n;
+       idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t row = idx / hd4;
+    float m = -INFINITY;
+    for (int g = 0; g < G; ++g) m = fmaxf(m, lses[g * rows + row]);
+    float w = 0.f, tot = 0.f;
+    if (m > -INFINITY) {
+      for (int g = 0; g < G; ++g) tot += expf(lses[g * rows + row] - m);
+      w = expf(lses[rank * rows + row] - m) / tot;
+    }
+    float4 o = part[idx];
+    o.x *= w;
+    o.y *= w;
+    o.z *= w;
+    o.w *= w;
+    part[idx] = o;
+    if (lse_out != nullptr && idx % hd4 == 0) lse_out[row] = m > -INFINITY ? m + logf(tot) : -INFINITY;
+  }
+}
+
 }  // namespace
+
+medusa_status_t launch_attention_rescale(int G, int rank, size_t rows, int hd, const float* lses, float* part,
+                                         float* lse_out, cudaStream_t stream) {
+  const size_t n = rows * static_cast<size_t>(hd / 4);
+  const size_t want = (n + 255) / 256;
+  const size_t cap = static_cast<size_t>(sm_count() > 0 ? sm_count() : 1) * 16;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  attention_rescale_kernel<<<grid, 256, 0, stream>>>(G, rank, rows, hd / 4, lses, reinterpret_cast<float4*>(part),
+                                                     lse_out);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_attention_rescale", e);
+}
 
 medusa_status_t launch_attention_split(const TreeDev& t, int layers, int B, int H, int hd, medusa_dtype_t dtype,
                                        const void* q, const void* k_cache, const void* v_cache, int Lcap,

@@ -56,6 +56,11 @@ struct TreeBuild {
   int32_t* position_ids;        // [B, T]
 };
 
+// Host-side argument checks of medusa_heads_topk (api.cu); nothing is enqueued.
+medusa_status_t check_heads(const void* h, const void* W1, const void* b1, const void* Wout, int B, int d, int V,
+                            int K, int topk, medusa_dtype_t dtype, const float* head_logits, const int32_t* topk_ids,
+                            const float* topk_vals, const void* ws, size_t ws_bytes);
+
 // Kernel launchers (heads.cu, tree_kernels.cu, attention.cu, posterior.cu, accept.cu).
 size_t heads_workspace_bytes(int B, int d, int V, int K, int topk);
 medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, const void* Wout,
@@ -99,6 +104,9 @@ medusa_status_t launch_attention_split(const TreeDev& t, int layers, int B, int 
                                        float* lse, cudaStream_t stream);
 medusa_status_t launch_attention_combine(int G, size_t rows, int hd, const float* outs, const float* lses,
                                          float* out, float* lse_out, cudaStream_t stream);
+
+medusa_status_t launch_attention_rescale(int G, int rank, size_t rows, int hd, const float* lses, float* part,
+                                         float* lse_out, cudaStream_t stream);
 
 medusa_status_t launch_topk_merge(const float* vals, const int32_t* ids, const int32_t* row0, int G, int B,
                                   int K, int topk, float* out_vals, int32_t* out_ids, cudaStream_t stream);

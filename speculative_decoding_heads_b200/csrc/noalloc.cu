@@ -11,7 +11,10 @@
 //
 // In host code the array's name only stands for the symbol; the device
 // address is fetched with cudaGetSymbolAddress once per device, with that
-// device current, on the first call made on it.
+// device current, on the first call made on it, and kept for the life of the
+// process.  After a device reset (cudaDeviceReset, or the primary context
+// torn down) the array may sit elsewhere, so this entry point must not be
+// used across a reset.
 #include <mutex>
 #include <string>
 
@@ -66,11 +69,15 @@ extern "C" medusa_status_t medusa_heads_topk_noalloc(const void* h, const void* 
   void* scratch = nullptr;
   medusa_status_t st = scratch_address(&scratch);
   if (st != MEDUSA_OK) return st;
+  // Every argument is checked before the shared array is touched: a call that
+  // is refused enqueues nothing, not even the clearing below.
+  st = check_heads(h, W1, b1, Wout, B, d, V, K, topk, dtype, head_logits, topk_ids, topk_vals, scratch,
+                   kNoAllocScratchBytes);
+  if (st != MEDUSA_OK) return st;
   // The array keeps whatever the previous call left.  The kernel's completion
   // counters must start at zero, so the part of the array this call uses is
   // cleared on the stream first (a memset, not an allocation).
   cudaError_t e = cudaMemsetAsync(scratch, 0, need, stream);
   if (e != cudaSuccess) return cuda_fail("medusa_heads_topk_noalloc: clearing the scratch", e);
-  return medusa_heads_topk(h, W1, b1, Wout, B, d, V, K, topk, dtype, head_logits, topk_ids, topk_vals, scratch,
-                           kNoAllocScratchBytes, stream);
+  return launch_heads(h, W1, b1, Wout, B, d, V, K, topk, dtype, head_logits, topk_ids, topk_vals, scratch, stream);
 }

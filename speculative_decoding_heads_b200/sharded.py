@@ -12,20 +12,34 @@ V, so the merged lists are those of the unsplit call bit for bit.
 
 Tree attention can split the same way along each slice's cached prefix:
 rank r attends to its window of prefix rows (the last rank also to the tree
-rows), the ranks all-gather their (output, lse) partials, and the log-sum-exp
-combine gives the unsplit result (tree_attention_sharded).
+rows), the ranks all-gather their lse values only, each rank scales its own
+output by its log-sum-exp weight, and an all-reduce (sum) of the scaled
+outputs gives the unsplit result (tree_attention_sharded).  That moves one
+output per rank instead of gathering G of them.
 
 Every step runs in the library's kernels; torch.distributed only moves the
-gathered lists (NCCL between GPUs, gloo on the host for the tests).
+gathered lists, the lse values and the sum (NCCL between GPUs, gloo on the
+host for the tests).
+
+When the caller passes `stream`, everything -- the temporaries, the kernels
+and the collectives -- runs with `stream` as torch's current stream, so the
+caching allocator never hands a temporary to another stream while a kernel
+on `stream` may still read it.
 """
 
+import contextlib
 from typing import List, Optional, Tuple
 
 import torch
 import torch.distributed as dist
 
-from . import (MAX_SHARDS, medusa_attention_combine, medusa_heads_topk, medusa_heads_workspace_size,
+from . import (MAX_SHARDS, medusa_attention_rescale, medusa_heads_topk, medusa_heads_workspace_size,
                medusa_topk_merge, medusa_tree_attention, medusa_tree_attention_split, workspace)
+
+
+def _on(stream):
+    """Makes `stream` torch's current stream (no-op when None)."""
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
 
 
 def shard_bounds(V: int, G: int) -> List[Tuple[int, int]]:
@@ -60,8 +74,9 @@ def heads_topk_sharded(h: torch.Tensor, W1: torch.Tensor, b1: torch.Tensor, Wout
 
     Wout_shard [K, n_g, d] holds rows shard_bounds(V, G)[rank] of every head (G, rank from
     `group`, or a single shard when torch.distributed is not initialised).  Returns the global
-    (topk_ids [B, K, topk] int32, topk_vals [B, K, topk] fp32) on every rank.  head_logits, if
-    given, receives this rank's [B, K, n_g] logits."""
+    (topk_ids [B, K, topk] int32, topk_vals [B, K, topk] fp32) on every rank, produced on
+    `stream` (torch's current stream when None).  head_logits, if given, receives this rank's
+    [B, K, n_g] logits."""
     G = dist.get_world_size(group) if dist.is_initialized() else 1
     rank = dist.get_rank(group) if dist.is_initialized() else 0
     bounds = shard_bounds(V, G)
@@ -70,50 +85,42 @@ def heads_topk_sharded(h: torch.Tensor, W1: torch.Tensor, b1: torch.Tensor, Wout
         raise ValueError(f"rank {rank} of {G} holds {Wout_shard.shape[1]} rows of Wout, expected {n}")
     B, K = h.shape[0], Wout_shard.shape[0]
     dev = h.device
-    if ws is None:
-        ws = workspace(medusa_heads_workspace_size(B, h.shape[1], n, K, topk), dev)
-    ids = torch.empty((B, K, topk), dtype=torch.int32, device=dev)
-    vals = torch.empty((B, K, topk), dtype=torch.float32, device=dev)
-    medusa_heads_topk(h, W1, b1, Wout_shard, topk, ids, vals, ws, head_logits=head_logits, stream=stream)
-    if G == 1:
-        all_vals, all_ids = vals.unsqueeze(0), ids.unsqueeze(0)
-    else:
-        # The collective runs on torch's current stream: order it after the
-        # heads kernel and the merge after it when the caller gave a stream.
-        if stream is not None:
-            torch.cuda.current_stream(dev).wait_stream(stream)
-        all_vals, all_ids = gather_shard_lists(vals, ids, group)
-        if stream is not None:
-            stream.wait_stream(torch.cuda.current_stream(dev))
-    out_ids = torch.empty_like(ids)
-    out_vals = torch.empty_like(vals)
-    medusa_topk_merge(all_vals, all_ids, [b[0] for b in bounds], V, out_vals, out_ids, stream=stream)
+    with _on(stream):
+        if ws is None:
+            ws = workspace(medusa_heads_workspace_size(B, h.shape[1], n, K, topk), dev)
+        ids = torch.empty((B, K, topk), dtype=torch.int32, device=dev)
+        vals = torch.empty((B, K, topk), dtype=torch.float32, device=dev)
+        medusa_heads_topk(h, W1, b1, Wout_shard, topk, ids, vals, ws, head_logits=head_logits)
+        if G == 1:
+            all_vals, all_ids = vals.unsqueeze(0), ids.unsqueeze(0)
+        else:
+            all_vals, all_ids = gather_shard_lists(vals, ids, group)
+        out_ids = torch.empty_like(ids)
+        out_vals = torch.empty_like(vals)
+        medusa_topk_merge(all_vals, all_ids, [b[0] for b in bounds], V, out_vals, out_ids)
     return out_ids, out_vals
 
 
 def tree_attention_sharded(tree, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                            seq_lens: torch.Tensor, scale: float, out: torch.Tensor, group=None, stream=None):
-    """S5 with every slice's cached prefix split over the ranks of `group`: this rank's window
-    (medusa_tree_attention_split), an all-gather of the G partial outputs and lse values, and the
-    combine.  `out` [layers, B, T, H, hd] receives medusa_tree_attention's result on every rank;
-    with one rank (or no process group) it is that call.  Each rank needs only its window's rows
-    of the caches (and the last rank the tree rows), in the full [.., Lcap, hd] layout."""
+    """S5 with every slice's cached prefix split over the ranks of `group`.
+
+    This rank's window (medusa_tree_attention_split) goes straight into `out`; the ranks
+    all-gather their lse values ([layers, B, T, H] fp32 each); each rank scales its window output
+    by exp(lse_rank - lse) in place (medusa_attention_rescale); an all-reduce (sum) of `out` then
+    leaves medusa_tree_attention's result on every rank.  With one rank (or no process group) it
+    is that call.  Each rank needs only its window's rows of the caches (and the last rank the
+    tree rows), in the full [.., Lcap, hd] layout."""
     G = dist.get_world_size(group) if dist.is_initialized() else 1
-    if G == 1:
-        medusa_tree_attention(tree, q, k_cache, v_cache, seq_lens, scale, out, stream=stream)
-        return out
-    rank = dist.get_rank(group)
-    dev = out.device
-    part = torch.empty_like(out)
-    lse = torch.empty(tuple(out.shape[:-1]), dtype=torch.float32, device=dev)
-    medusa_tree_attention_split(tree, q, k_cache, v_cache, seq_lens, scale, rank, G, part, lse, stream=stream)
-    if stream is not None:
-        torch.cuda.current_stream(dev).wait_stream(stream)
-    all_o = torch.empty((G,) + tuple(out.shape), dtype=torch.float32, device=dev)
-    all_l = torch.empty((G,) + tuple(lse.shape), dtype=torch.float32, device=dev)
-    dist.all_gather(list(all_o.unbind(0)), part, group=group)
-    dist.all_gather(list(all_l.unbind(0)), lse, group=group)
-    if stream is not None:
-        stream.wait_stream(torch.cuda.current_stream(dev))
-    medusa_attention_combine(all_o, all_l, out, stream=stream)
+    with _on(stream):
+        if G == 1:
+            medusa_tree_attention(tree, q, k_cache, v_cache, seq_lens, scale, out)
+            return out
+        rank = dist.get_rank(group)
+        lse = torch.empty(tuple(out.shape[:-1]), dtype=torch.float32, device=out.device)
+        medusa_tree_attention_split(tree, q, k_cache, v_cache, seq_lens, scale, rank, G, out, lse)
+        all_l = torch.empty((G,) + tuple(lse.shape), dtype=torch.float32, device=out.device)
+        dist.all_gather(list(all_l.unbind(0)), lse, group=group)
+        medusa_attention_rescale(all_l, rank, out)
+        dist.all_reduce(out, op=dist.ReduceOp.SUM, group=group)
     return out

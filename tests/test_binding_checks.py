@@ -1,0 +1,174 @@
+"""Host-side checks of the Python binding: every tensor argument's shape,
+dtype and layout are checked before any call reaches the C ABI (which takes
+bare pointers and sizes, so a tensor smaller than the sizes imply would be
+read or written past its end on the device).  CPU tensors are enough here:
+each case must fail its check with ValueError before the binding looks at
+where the tensor lives."""
+
+import pytest
+import torch
+
+
+@pytest.fixture(scope="module")
+def mb(built):
+    import speculative_decoding_heads_b200 as mb
+    return mb
+
+
+@pytest.fixture(scope="module")
+def tree(mb):
+    t = mb.Tree([(0,), (1,), (0, 0), (0, 1), (1, 0), (1, 1)], 2, 2, upload=False)
+    yield t
+    t.close()
+
+
+B, d, V, K, topk = 2, 256, 300, 2, 2
+bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+
+
+def _heads(**over):
+    a = dict(h=torch.zeros(B, d, dtype=bf), W1=torch.zeros(K, d, d, dtype=bf), b1=torch.zeros(K, d, dtype=bf),
+             Wout=torch.zeros(K, V, d, dtype=bf), ids=torch.zeros(B, K, topk, dtype=i32),
+             vals=torch.zeros(B, K, topk, dtype=f32), ws=torch.zeros(4096, dtype=torch.uint8), logits=None)
+    a.update(over)
+    return a
+
+
+HEADS_CASES = {
+    "W1 fp32 with bf16 h": dict(W1=torch.zeros(K, d, d, dtype=f32)),
+    "b1 wrong length": dict(b1=torch.zeros(K, d + 8, dtype=bf)),
+    "Wout fp32": dict(Wout=torch.zeros(K, V, d, dtype=f32)),
+    "W1 transposed view": dict(W1=torch.zeros(K, d, d, dtype=bf).transpose(1, 2)),
+    "Wout strided": dict(Wout=torch.zeros(K, 2 * V, d, dtype=bf)[:, ::2]),
+    "topk_ids too small": dict(ids=torch.zeros(B, K, topk - 1, dtype=i32)),
+    "topk_ids int64": dict(ids=torch.zeros(B, K, topk, dtype=torch.int64)),
+    "topk_vals bf16": dict(vals=torch.zeros(B, K, topk, dtype=bf)),
+    "head_logits short": dict(logits=torch.zeros(B, K, V - 1, dtype=f32)),
+    "head_logits bf16": dict(logits=torch.zeros(B, K, V, dtype=bf)),
+    "workspace strided": dict(ws=torch.zeros(8192, dtype=torch.uint8)[::2]),
+}
+
+
+@pytest.mark.parametrize("case", sorted(HEADS_CASES))
+def test_heads_refuses(mb, case):
+    a = _heads(**HEADS_CASES[case])
+    with pytest.raises(ValueError):
+        mb.medusa_heads_topk(a["h"], a["W1"], a["b1"], a["Wout"], topk, a["ids"], a["vals"], a["ws"],
+                             head_logits=a["logits"])
+    with pytest.raises(ValueError):
+        if case.startswith("workspace"):
+            raise ValueError("no workspace in this call")
+        mb.medusa_heads_topk_noalloc(a["h"], a["W1"], a["b1"], a["Wout"], topk, a["ids"], a["vals"],
+                                     head_logits=a["logits"])
+
+
+def test_heads_well_formed_reaches_the_device_check(mb):
+    a = _heads()
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        mb.medusa_heads_topk(a["h"], a["W1"], a["b1"], a["Wout"], topk, a["ids"], a["vals"], a["ws"])
+
+
+def _attn(tree, layers=2, H=3, hd=128, Lcap=40, dt=bf, **over):
+    a = dict(q=torch.zeros(layers, B, tree.T, H, hd, dtype=dt),
+             k=torch.zeros(layers, B, H, Lcap, hd, dtype=dt), v=torch.zeros(layers, B, H, Lcap, hd, dtype=dt),
+             lens=torch.zeros(B, dtype=i32), out=torch.zeros(layers, B, tree.T, H, hd, dtype=f32))
+    a.update(over)
+    return a
+
+
+ATTN_CASES = {
+    "q fp32 with bf16 caches": lambda tr: dict(q=torch.zeros(2, B, tr.T, 3, 128, dtype=f32)),
+    "q with another tree size": lambda tr: dict(q=torch.zeros(2, B, tr.T + 1, 3, 128, dtype=bf)),
+    "v_cache shorter": lambda tr: dict(v=torch.zeros(2, B, 3, 39, 128, dtype=bf)),
+    "k_cache heads-major mismatch": lambda tr: dict(k=torch.zeros(2, 3, B, 40, 128, dtype=bf)),
+    "out bf16": lambda tr: dict(out=torch.zeros(2, B, tr.T, 3, 128, dtype=bf)),
+    "out too small": lambda tr: dict(out=torch.zeros(2, B, tr.T, 3, 64, dtype=f32)),
+    "seq_lens int64": lambda tr: dict(lens=torch.zeros(B, dtype=torch.int64)),
+    "k_cache strided": lambda tr: dict(k=torch.zeros(2, B, 3, 80, 128, dtype=bf)[:, :, :, ::2]),
+}
+
+
+@pytest.mark.parametrize("case", sorted(ATTN_CASES))
+def test_attention_refuses(mb, tree, case):
+    a = _attn(tree, **ATTN_CASES[case](tree))
+    with pytest.raises(ValueError):
+        mb.medusa_tree_attention(tree, a["q"], a["k"], a["v"], a["lens"], 0.1, a["out"])
+    lse = torch.zeros(a["out"].shape[:-1], dtype=f32)
+    with pytest.raises(ValueError):
+        mb.medusa_tree_attention_split(tree, a["q"], a["k"], a["v"], a["lens"], 0.1, 0, 2, a["out"], lse)
+
+
+def test_split_refuses_a_wrong_lse(mb, tree):
+    a = _attn(tree)
+    with pytest.raises(ValueError, match="lse"):
+        mb.medusa_tree_attention_split(tree, a["q"], a["k"], a["v"], a["lens"], 0.1, 0, 2, a["out"],
+                                       torch.zeros(2, B, tree.T, 2, dtype=f32))
+
+
+def test_accept_kv_refuses(mb, tree):
+    a = _attn(tree)
+    one = torch.zeros(B, dtype=i32)
+    with pytest.raises(ValueError):
+        mb.medusa_accept_kv(tree, a["k"], a["v"][:, :, :, :30].contiguous(), a["lens"], one, one)
+    with pytest.raises(ValueError):
+        mb.medusa_accept_kv(tree, a["k"], a["v"].float(), a["lens"], one, one)
+    with pytest.raises(ValueError):
+        mb.medusa_accept_kv(tree, a["k"], a["v"], a["lens"], torch.zeros(B + 1, dtype=i32), one)
+
+
+def _post(tree, **over):
+    D1 = tree.D + 1
+    a = dict(logits=torch.zeros(B, tree.T, V, dtype=f32), cand=torch.zeros(B, tree.P, D1, dtype=i32),
+             best=torch.zeros(B, dtype=i32), alen=torch.zeros(B, dtype=i32), acc=torch.zeros(B, D1, dtype=i32),
+             nxt=torch.zeros(B, dtype=i32), ws=torch.zeros(1024, dtype=torch.uint8))
+    a.update(over)
+    return a
+
+
+POST_CASES = {
+    "logits bf16": lambda tr: dict(logits=torch.zeros(B, tr.T, V, dtype=bf)),
+    "logits for another tree": lambda tr: dict(logits=torch.zeros(B, tr.T - 1, V, dtype=f32)),
+    "candidates short": lambda tr: dict(cand=torch.zeros(B, tr.P - 1, tr.D + 1, dtype=i32)),
+    "accepted_tokens short": lambda tr: dict(acc=torch.zeros(B, tr.D, dtype=i32)),
+    "next_token int64": lambda tr: dict(nxt=torch.zeros(B, dtype=torch.int64)),
+    "logits strided": lambda tr: dict(logits=torch.zeros(B, tr.T, 2 * V, dtype=f32)[:, :, ::2]),
+}
+
+
+@pytest.mark.parametrize("case", sorted(POST_CASES))
+def test_posterior_refuses(mb, tree, case):
+    a = _post(tree, **POST_CASES[case](tree))
+    with pytest.raises(ValueError):
+        mb.medusa_evaluate_posterior(tree, a["logits"], a["cand"], mb.MEDUSA_GREEDY, a["best"], a["alen"], a["acc"],
+                                     a["nxt"], a["ws"])
+
+
+def test_build_tree_refuses(mb, tree):
+    ok = dict(root=torch.zeros(B, dtype=i32), ids=torch.zeros(B, tree.K, tree.topk, dtype=i32),
+              lens=torch.zeros(B, dtype=i32), toks=torch.zeros(B, tree.T, dtype=i32),
+              cand=torch.zeros(B, tree.P, tree.D + 1, dtype=i32), pos=torch.zeros(B, tree.T, dtype=i32))
+    for key, bad in [("ids", torch.zeros(B, tree.K, tree.topk + 1, dtype=i32)),
+                     ("toks", torch.zeros(B, tree.T - 1, dtype=i32)),
+                     ("cand", torch.zeros(B, tree.P, tree.D, dtype=i32)),
+                     ("pos", torch.zeros(B, tree.T, dtype=torch.int64))]:
+        a = dict(ok, **{key: bad})
+        with pytest.raises(ValueError):
+            mb.medusa_build_tree(tree, a["root"], a["ids"], a["lens"], a["toks"], a["cand"], a["pos"])
+
+
+def test_merge_combine_and_rescale_refuse(mb):
+    G = 2
+    vals, ids = torch.zeros(G, B, K, topk), torch.zeros(G, B, K, topk, dtype=i32)
+    with pytest.raises(ValueError):
+        mb.medusa_topk_merge(vals, ids.long(), [0, 150], V, torch.zeros(B, K, topk), torch.zeros(B, K, topk, dtype=i32))
+    with pytest.raises(ValueError):
+        mb.medusa_topk_merge(vals, ids, [0, 150], V, torch.zeros(B, K, topk + 1), torch.zeros(B, K, topk, dtype=i32))
+    outs, lses = torch.zeros(G, 10, 8), torch.zeros(G, 10)
+    with pytest.raises(ValueError):
+        mb.medusa_attention_combine(outs, torch.zeros(G, 9), torch.zeros(10, 8))
+    with pytest.raises(ValueError):
+        mb.medusa_attention_combine(outs, lses, torch.zeros(10, 4))
+    with pytest.raises(ValueError):
+        mb.medusa_attention_rescale(lses, 0, torch.zeros(11, 8))
+    with pytest.raises(ValueError):
+        mb.medusa_attention_rescale(lses.double(), 0, torch.zeros(10, 8))

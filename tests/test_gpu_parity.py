@@ -359,20 +359,24 @@ def test_invalid_arguments_launch_nothing(mb, dev):
     t = dev.materialise(w, fill=False)
     ws = mb.workspace(mb.medusa_heads_workspace_size(w.B, w.d, w.V, w.K, w.topk))
     t["topk_ids"].fill_(-5)
+    ids33 = torch.full((w.B, w.K, 33), -5, dtype=torch.int32, device="cuda")
+    vals33 = torch.zeros((w.B, w.K, 33), device="cuda")
     cases = [
-        (dict(topk=33), mb.MEDUSA_ERR_INVALID_ARG),
+        (dict(topk=33, ids=ids33, vals=vals33), mb.MEDUSA_ERR_INVALID_ARG),
         (dict(ws=mb.workspace(256)), mb.MEDUSA_ERR_INVALID_ARG),
-        (dict(h=t["h"][:, :100].contiguous(), W1=t["W1"][:, :100, :100].contiguous()), mb.MEDUSA_ERR_UNSUPPORTED),
+        (dict(h=t["h"][:, :100].contiguous(), W1=t["W1"][:, :100, :100].contiguous(),
+              b1=t["b1"][:, :100].contiguous(), Wout=t["Wout"][:, :, :100].contiguous()), mb.MEDUSA_ERR_UNSUPPORTED),
     ]
     for over, code in cases:
-        kw = dict(h=t["h"], W1=t["W1"], b1=t["b1"], Wout=t["Wout"], topk=w.topk, ws=ws)
+        kw = dict(h=t["h"], W1=t["W1"], b1=t["b1"], Wout=t["Wout"], topk=w.topk, ws=ws, ids=t["topk_ids"],
+                  vals=t["topk_vals"])
         kw.update(over)
         with pytest.raises(mb.MedusaError) as ei:
-            mb.medusa_heads_topk(kw["h"], kw["W1"], kw["b1"], kw["Wout"], kw["topk"], t["topk_ids"],
-                                 t["topk_vals"], kw["ws"])
+            mb.medusa_heads_topk(kw["h"], kw["W1"], kw["b1"], kw["Wout"], kw["topk"], kw["ids"], kw["vals"],
+                                 kw["ws"])
         assert ei.value.code == code
     torch.cuda.synchronize()
-    assert (t["topk_ids"] == -5).all()
+    assert (t["topk_ids"] == -5).all() and (ids33 == -5).all()
     tree = _tree(mb, w)
     logits = torch.zeros((w.B, tree.T, w.V), device="cuda")
     cand = torch.zeros((w.B, tree.P, tree.D + 1), dtype=torch.int32, device="cuda")

@@ -145,3 +145,30 @@ def test_single_shard_entry_point_equals_unsplit(mb, sh, dev):
     out_ids, out_vals = sh.heads_topk_sharded(t["h"], t["W1"], t["b1"], t["Wout"], w.V, w.topk)
     torch.cuda.synchronize()
     assert torch.equal(out_ids, ids) and torch.equal(out_vals, vals)
+
+
+def test_sharded_calls_on_a_side_stream_with_a_busy_allocator(mb, sh, dev):
+    """heads_topk_sharded and tree_attention_sharded given their own stream: their temporaries
+    belong to that stream, so allocations on the default stream right after the call (which
+    would reuse freed blocks) cannot clobber what the stream's kernels still read."""
+    w = SMALL["v13b_small"]
+    sub_h, _, _ = pick_sub_h(w)
+    t = dev.materialise(w, sub_h=sub_h)
+    ref_ids, ref_vals, _ = _unsplit(mb, t, w)
+    tree = mb.Tree(O.ranksum_choices(w.K, w.topk, w.n_nodes), w.K, w.topk)
+    scale = O.attention_scale(w.hd)
+    ref_out = torch.empty_like(t["attn_out"])
+    mb.medusa_tree_attention(tree, t["q"], t["k_cache"], t["v_cache"], t["seq_lens"], scale, ref_out)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    for _ in range(3):
+        side.wait_stream(torch.cuda.current_stream())
+        ids, vals = sh.heads_topk_sharded(t["h"], t["W1"], t["b1"], t["Wout"], w.V, w.topk, stream=side)
+        out = torch.empty_like(t["attn_out"])
+        side.wait_stream(torch.cuda.current_stream())
+        sh.tree_attention_sharded(tree, t["q"], t["k_cache"], t["v_cache"], t["seq_lens"], scale, out, stream=side)
+        junk = [torch.full((1 << 20,), -7.0, device="cuda") for _ in range(16)]   # the default stream, busy
+        side.synchronize()
+        assert torch.equal(ids, ref_ids) and torch.equal(vals, ref_vals)
+        assert torch.equal(out, ref_out)
+        del junk

@@ -149,3 +149,45 @@ def test_split_rejects_unsupported_shapes(mb, dev, name):
                                        O.attention_scale(w.hd), 0, 2, torch.empty(shape, device="cuda"),
                                        torch.empty(shape[:-1], device="cuda"))
     assert e.value.code == mb.MEDUSA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("name,G", [("v7b_small", 2), ("v13b_small", 3), ("b3_small", 4)])
+def test_rescaled_partials_sum_to_the_combine(mb, dev, name, G):
+    """medusa_attention_rescale: each rank scales its own window output; the sum over ranks (what
+    the all-reduce computes) equals medusa_attention_combine's output and lse."""
+    w = SMALL[name]
+    t, tree = _case(mb, dev, w)
+    outs, lses, out, lse = _split(mb, t, tree, O.attention_scale(w.hd), G)
+    acc = torch.zeros_like(out)
+    lse2 = torch.empty_like(lse)
+    for r in range(G):
+        part = outs[r].clone()
+        mb.medusa_attention_rescale(lses, r, part, lse2)
+        acc += part
+    torch.cuda.synchronize()
+    assert (acc - out).abs().max().item() <= 1e-5
+    assert torch.allclose(lse2, lse, atol=1e-6, rtol=0)
+
+
+def test_rescale_kernel_matches_oracle_with_empty_windows(mb):
+    rng = np.random.default_rng(4)
+    G, rows, hd = 4, 500, 128
+    outs = rng.normal(size=(G, rows, hd)).astype(np.float32)
+    lses = rng.normal(scale=4.0, size=(G, rows)).astype(np.float32)
+    lses[:, 10] = -np.inf
+    lses[1:, 11] = -np.inf
+    lses[0, 12:40] = -np.inf
+    ref_o, ref_l = O.combine_partials(outs.astype(np.float64), lses.astype(np.float64))
+    lg = torch.from_numpy(lses).cuda()
+    acc = torch.zeros(rows, hd, device="cuda")
+    lse = torch.empty(rows, device="cuda")
+    for r in range(G):
+        part = torch.from_numpy(outs[r]).cuda()
+        mb.medusa_attention_rescale(lg, r, part, lse)
+        acc += part
+    torch.cuda.synchronize()
+    assert np.allclose(_np(acc), ref_o, atol=1e-5, rtol=1e-5)
+    got_l = _np(lse)
+    assert np.all(got_l[10] == -np.inf) and not _np(acc)[10].any()
+    fin = np.isfinite(ref_l)
+    assert np.allclose(got_l[fin], ref_l[fin], atol=1e-5, rtol=1e-5)

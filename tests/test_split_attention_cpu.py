@@ -126,3 +126,89 @@ def test_combine_rejects_overlap_and_misalignment(mb):
     assert "null pointer" in str(e.value)
     with pytest.raises(ValueError, match="CUDA tensors"):
         mb.medusa_attention_combine(outs, lses, torch.zeros(4, 8))
+
+
+# ---------------------------------------------------------------------------
+# tree_attention_sharded's exchange on two gloo ranks: each rank's window
+# output and lse, an all-gather of the lse values only, the per-rank scaling
+# by exp(lse_r - lse) and an all-reduce (sum) must give the unsplit oracle.
+# The two library calls are replaced by oracle stand-ins on the host, so what
+# runs here is the exchange itself.
+
+
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _sharded_main(rank, world, port, q):
+    import os
+    import sys
+    import torch
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import torch.distributed as dist
+    import oracle.medusa_oracle as Om
+    import speculative_decoding_heads_b200.sharded as sh
+    tr = Om.tree_tables(Om.ranksum_choices(3, 3, 9), 3, 3)
+    L, hd, layers, B, H = 23, 8, 1, 2, 2
+    rng = np.random.default_rng(11)
+    qq = rng.normal(size=(layers, B, tr["T"], H, hd))
+    kc = rng.normal(size=(layers, B, H, L + tr["T"], hd))
+    vc = rng.normal(size=(layers, B, H, L + tr["T"], hd))
+    lens = np.array([L, L - 6])
+    scale = 0.4
+
+    class _Tree:
+        T = tr["T"]
+
+    def split(tree, q, k_cache, v_cache, seq_lens, sc, r, G, out, lse, stream=None):
+        for l in range(layers):
+            for b in range(B):
+                for e in range(H):
+                    lo, hi = Om.attention_window(G, r, int(seq_lens[b]))
+                    o, s = Om.tree_attention_window_slice(tr, q[l, b, :, e].numpy(), k_cache[l, b, e].numpy(),
+                                                          v_cache[l, b, e].numpy(), int(seq_lens[b]), sc, lo, hi,
+                                                          with_tree=(r == G - 1))
+                    out[l, b, :, e] = torch.from_numpy(o)
+                    lse[l, b, :, e] = torch.from_numpy(s)
+
+    def rescale(lses, r, part, lse_out=None, stream=None):
+        tot = torch.logsumexp(lses, dim=0)
+        part *= torch.exp(lses[r] - tot).unsqueeze(-1)
+
+    sh.medusa_tree_attention_split = split
+    sh.medusa_attention_rescale = rescale
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        out = torch.zeros((layers, B, tr["T"], H, hd), dtype=torch.float64)
+        sh.tree_attention_sharded(_Tree(), torch.from_numpy(qq), torch.from_numpy(kc), torch.from_numpy(vc),
+                                  torch.from_numpy(lens), scale, out)
+        err = 0.0
+        for l in range(layers):
+            for b in range(B):
+                for e in range(H):
+                    ref = Om.tree_attention_slice(tr, qq[l, b, :, e], kc[l, b, e], vc[l, b, e], int(lens[b]), scale)
+                    err = max(err, float(np.abs(out[l, b, :, e].numpy() - ref).max()))
+        q.put((rank, err))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_attention_exchange_two_gloo_ranks(built):
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sharded_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=5) for _ in range(2))
+    assert [r for r, _ in res] == [0, 1]
+    # the lse buffers are fp32, as the library's are: about 1e-7 of rounding
+    assert all(err < 1e-5 for _, err in res), res

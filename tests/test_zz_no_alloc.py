@@ -7,6 +7,8 @@ call after call, because it keeps its scratch in one fixed array that every
 call reuses.  The file name makes pytest collect it last.
 """
 
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -62,8 +64,12 @@ def test_noalloc_rejects_shapes_above_its_fixed_scratch(mb):
     Wout = torch.zeros((K, V, d), dtype=torch.bfloat16, device="cuda")
     ids = torch.full((B, K, topk), -3, dtype=torch.int32, device="cuda")
     vals = torch.zeros((B, K, topk), dtype=torch.float32, device="cuda")
+    # Straight through the C ABI: the size check comes before any pointer is
+    # used, so h stands in for W1 and b1 here (the binding would refuse their shapes).
+    p = lambda x: ctypes.c_void_p(x.data_ptr())
     with pytest.raises(mb.MedusaError) as ei:
-        mb.medusa_heads_topk_noalloc(h, h, h, Wout, topk, ids, vals)
+        mb._check(mb._lib.medusa_heads_topk_noalloc(p(h), p(h), p(h), p(Wout), B, d, V, K, topk, mb.MEDUSA_BF16,
+                                                    None, p(ids), p(vals), None))
     assert ei.value.code == mb.MEDUSA_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert (ids == -3).all()
