@@ -39,7 +39,13 @@ Readings where the pages are silent or disagree:
     above min(eps, alpha * exp(-H)), H the natural-log entropy of the same
     tempered distribution;  ties: top-k by (value desc, id asc), argmax by
     lowest id, best path by lowest path index;  the next token is the argmax
-    at the last accepted node in both modes;
+    at the last accepted node;
+  * the API's sampling='nucleus' with top_p (default 0.8) accepts a child
+    whose token lies in the top_p nucleus of the parent's tempered
+    distribution (the typical rule's form, with nucleus membership in place
+    of the threshold);  given one caller-drawn uniform u per sequence, the
+    next token is drawn instead, by inverse CDF in token-id order, from the
+    last accepted node's tempered distribution (typical) or its nucleus;
   * after acceptance the a+1 accepted nodes' K/V rows move to prefix
     positions L_b..L_b+a and the sequence grows by a+1.
 """
@@ -320,18 +326,44 @@ def node_statistics(logits_b: np.ndarray, temperature: float, eps: float, alpha:
     return dict(argmax=argmax, prob=prob, entropy=ent, threshold=thr)
 
 
+def nucleus_mask(prob_row: np.ndarray, top_p: float) -> np.ndarray:
+    """The top-p nucleus of one distribution, as a boolean mask over the vocabulary.
+
+    Tokens are taken in order of probability (descending, lower id first on
+    equal values) for as long as the mass of the tokens taken before them is
+    below top_p: the shortest such prefix whose mass reaches top_p.
+    """
+    prob_row = np.asarray(prob_row, dtype=np.float64)
+    order = np.lexsort((np.arange(prob_row.shape[0]), -prob_row))
+    before = np.concatenate([[0.0], np.cumsum(prob_row[order])[:-1]])
+    mask = np.zeros(prob_row.shape[0], dtype=bool)
+    mask[order] = before < top_p
+    return mask
+
+
+def sample_index(weights: np.ndarray, u: float) -> int:
+    """An inverse-CDF draw in token-id order: the first v whose cumulative
+    weight exceeds u * (total weight), u in [0, 1).  Zero weights are never drawn."""
+    c = np.cumsum(np.asarray(weights, dtype=np.float64))
+    return int(np.searchsorted(c, u * c[-1], side="right"))
+
+
 def evaluate_posterior(tree, logits, candidates, mode: str, temperature=0.0,
-                       eps=0.09, alpha=0.3):
+                       eps=0.09, alpha=0.3, top_p=0.8, uniforms=None):
     """Best path, accept length, accepted tokens and next token per sequence.
 
     logits [B, T, V] base-model logits at each tree node; candidates
     [B, P, D+1] from ``build_tree``.  For path p and depth j the child token
     candidates[b, p, j] is accepted when (greedy) it equals the argmax of its
-    parent's logits, or (typical) its tempered probability at the parent is
-    strictly above the parent's threshold.  acc_p counts the leading accepted
-    depths; the best path is the lowest p with the largest acc_p; a = acc_best.
-    accepted_tokens = candidates[b, best, 0..a] padded with -1; next_token =
-    argmax of the logits at node retrieve[best, a].
+    parent's logits, (typical) its tempered probability at the parent is
+    strictly above the parent's threshold, or (nucleus) it lies in the top_p
+    nucleus of the parent's tempered distribution.  acc_p counts the leading
+    accepted depths; the best path is the lowest p with the largest acc_p;
+    a = acc_best.  accepted_tokens = candidates[b, best, 0..a] padded with -1.
+    next_token is taken at node n = retrieve[best, a]: the argmax of its logits
+    when ``uniforms`` is None or in greedy mode; otherwise an inverse-CDF draw
+    with uniforms[b] from n's tempered distribution (typical) or from that
+    distribution restricted to its nucleus (nucleus).
     """
     B, T, V = logits.shape
     P, D = tree["P"], tree["D"]
@@ -341,8 +373,11 @@ def evaluate_posterior(tree, logits, candidates, mode: str, temperature=0.0,
     accepted = np.full((B, D + 1), -1, dtype=np.int64)
     nxt = np.zeros(B, dtype=np.int64)
     accs = np.zeros((B, P), dtype=np.int64)
+    if mode not in ("greedy", "typical", "nucleus"):
+        raise ValueError(mode)
     for b in range(B):
-        st = node_statistics(logits[b], temperature if mode == "typical" else None, eps, alpha)
+        st = node_statistics(logits[b], temperature if mode != "greedy" else None, eps, alpha)
+        nucleus = {}
         for p in range(P):
             acc = 0
             for j in range(1, D + 1):
@@ -356,7 +391,9 @@ def evaluate_posterior(tree, logits, candidates, mode: str, temperature=0.0,
                 elif mode == "typical":
                     ok = st["prob"][par, tok] > st["threshold"][par]
                 else:
-                    raise ValueError(mode)
+                    if par not in nucleus:
+                        nucleus[par] = nucleus_mask(st["prob"][par], top_p)
+                    ok = bool(nucleus[par][tok])
                 if not ok:
                     break
                 acc += 1
@@ -365,7 +402,14 @@ def evaluate_posterior(tree, logits, candidates, mode: str, temperature=0.0,
         best[b] = bp
         alen[b] = accs[b, bp]
         accepted[b, :alen[b] + 1] = candidates[b, bp, :alen[b] + 1]
-        nxt[b] = st["argmax"][ret[bp, alen[b]]]
+        last = ret[bp, alen[b]]
+        if uniforms is None or mode == "greedy":
+            nxt[b] = st["argmax"][last]
+        else:
+            w = st["prob"][last]
+            if mode == "nucleus":
+                w = np.where(nucleus_mask(w, top_p), w, 0.0)
+            nxt[b] = sample_index(w, float(uniforms[b]))
     return dict(best_path=best, accept_len=alen, accepted_tokens=accepted,
                 next_token=nxt, path_accept=accs)
 
@@ -432,6 +476,37 @@ def typical_margin_ok(tree, logits, candidates, temperature, eps, alpha,
                 if abs(pr - th) < rel * max(pr, th):
                     return False
     return True
+
+
+def nucleus_margin_ok(logits, temperature, top_p, rel: float = 1e-4) -> bool:
+    """True when every node's nucleus boundary is clear of top_p by >= rel (of
+    the total mass 1) on both sides, and its last member's probability is
+    >= rel (relative) above the next token's, so that every membership
+    decision holds under any summation order.  logits [B, T, V]."""
+    z = np.asarray(logits, dtype=np.float64)
+    for b in range(z.shape[0]):
+        st = node_statistics(z[b], temperature, 0.0, 0.0)
+        for i in range(z.shape[1]):
+            pr = st["prob"][i]
+            order = np.lexsort((np.arange(pr.shape[0]), -pr))
+            cum = np.cumsum(pr[order])
+            m = int(np.searchsorted(cum, top_p, side="left"))   # first prefix reaching top_p
+            m = min(m, pr.shape[0] - 1)
+            before = cum[m - 1] if m > 0 else 0.0
+            if top_p - before < rel or cum[m] - top_p < rel:
+                return False
+            if m + 1 < pr.shape[0] and pr[order[m]] - pr[order[m + 1]] < rel * pr[order[m]]:
+                return False
+    return True
+
+
+def sample_margin_ok(weights, u: float, rel: float = 1e-4) -> bool:
+    """True when u * total lies >= rel * total inside the drawn token's CDF interval."""
+    c = np.cumsum(np.asarray(weights, dtype=np.float64))
+    x = u * c[-1]
+    v = int(np.searchsorted(c, x, side="right"))
+    lo = c[v - 1] if v > 0 else 0.0
+    return x - lo >= rel * c[-1] and c[v] - x >= rel * c[-1]
 
 
 def attention_scale(hd: int) -> float:

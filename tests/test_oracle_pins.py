@@ -402,6 +402,146 @@ def test_typical_bruteforce(seed):
 
 
 # ---------------------------------------------------------------------------
+# nucleus acceptance and the sampled next token
+# ---------------------------------------------------------------------------
+
+
+def _nucleus_brute(pr, top_p):
+    """Smallest m such that the m most probable tokens (lower id first on ties) hold >= top_p."""
+    order = sorted(range(len(pr)), key=lambda i: (-pr[i], i))
+    for m in range(1, len(pr) + 1):
+        if sum(pr[i] for i in order[:m]) >= top_p:
+            return set(order[:m])
+    return set(order)
+
+
+def check_nucleus_mask(O):
+    pr = np.array([0.2, 0.5, 0.3])
+    assert list(O.nucleus_mask(pr, 0.8)) == [False, True, True]   # 0.5 + 0.3 reaches 0.8 exactly
+    assert list(O.nucleus_mask(pr, 0.81)) == [True, True, True]
+    assert list(O.nucleus_mask(pr, 0.5)) == [False, True, False]
+    assert list(O.nucleus_mask(pr, 1e-9)) == [False, True, False]  # only the most probable token
+    assert list(O.nucleus_mask(np.full(4, 0.25), 0.5)) == [True, True, False, False]   # ties by id
+    rng = np.random.default_rng(7)
+    for _ in range(40):
+        V = int(rng.integers(2, 12))
+        pr = rng.dirichlet(np.ones(V) * 0.7)
+        pr[rng.integers(V)] = pr[rng.integers(V)]                 # an exact tie now and then
+        pr = pr / pr.sum()
+        for top_p in (0.3, 0.8, 0.95):
+            got = set(np.flatnonzero(O.nucleus_mask(pr, top_p)))
+            assert got == _nucleus_brute(pr, top_p), (pr, top_p)
+
+
+def test_nucleus_mask():
+    check_nucleus_mask(O)
+
+
+def check_sample_index(O):
+    w = np.array([1.0, 0.0, 3.0])
+    assert O.sample_index(w, 0.0) == 0
+    assert O.sample_index(w, 0.2499) == 0
+    assert O.sample_index(w, 0.25) == 2          # cumulative 1.0 is not above 0.25 * 4: token 1 has no weight
+    assert O.sample_index(w, 0.999) == 2
+    # a fine grid of u reproduces the weights
+    w = np.array([0.1, 0.0, 0.45, 0.2, 0.25])
+    n = 20000
+    counts = np.bincount([O.sample_index(w, (i + 0.5) / n) for i in range(n)], minlength=5)
+    assert np.abs(counts / n - w / w.sum()).max() <= 1.0 / n
+
+
+def test_sample_index():
+    check_sample_index(O)
+
+
+def check_nucleus_posterior(O, seed):
+    rng = np.random.default_rng(seed)
+    K, topk, V = 3, 3, 10
+    tr = O.tree_tables(O.ranksum_choices(K, topk, 12), K, topk)
+    topk_ids = np.stack([rng.permutation(V)[:topk] for _ in range(K)])[None]
+    toks, cand, _ = O.build_tree(tr, np.array([4]), topk_ids, np.array([0]))
+    z = rng.normal(scale=1.5, size=(1, tr["T"], V))
+    for temp, top_p in [(0.7, 0.8), (1.3, 0.5), (0.4, 0.95)]:
+        u = np.array([rng.random()])
+        post = O.evaluate_posterior(tr, z, cand, "nucleus", temp, top_p=top_p, uniforms=u)
+        accs = []
+        probs_of = lambda node: [math.exp(z[0, node, v] / temp) / sum(math.exp(z[0, node, x] / temp) for x in range(V))
+                                 for v in range(V)]
+        for p in range(tr["P"]):
+            acc = 0
+            for j in range(1, tr["D"] + 1):
+                node = tr["retrieve"][p][j]
+                if node < 0:
+                    break
+                if cand[0, p, j] not in _nucleus_brute(probs_of(tr["retrieve"][p][j - 1]), top_p):
+                    break
+                acc += 1
+            accs.append(acc)
+        best = accs.index(max(accs))
+        assert post["best_path"][0] == best and post["accept_len"][0] == max(accs)
+        last = tr["retrieve"][best][max(accs)]
+        pr = probs_of(last)
+        nuc = _nucleus_brute(pr, top_p)
+        w = [pr[v] if v in nuc else 0.0 for v in range(V)]
+        tot, cum, draw = sum(w), 0.0, None
+        for v in range(V):
+            cum += w[v]
+            if cum > u[0] * tot:
+                draw = v
+                break
+        assert post["next_token"][0] == draw
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_nucleus_posterior_bruteforce(seed):
+    check_nucleus_posterior(O, seed)
+
+
+def test_nucleus_and_sampling_special_cases():
+    rng = np.random.default_rng(5)
+    K, topk, V = 4, 3, 40
+    tr = O.tree_tables(O.ranksum_choices(K, topk, 30), K, topk)
+    topk_ids = np.stack([rng.permutation(V)[:topk] for _ in range(K)])[None]
+    toks, cand, _ = O.build_tree(tr, np.array([1]), topk_ids, np.array([0]))
+    z = _planted_logits(tr, toks, V, 0.8, seed=5)
+    greedy = O.evaluate_posterior(tr, z, cand, "greedy")
+    # top_p -> 0: the nucleus is the argmax alone, so acceptance is greedy acceptance
+    tiny = O.evaluate_posterior(tr, z, cand, "nucleus", 1.0, top_p=1e-12)
+    for k in ("best_path", "accept_len", "accepted_tokens", "next_token"):
+        assert np.array_equal(tiny[k], greedy[k]), k
+    # ... and a draw from a one-token nucleus is that token, whatever u
+    for u in (0.0, 0.37, 0.9999):
+        assert O.evaluate_posterior(tr, z, cand, "nucleus", 1.0, top_p=1e-12,
+                                    uniforms=np.array([u]))["next_token"][0] == greedy["next_token"][0]
+    # top_p = 1 keeps every token: every candidate of nonzero probability is accepted
+    full = O.evaluate_posterior(tr, z, cand, "nucleus", 1.0, top_p=1.0)
+    assert full["accept_len"][0] == tr["D"]
+    assert full["best_path"][0] == int(np.argmax((tr["retrieve"] >= 0).sum(1)))   # the first path of full depth
+    # without uniforms the typical and nucleus next token is the argmax (the reading used so far)
+    typ = O.evaluate_posterior(tr, z, cand, "typical", 0.7)
+    assert typ["next_token"][0] == int(np.argmax(z[0, tr["retrieve"][typ["best_path"][0], typ["accept_len"][0]]]))
+
+
+def check_sampling_guards(O):
+    # nucleus boundary: probabilities [0.5, 0.3, 0.2]; at top_p 0.8 the boundary mass is exactly top_p
+    z = np.log(np.array([[[0.5, 0.3, 0.2]]]))
+    assert not O.nucleus_margin_ok(z, 1.0, 0.8)
+    assert O.nucleus_margin_ok(z, 1.0, 0.7)                    # 0.5 < 0.7 - 1e-4 and 0.8 > 0.7 + 1e-4
+    assert not O.nucleus_margin_ok(z, 1.0, 0.5 + 5e-5)         # the mass before the last member is too close
+    # the last member and the first token left out tie: which one is in depends on rounding
+    assert not O.nucleus_margin_ok(np.log(np.array([[[0.4, 0.3, 0.3]]])), 1.0, 0.6)
+    assert O.nucleus_margin_ok(np.log(np.array([[[0.4, 0.4, 0.2]]])), 1.0, 0.6)    # a tie inside the nucleus is harmless
+    # the draw's interval: weights [1, 3], u * 4 = 1 exactly is a boundary
+    assert not O.sample_margin_ok([1.0, 3.0], 0.25)
+    assert not O.sample_margin_ok([1.0, 3.0], 0.25 - 1e-5)
+    assert O.sample_margin_ok([1.0, 3.0], 0.25 + 1e-3) and O.sample_margin_ok([1.0, 3.0], 0.1)
+
+
+def test_sampling_guards():
+    check_sampling_guards(O)
+
+
+# ---------------------------------------------------------------------------
 # accept KV
 # ---------------------------------------------------------------------------
 
@@ -616,6 +756,22 @@ def _margin_rel_smaller(tree, logits, candidates, temperature, eps, alpha, rel=1
     return True
 
 
+def _nucleus_inclusive(prob_row, top_p):
+    prob_row = np.asarray(prob_row, dtype=np.float64)
+    order = np.lexsort((np.arange(prob_row.shape[0]), -prob_row))
+    before = np.concatenate([[0.0], np.cumsum(prob_row[order])[:-1]])
+    mask = np.zeros(prob_row.shape[0], dtype=bool)
+    mask[order] = before <= top_p                # keeps one token too many at an exact boundary
+    return mask
+
+
+def _draw_by_probability(weights, u):
+    w = np.asarray(weights, dtype=np.float64)
+    order = np.argsort(-w, kind="stable")         # walks the CDF in probability order, not id order
+    c = np.cumsum(w[order])
+    return int(order[np.searchsorted(c, u * c[-1], side="right")])
+
+
 def _tables_bad_index(choices, K, topk):
     tr = O.tree_tables(choices, K, topk)
     tr = dict(tr)
@@ -639,6 +795,10 @@ MUTANTS = {
     "gap guard relative to the smaller value": (dict(topk_gap_ok=_gap_rel_smaller), [check_topk_gap_guard]),
     "margin guard relative to the smaller value": (dict(typical_margin_ok=_margin_rel_smaller),
                                                    [check_typical_margin_guard]),
+    "nucleus keeps the token at the boundary": (dict(nucleus_mask=_nucleus_inclusive),
+                                                [check_nucleus_mask, lambda M: check_nucleus_posterior(M, 0)]),
+    "draw in probability order": (dict(sample_index=_draw_by_probability),
+                                  [check_sample_index, lambda M: check_nucleus_posterior(M, 1)]),
 }
 
 
