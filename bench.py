@@ -176,6 +176,7 @@ class OracleSample:
         self.sub_l = sub_l
         self.logits = None
         self.cores = 1
+        self.sample_times = []      # measured seconds of each sampled step, before the scaling
         self.desc = (f"heads, top-k, tree and posterior in full; attention and KV compaction on "
                      f"{len(self.slices)} of {total} (layer, seq, head) slices, scaled x{self.scale_slices:.0f}; "
                      f"fp64, 1 BLAS thread")
@@ -208,6 +209,7 @@ class OracleSample:
             k2[L:L + a + 1] = k[rows]
             v2[L:L + a + 1] = v[rows]
         t_sample = time.perf_counter() - t2
+        self.sample_times.append(t_full + t_sample)
         return t_full + t_sample * self.scale_slices
 
 
@@ -235,7 +237,10 @@ def run_reference(a, w):
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w),
-            "cpu_baseline": {"value": us, "unit": "us", "cores": samp.cores, "kind": "oracle", "sample": samp.desc},
+            # the value is a full step's time extrapolated from a sampled one (see "sample")
+            "extrapolated": True, "measured_sample_us": statistics.median(samp.sample_times) * 1e6,
+            "cpu_baseline": {"value": us, "unit": "us", "cores": samp.cores, "host_cores": os.cpu_count(),
+                             "kind": "oracle", "sample": samp.desc},
             "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -292,8 +297,8 @@ def run_ours(a, w):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
-    # heads (+ tree build) per group of <= 4 sequences, attention, posterior, accept rows, length update
-    launches_per_step = (w.B + 3) // 4 + 1 + 1 + 2
+    # heads (+ tree build) per group of <= 4 sequences, attention, posterior with the KV compaction
+    launches_per_step = (w.B + 3) // 4 + 1 + 1
 
     def step():
         t["seq_lens"].copy_(t["seq_lens0"])
@@ -347,6 +352,24 @@ def run_ours(a, w):
     if st != 0:
         raise RuntimeError(f"device status {st} detail {det} after the timed region")
 
+    # ---- per-step distribution, graph replay and eager launches side by side ----
+    def per_step(fn, k):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(k + 1)]
+        with torch.cuda.stream(stream):
+            evs[0].record(stream)
+            for i in range(k):
+                fn()
+                evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+        xs = sorted(evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(k))
+        return {"mean": statistics.mean(xs), "median": statistics.median(xs), "min": xs[0],
+                "p90": xs[min(k - 1, int(round(0.9 * (k - 1))))], "n": k}
+
+    dist_steps = max(a.steps, 20)
+    step_us = {"eager": per_step(step, dist_steps)}
+    if graph is not None:
+        step_us["graph"] = per_step(graph.replay, dist_steps)
+
     # ---- per-stage breakdown (eager, CUDA events on the launching stream) ----
     peak, peak_kind = load_peaks()
     stage = {}
@@ -382,9 +405,8 @@ def run_ours(a, w):
     esz = 2 if w.dtype == "bf16" else 4
     head_bytes = w.K * (w.d * w.d + w.d + w.V * w.d) * esz
     kv_bytes = w.metric_bytes() - head_bytes
-    # The heads kernel reads the weights once per group of up to four sequences, one launch each.
-    head_launches = (w.B + 3) // 4
-    heads_gbs = head_bytes * head_launches / (stage["heads_topk"] * 1e-6) / 1e9
+    # Algorithmic bytes: the head weights once per step, whatever the batch.
+    heads_gbs = head_bytes / (stage["heads_topk"] * 1e-6) / 1e9
     attn_gbs = kv_bytes / (stage["tree_attention"] * 1e-6) / 1e9
     traffic = None
     tpath = os.path.join(REPO, "profiles", "heads_topk_traffic.json")
@@ -425,7 +447,8 @@ def run_ours(a, w):
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         samp = OracleSample(w)
         secs = [samp.step_seconds() for _ in range(2)]
-        cpu = {"value": min(secs) * 1e6, "unit": "us", "cores": samp.cores, "kind": "oracle", "sample": samp.desc}
+        cpu = {"value": min(secs) * 1e6, "unit": "us", "cores": samp.cores, "host_cores": os.cpu_count(),
+               "kind": "oracle", "sample": samp.desc, "extrapolated": True}
 
     if world > 1:
         dist.barrier()
@@ -443,6 +466,7 @@ def run_ours(a, w):
         "achieved_step_gbs": w.metric_bytes() / (us * 1e-6) / 1e9,
         "tree_tokens_per_s": world * w.B * w.T / (us * 1e-6),
         "stage_us": stage,
+        "step_us": step_us,
         "roofline": {"bound": "hbm", "kernel": "heads_topk", "achieved": heads_gbs, "peak": peak,
                      "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback 6650 GB/s", "unit": "GB/s", "frac": heads_gbs / peak, "traffic": traffic,

@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define MEDUSA_ABI_VERSION 3
+#define MEDUSA_ABI_VERSION 4
 #define MEDUSA_MAX_T 256     /* tree tokens including the root */
 #define MEDUSA_MAX_K 16      /* heads (so tree depth <= 16) */
 #define MEDUSA_MAX_TOPK 32   /* candidates per head */
@@ -89,7 +89,12 @@ typedef enum medusa_status {
 
 typedef enum medusa_dtype { MEDUSA_F32 = 0, MEDUSA_BF16 = 1 } medusa_dtype_t;
 
-typedef enum medusa_mode { MEDUSA_GREEDY = 0, MEDUSA_TYPICAL = 1 } medusa_mode_t;
+/* Acceptance rule of the posterior (S6).  NUCLEUS is the API's
+ * sampling='nucleus' with top_p ("Medusa API参考", evaluate_posterior); the
+ * pages name it without defining it, and this library reads it in the form
+ * of the typical rule: a child is accepted when its token lies in the top_p
+ * nucleus of its parent's tempered distribution. */
+typedef enum medusa_mode { MEDUSA_GREEDY = 0, MEDUSA_TYPICAL = 1, MEDUSA_NUCLEUS = 2 } medusa_mode_t;
 
 typedef struct medusa_tree medusa_tree_t;
 
@@ -310,19 +315,28 @@ medusa_status_t medusa_attention_rescale(int G, int rank, int64_t rows, int hd, 
 size_t medusa_posterior_workspace_size(const medusa_tree_t* tree, int B);
 
 /* Per node i of sequence b: g_i = argmax_v logits[b,i,v] (lowest id on ties);
- * typical: p_i = softmax(logits[b,i,:] / temperature), H_i = -sum p ln p,
- * thr_i = min(eps, alpha * exp(-H_i)).
- * Path p accepts depth j when candidates[b,p,j] == g_parent (GREEDY) or
- * p_parent(candidates[b,p,j]) > thr_parent (TYPICAL); acc_p counts leading
- * accepted depths.  best_path[b] = lowest p with the largest acc_p;
- * accept_len[b] = a = acc_best (0..D); accepted_tokens[b, 0..D] =
- * candidates[b, best, 0..a], -1 after; next_token[b] = g at node
- * retrieve[best, a].  TYPICAL needs temperature > 0 (defaults of the pages:
- * eps = 0.09, alpha = 0.3).  logits [B,T,V] fp32; candidates [B,P,D+1]. */
+ * typical / nucleus: p_i = softmax(logits[b,i,:] / temperature),
+ * H_i = -sum p ln p, thr_i = min(eps, alpha * exp(-H_i)); the nucleus N_i
+ * holds the tokens, in order of p descending (lower id first on equal
+ * values), whose preceding mass is below top_p.
+ * Path p accepts depth j when candidates[b,p,j] == g_parent (GREEDY),
+ * p_parent(candidates[b,p,j]) > thr_parent (TYPICAL), or candidates[b,p,j]
+ * is in N_parent (NUCLEUS); acc_p counts leading accepted depths.
+ * best_path[b] = lowest p with the largest acc_p; accept_len[b] = a = acc_best
+ * (0..D); accepted_tokens[b, 0..D] = candidates[b, best, 0..a], -1 after.
+ * next_token[b], at node n = retrieve[best, a]: g_n when uniforms is NULL or
+ * mode is GREEDY; otherwise the first token v, in id order, whose cumulative
+ * weight exceeds uniforms[b] * (total weight), the weights being p_n (TYPICAL)
+ * or p_n restricted to N_n (NUCLEUS): a draw by inverse CDF with the
+ * caller's uniform (uniforms [B] fp32 in [0, 1), device).
+ * TYPICAL and NUCLEUS need temperature > 0; NUCLEUS needs 0 < top_p <= 1
+ * (defaults of the pages: eps = 0.09, alpha = 0.3, top_p = 0.8).
+ * logits [B,T,V] fp32; candidates [B,P,D+1]. */
 medusa_status_t medusa_evaluate_posterior(const medusa_tree_t* tree, int B, int V,
                                           const float* logits, const int32_t* candidates,
                                           medusa_mode_t mode, float temperature, float eps,
-                                          float alpha, int32_t* best_path, int32_t* accept_len,
+                                          float alpha, float top_p, const float* uniforms,
+                                          int32_t* best_path, int32_t* accept_len,
                                           int32_t* accepted_tokens, int32_t* next_token,
                                           void* workspace, size_t workspace_bytes,
                                           cudaStream_t stream);
@@ -380,6 +394,8 @@ typedef struct medusa_step_args {
    * copy those inputs on another stream while the heads run. */
   cudaEvent_t attn_inputs_ready;
   cudaEvent_t posterior_inputs_ready;
+  float top_p;                    /* nucleus acceptance (MEDUSA_NUCLEUS) */
+  const float* uniforms;          /* [B] or NULL: draws for the next token (see medusa_evaluate_posterior) */
 } medusa_step_args_t;
 
 size_t medusa_step_workspace_size(const medusa_step_args_t* args);
@@ -388,8 +404,9 @@ size_t medusa_step_workspace_size(const medusa_step_args_t* args);
  * medusa_tree_attention, medusa_evaluate_posterior and medusa_accept_kv, in
  * that order, on stream, with the same outputs.  The candidate tree is built
  * by the heads kernel's last CTA (one launch for S1-S4 per group of up to
- * four sequences); five launches per step at B <= 4.  Capturable in a CUDA
- * graph (no allocation, no synchronisation).  Validation errors are returned
+ * four sequences), and the posterior and the compaction share one launch
+ * (S6-S7): three launches per step at B <= 4.  Capturable in a CUDA graph
+ * (no allocation, no synchronisation).  Validation errors are returned
  * before anything is enqueued. */
 medusa_status_t medusa_step(const medusa_step_args_t* args, void* workspace,
                             size_t workspace_bytes, cudaStream_t stream);

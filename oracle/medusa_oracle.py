@@ -478,30 +478,51 @@ def typical_margin_ok(tree, logits, candidates, temperature, eps, alpha,
     return True
 
 
-def nucleus_margin_ok(logits, temperature, top_p, rel: float = 1e-4) -> bool:
-    """True when every node's nucleus boundary is clear of top_p by >= rel (of
-    the total mass 1) on both sides, and its last member's probability is
-    >= rel (relative) above the next token's, so that every membership
-    decision holds under any summation order.  logits [B, T, V]."""
-    z = np.asarray(logits, dtype=np.float64)
-    for b in range(z.shape[0]):
-        st = node_statistics(z[b], temperature, 0.0, 0.0)
-        for i in range(z.shape[1]):
-            pr = st["prob"][i]
-            order = np.lexsort((np.arange(pr.shape[0]), -pr))
-            cum = np.cumsum(pr[order])
-            m = int(np.searchsorted(cum, top_p, side="left"))   # first prefix reaching top_p
-            m = min(m, pr.shape[0] - 1)
-            before = cum[m - 1] if m > 0 else 0.0
-            if top_p - before < rel or cum[m] - top_p < rel:
-                return False
-            if m + 1 < pr.shape[0] and pr[order[m]] - pr[order[m + 1]] < rel * pr[order[m]]:
-                return False
+# The nucleus decisions are comparisons of sums of tempered probabilities
+# with top_p.  Summed in fp32 over at most 65536 tokens, as the GPU does, such
+# a sum is off by at most a few 1e-6 of the total mass, so these guards keep
+# every such decision at least 1e-5 of the total mass away from its boundary.
+NUCLEUS_REL = 1e-5
+
+
+def nucleus_margin_ok(tree, logits, candidates, temperature, top_p, rel: float = NUCLEUS_REL) -> bool:
+    """True when, on every tree edge, the tempered mass of the tokens ranking
+    before the child's token (larger probability, or equal and lower id) is at
+    least rel away from top_p, so its nucleus membership holds under any
+    summation order.  logits [B, T, V]; candidates [B, P, D+1]."""
+    ret = tree["retrieve"]
+    for b in range(logits.shape[0]):
+        st = node_statistics(logits[b], temperature, 0.0, 0.0)
+        for p in range(tree["P"]):
+            for j in range(1, tree["D"] + 1):
+                if ret[p, j] < 0:
+                    break
+                pr = st["prob"][ret[p, j - 1]]
+                tok = int(candidates[b, p, j])
+                ids = np.arange(pr.shape[0])
+                before = pr[(pr > pr[tok]) | ((pr == pr[tok]) & (ids < tok))].sum()
+                if abs(before - top_p) < rel:
+                    return False
     return True
 
 
-def sample_margin_ok(weights, u: float, rel: float = 1e-4) -> bool:
-    """True when u * total lies >= rel * total inside the drawn token's CDF interval."""
+def nucleus_cut_ok(prob_row, top_p, rel: float = NUCLEUS_REL) -> bool:
+    """True when one distribution's nucleus boundary is clear: top_p is at
+    least rel from the mass before its last member and from the mass through
+    it, and that member's probability is above the next token's by at least
+    1e-6 relative (so no rounding can reorder the two)."""
+    pr = np.asarray(prob_row, dtype=np.float64)
+    order = np.lexsort((np.arange(pr.shape[0]), -pr))
+    cum = np.cumsum(pr[order])
+    m = min(int(np.searchsorted(cum, top_p, side="left")), pr.shape[0] - 1)   # first prefix reaching top_p
+    before = cum[m - 1] if m > 0 else 0.0
+    if top_p - before < rel or cum[m] - top_p < rel:
+        return False
+    return not (m + 1 < pr.shape[0] and pr[order[m]] - pr[order[m + 1]] < 1e-6 * pr[order[m]])
+
+
+def sample_margin_ok(weights, u: float, rel: float = NUCLEUS_REL) -> bool:
+    """True when u * total lies at least rel * total inside the drawn token's CDF interval."""
     c = np.cumsum(np.asarray(weights, dtype=np.float64))
     x = u * c[-1]
     v = int(np.searchsorted(c, x, side="right"))

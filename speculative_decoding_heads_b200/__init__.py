@@ -26,7 +26,7 @@ if not os.path.exists(LIB_PATH):
         "`python -m speculative_decoding_heads_b200._build` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
-ABI_VERSION = 3   # layout of medusa_step_args_t (StepArgs below) and of every signature
+ABI_VERSION = 4   # layout of medusa_step_args_t (StepArgs below) and of every signature
 _lib.medusa_abi_version.restype = ctypes.c_int
 if _lib.medusa_abi_version() != ABI_VERSION:
     raise ImportError(f"{LIB_PATH} has ABI version {_lib.medusa_abi_version()}, this binding needs "
@@ -42,6 +42,7 @@ MEDUSA_F32 = 0
 MEDUSA_BF16 = 1
 MEDUSA_GREEDY = 0
 MEDUSA_TYPICAL = 1
+MEDUSA_NUCLEUS = 2
 MAX_T, MAX_K, MAX_TOPK, MAX_B, MAX_SHARDS = 256, 16, 32, 64, 64
 
 # Every symbol the header declares (checked by the CPU tests).
@@ -86,6 +87,7 @@ class StepArgs(ctypes.Structure):
         ("attn_out", _vp),
         ("best_path", _vp), ("accept_len", _vp), ("accepted_tokens", _vp), ("next_token", _vp),
         ("attn_inputs_ready", _vp), ("posterior_inputs_ready", _vp),
+        ("top_p", _f32), ("uniforms", _vp),
     ]
 
 
@@ -118,7 +120,7 @@ _sig("medusa_attention_combine", _i32, [_i32, ctypes.c_int64, _i32, _vp, _vp, _v
 _sig("medusa_attention_rescale", _i32, [_i32, _i32, ctypes.c_int64, _i32, _vp, _vp, _vp, _vp])
 _sig("medusa_posterior_workspace_size", _sz, [_vp, _i32])
 _sig("medusa_evaluate_posterior", _i32,
-     [_vp, _i32, _i32, _vp, _vp, _i32, _f32, _f32, _f32, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
+     [_vp, _i32, _i32, _vp, _vp, _i32, _f32, _f32, _f32, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _sig("medusa_accept_kv", _i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp])
 _sig("medusa_step_workspace_size", _sz, [ctypes.POINTER(StepArgs)])
 _sig("medusa_step", _i32, [ctypes.POINTER(StepArgs), _vp, _sz, _vp])
@@ -413,7 +415,9 @@ def medusa_posterior_workspace_size(tree: Tree, B) -> int:
 
 def medusa_evaluate_posterior(tree: Tree, logits, candidates, mode, best_path, accept_len,
                               accepted_tokens, next_token, ws, temperature=0.0, eps=0.09,
-                              alpha=0.3, stream=None):
+                              alpha=0.3, top_p=0.8, uniforms=None, stream=None):
+    """S6.  ``uniforms`` [B] fp32 in [0, 1) (optional): the next token is drawn with them (typical
+    and nucleus modes) instead of taken as the arg-max."""
     _require(logits.dim() == 3, "logits must be [B, T, V]")
     B, T, V = logits.shape
     _require(T == tree.T, f"logits hold {T} tree nodes per sequence; the tree has {tree.T}")
@@ -422,10 +426,12 @@ def medusa_evaluate_posterior(tree: Tree, logits, candidates, mode, best_path, a
     for name, t in (("best_path", best_path), ("accept_len", accept_len), ("next_token", next_token)):
         _spec(name, t, (B,), torch.int32)
     _spec("accepted_tokens", accepted_tokens, (B, tree.D + 1), torch.int32)
+    if uniforms is not None:
+        _spec("uniforms", uniforms, (B,), torch.float32)
     nbytes = _nbytes("ws", ws)
     _check(_lib.medusa_evaluate_posterior(tree.handle, B, V, _p(logits), _p(candidates), int(mode),
-                                          float(temperature), float(eps), float(alpha),
-                                          _p(best_path), _p(accept_len), _p(accepted_tokens),
+                                          float(temperature), float(eps), float(alpha), float(top_p),
+                                          _p(uniforms), _p(best_path), _p(accept_len), _p(accepted_tokens),
                                           _p(next_token), _p(ws), nbytes, _stream(stream)))
 
 
@@ -443,8 +449,9 @@ def medusa_accept_kv(tree: Tree, k_cache, v_cache, seq_lens, best_path, accept_l
 
 
 def make_step_args(tree: Tree, t: dict, mode: int, temperature=0.0, eps=0.09, alpha=0.3,
-                   scale=None) -> StepArgs:
-    """Builds ``medusa_step_args_t`` from a dict of device tensors (see ``StepBuffers``)."""
+                   scale=None, top_p=0.8) -> StepArgs:
+    """Builds ``medusa_step_args_t`` from a dict of device tensors (the keys are the fields'
+    names; ``head_logits`` and ``uniforms`` may be absent or None)."""
     layers, B, T, H, hd, Lcap = _attention_specs(tree, t["q"], t["k_cache"], t["v_cache"], t["seq_lens"],
                                                  t["attn_out"])
     _require(t["q"].dtype == t["h"].dtype, "q and the caches must have the dtype of h and the weights")
@@ -474,6 +481,10 @@ def make_step_args(tree: Tree, t: dict, mode: int, temperature=0.0, eps=0.09, al
     a.scale = float(scale if scale is not None else hd ** -0.5)
     a.mode = int(mode)
     a.temperature, a.eps, a.alpha = float(temperature), float(eps), float(alpha)
+    a.top_p = float(top_p)
+    if t.get("uniforms") is not None:
+        _spec("uniforms", t["uniforms"], (B,), torch.float32)
+        a.uniforms = _p(t["uniforms"]).value
     return a
 
 

@@ -275,22 +275,25 @@ extern "C" size_t medusa_posterior_workspace_size(const medusa_tree_t* tree, int
 
 static medusa_status_t check_posterior(const medusa_tree_t* tree, int B, int V, const float* logits,
                                        const int32_t* candidates, medusa_mode_t mode, float temperature,
-                                       float eps, float alpha, const int32_t* best_path, const int32_t* accept_len,
-                                       const int32_t* accepted_tokens, const int32_t* next_token, const void* ws,
-                                       size_t ws_bytes) {
+                                       float eps, float alpha, float top_p, const int32_t* best_path,
+                                       const int32_t* accept_len, const int32_t* accepted_tokens,
+                                       const int32_t* next_token, const void* ws, size_t ws_bytes) {
   const char* fn = "medusa_evaluate_posterior";
   medusa_status_t st = check_tree(tree, fn);
   if (st != MEDUSA_OK) return st;
   if (!logits || !candidates || !best_path || !accept_len || !accepted_tokens || !next_token || !ws)
     return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
   if (B < 1 || B > MEDUSA_MAX_B || V < 1) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": B or V");
-  if (mode != MEDUSA_GREEDY && mode != MEDUSA_TYPICAL) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": mode");
-  if (mode == MEDUSA_TYPICAL) {
+  if (mode != MEDUSA_GREEDY && mode != MEDUSA_TYPICAL && mode != MEDUSA_NUCLEUS)
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": mode");
+  if (mode != MEDUSA_GREEDY) {
     if (!(temperature > 0.f) || !std::isfinite(temperature))
-      return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": typical acceptance needs temperature > 0");
+      return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": typical and nucleus acceptance need temperature > 0");
     if (!std::isfinite(eps) || !std::isfinite(alpha) || eps < 0.f || alpha < 0.f)
       return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": eps and alpha must be finite and >= 0");
   }
+  if (mode == MEDUSA_NUCLEUS && !(top_p > 0.f && top_p <= 1.f))
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": nucleus acceptance needs 0 < top_p <= 1");
   if (ws_bytes < posterior_workspace_bytes(tree->dev, B))
     return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": workspace too small");
   return MEDUSA_OK;
@@ -298,15 +301,17 @@ static medusa_status_t check_posterior(const medusa_tree_t* tree, int B, int V, 
 
 extern "C" medusa_status_t medusa_evaluate_posterior(const medusa_tree_t* tree, int B, int V, const float* logits,
                                                      const int32_t* candidates, medusa_mode_t mode,
-                                                     float temperature, float eps, float alpha, int32_t* best_path,
+                                                     float temperature, float eps, float alpha, float top_p,
+                                                     const float* uniforms, int32_t* best_path,
                                                      int32_t* accept_len, int32_t* accepted_tokens,
                                                      int32_t* next_token, void* workspace, size_t workspace_bytes,
                                                      cudaStream_t stream) {
-  medusa_status_t st = check_posterior(tree, B, V, logits, candidates, mode, temperature, eps, alpha, best_path,
-                                       accept_len, accepted_tokens, next_token, workspace, workspace_bytes);
+  medusa_status_t st = check_posterior(tree, B, V, logits, candidates, mode, temperature, eps, alpha, top_p,
+                                       best_path, accept_len, accepted_tokens, next_token, workspace,
+                                       workspace_bytes);
   if (st != MEDUSA_OK) return st;
-  return launch_posterior(tree->dev, B, V, logits, candidates, mode, temperature, eps, alpha, best_path,
-                          accept_len, accepted_tokens, next_token, workspace, stream);
+  return launch_posterior(tree->dev, B, V, logits, candidates, mode, temperature, eps, alpha, top_p, uniforms,
+                          best_path, accept_len, accepted_tokens, next_token, workspace, stream);
 }
 
 static medusa_status_t check_accept(const medusa_tree_t* tree, int layers, int B, int H, int hd,
@@ -383,7 +388,7 @@ extern "C" medusa_status_t medusa_step(const medusa_step_args_t* a, void* worksp
                        a->seq_lens, a->scale, a->attn_out);
   if (st != MEDUSA_OK) return st;
   st = check_posterior(a->tree, a->B, a->V, a->base_logits, a->candidates, a->mode, a->temperature, a->eps, a->alpha,
-                       a->best_path, a->accept_len, a->accepted_tokens, a->next_token, ws_post, l.post);
+                       a->top_p, a->best_path, a->accept_len, a->accepted_tokens, a->next_token, ws_post, l.post);
   if (st != MEDUSA_OK) return st;
   st = check_accept(a->tree, a->layers, a->B, a->H, a->hd, a->dtype, a->k_cache, a->v_cache, a->Lcap, a->seq_lens,
                     a->best_path, a->accept_len);
@@ -415,10 +420,10 @@ extern "C" medusa_status_t medusa_step(const medusa_step_args_t* a, void* worksp
     const cudaError_t e = cudaStreamWaitEvent(stream, a->posterior_inputs_ready, 0);
     if (e != cudaSuccess) return cuda_fail("medusa_step: wait for the posterior inputs", e);
   }
-  st = launch_posterior(a->tree->dev, a->B, a->V, a->base_logits, a->candidates, a->mode, a->temperature, a->eps,
-                        a->alpha, a->best_path, a->accept_len, a->accepted_tokens, a->next_token, ws_post, stream,
-                        true);
-  if (st != MEDUSA_OK) return st;
-  return launch_accept_kv(a->tree->dev, a->layers, a->B, a->H, a->hd, a->dtype, a->k_cache, a->v_cache, a->Lcap,
-                          a->seq_lens, a->best_path, a->accept_len, stream, true);
+  // S6 and S7 in one launch: node statistics, the path walk (which advances
+  // seq_lens), then the compaction of the accepted rows.
+  return launch_posterior_accept(a->tree->dev, a->B, a->V, a->base_logits, a->candidates, a->mode, a->temperature,
+                                 a->eps, a->alpha, a->top_p, a->uniforms, a->best_path, a->accept_len,
+                                 a->accepted_tokens, a->next_token, a->layers, a->H, a->hd, a->dtype, a->k_cache,
+                                 a->v_cache, a->Lcap, a->seq_lens, ws_post, stream, true);
 }

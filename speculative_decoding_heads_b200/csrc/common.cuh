@@ -17,6 +17,7 @@ enum DeviceDetail : int {
   kDetailAttnStageWait = 4,   // attention: a tile copy never completed
   kDetailAcceptSeqLen = 5,    // accept_kv: seq_lens[b] + T > Lcap or bad accept_len
   kDetailPosteriorArgs = 6,   // posterior: a candidate token outside [0, V)
+  kDetailPosteriorWait = 7,   // step: the compaction waited for a sequence's walk in vain
 };
 
 // Address of the current device's status word ([0] status, [1] detail).

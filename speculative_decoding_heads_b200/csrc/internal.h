@@ -20,6 +20,7 @@ struct TreeDev {
   const int32_t* depth;           // [T]
   const int32_t* retrieve;        // [P * (D+1)]
   const uint64_t* anc;            // [T * W]
+  const int32_t* path_of;         // [T] lowest path index through each node
 };
 
 }  // namespace medusa
@@ -28,7 +29,7 @@ struct medusa_tree {
   int T = 0, P = 0, D = 0, K = 0, topk = 0, W = 0;
   int device = -1;                // device holding the uploaded tables, -1 if none
   std::vector<std::vector<int32_t>> nodes;   // rank tuple of every node, nodes[0] empty
-  std::vector<int32_t> tree_indices, parent, depth, retrieve;
+  std::vector<int32_t> tree_indices, parent, depth, retrieve, path_of;
   std::vector<uint64_t> anc;
   void* dev_block = nullptr;      // one device allocation holding every table
   medusa::TreeDev dev{};
@@ -86,9 +87,18 @@ medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int
 size_t posterior_workspace_bytes(const TreeDev& t, int B);
 medusa_status_t launch_posterior(const TreeDev& t, int B, int V, const float* logits,
                                  const int32_t* candidates, medusa_mode_t mode, float temperature,
-                                 float eps, float alpha, int32_t* best_path, int32_t* accept_len,
-                                 int32_t* accepted_tokens, int32_t* next_token, void* ws,
+                                 float eps, float alpha, float top_p, const float* uniforms, int32_t* best_path,
+                                 int32_t* accept_len, int32_t* accepted_tokens, int32_t* next_token, void* ws,
                                  cudaStream_t stream, bool pdl = false);
+// S6 and S7 in one launch (medusa_step): the posterior's node CTAs, then
+// compaction CTAs that wait for every sequence's walk; the walk advances seq_lens.
+medusa_status_t launch_posterior_accept(const TreeDev& t, int B, int V, const float* logits,
+                                        const int32_t* candidates, medusa_mode_t mode, float temperature, float eps,
+                                        float alpha, float top_p, const float* uniforms, int32_t* best_path,
+                                        int32_t* accept_len, int32_t* accepted_tokens, int32_t* next_token,
+                                        int layers, int H, int hd, medusa_dtype_t dtype, void* k_cache,
+                                        void* v_cache, int Lcap, int32_t* seq_lens, void* ws, cudaStream_t stream,
+                                        bool pdl);
 
 medusa_status_t launch_accept_kv(const TreeDev& t, int layers, int B, int H, int hd,
                                  medusa_dtype_t dtype, void* k_cache, void* v_cache, int Lcap,

@@ -144,6 +144,13 @@ extern "C" medusa_status_t medusa_tree_create(const int32_t* ranks, const int32_
       n = t->parent[n];
     }
   }
+  // Lowest path through each node (the posterior reads a node's token from it).
+  t->path_of.assign(T, -1);
+  for (int p = t->P - 1; p >= 0; --p)
+    for (int j = 0; j <= D; ++j) {
+      const int n = t->retrieve[static_cast<size_t>(p) * (D + 1) + j];
+      if (n >= 0) t->path_of[n] = p;
+    }
   t->nodes = std::move(nodes);
 
   if (upload) {
@@ -153,7 +160,7 @@ extern "C" medusa_status_t medusa_tree_create(const int32_t* ranks, const int32_
       delete t;
       return medusa::cuda_fail("tree_create: cudaGetDevice", e);
     }
-    const size_t n32 = static_cast<size_t>(3 * T) + t->retrieve.size();
+    const size_t n32 = static_cast<size_t>(4 * T) + t->retrieve.size();
     const size_t off_anc = medusa::align_up(n32 * sizeof(int32_t), 256);
     const size_t bytes = off_anc + t->anc.size() * sizeof(uint64_t);
     std::vector<unsigned char> host(bytes, 0);
@@ -162,6 +169,7 @@ extern "C" medusa_status_t medusa_tree_create(const int32_t* ranks, const int32_
     std::memcpy(h32 + T, t->parent.data(), T * sizeof(int32_t));
     std::memcpy(h32 + 2 * T, t->depth.data(), T * sizeof(int32_t));
     std::memcpy(h32 + 3 * T, t->retrieve.data(), t->retrieve.size() * sizeof(int32_t));
+    std::memcpy(h32 + 3 * T + t->retrieve.size(), t->path_of.data(), T * sizeof(int32_t));
     std::memcpy(host.data() + off_anc, t->anc.data(), t->anc.size() * sizeof(uint64_t));
     e = cudaMalloc(&t->dev_block, bytes);
     if (e == cudaSuccess) e = cudaMemcpy(t->dev_block, host.data(), bytes, cudaMemcpyHostToDevice);
@@ -174,7 +182,8 @@ extern "C" medusa_status_t medusa_tree_create(const int32_t* ranks, const int32_
     const int32_t* d32 = static_cast<const int32_t*>(t->dev_block);
     t->dev = medusa::TreeDev{T, t->P, t->D, K, topk, t->W, d32, d32 + T, d32 + 2 * T, d32 + 3 * T,
                              reinterpret_cast<const uint64_t*>(
-                                 static_cast<const unsigned char*>(t->dev_block) + off_anc)};
+                                 static_cast<const unsigned char*>(t->dev_block) + off_anc),
+                             d32 + 3 * T + t->retrieve.size()};
   }
   *out = t;
   return MEDUSA_OK;

@@ -64,6 +64,7 @@ TID_BASE_LOGITS = 8
 TID_ROOT = 9
 TID_PLANT = 10
 TID_SEQLEN = 11
+TID_UNIFORM = 12          # one draw per sequence for the sampled next token
 SUBSEED_STRIDE = 64
 
 _CHUNK = 1 << 22

@@ -119,3 +119,8 @@ def base_logits(w: Workload, tree_tokens: np.ndarray, parent: np.ndarray,
     z = base_logits_raw(w, sub_logits)
     return gen.plant_agreement(z, tree_tokens, parent, w.agreement,
                                w.seed + 7919 * sub_logits)
+
+
+def uniforms(w: Workload, sub: int = 0) -> np.ndarray:
+    """One U[0, 1) draw per sequence (exact multiples of 2^-24, so fp32 holds them exactly)."""
+    return gen.uniform_01(w.seed, _tid(gen.TID_UNIFORM, sub), w.B)

@@ -70,6 +70,42 @@ def pick_logits(w, tr, toks, cand, max_tries=16):
     raise RuntimeError("no usable logits sub-seed")
 
 
+def pick_uniforms(w, tr, logits, cand, mode, top_p, max_tries=32):
+    """First uniforms sub-seed whose draws sit clear inside their token's CDF interval at the
+    node where each sequence's walk ends; None when that node's nucleus boundary itself is not
+    clear (other logits are needed then)."""
+    base = O.evaluate_posterior(tr, logits, cand, mode, w.temperature, w.eps, w.alpha, top_p)
+    wts = []
+    for b in range(w.B):
+        last = tr["retrieve"][base["best_path"][b], base["accept_len"][b]]
+        pr = O.node_statistics(logits[b, last:last + 1], w.temperature, w.eps, w.alpha)["prob"][0]
+        if mode == "nucleus":
+            if not O.nucleus_cut_ok(pr, top_p):
+                return None
+            pr = np.where(O.nucleus_mask(pr, top_p), pr, 0.0)
+        wts.append(pr)
+    for s in range(max_tries):
+        u = I.uniforms(w, s)
+        if all(O.sample_margin_ok(wts[b], float(u[b])) for b in range(w.B)):
+            return s, u
+    raise RuntimeError("no usable uniforms sub-seed")
+
+
+def pick_nucleus_inputs(w, tr, toks, cand, top_p, sampled, max_tries=16):
+    """Base logits (and uniforms when sampled) whose nucleus decisions all sit clear of their
+    boundaries: every tree edge's membership and, when sampled, the final node's cut-off and draw."""
+    for s in range(max_tries):
+        z = I.base_logits(w, toks, tr["parent"], s)
+        if not O.nucleus_margin_ok(tr, z, cand, w.temperature, top_p):
+            continue
+        if not sampled:
+            return s, z, None
+        got = pick_uniforms(w, tr, z, cand, "nucleus", top_p)
+        if got is not None:
+            return s, z, got[1]
+    raise RuntimeError("no usable logits sub-seed for nucleus acceptance")
+
+
 def check_logits(got, ref, rtol=LOGIT_RTOL):
     got = np.asarray(got, dtype=np.float64)
     scale = np.abs(ref).max()

@@ -13,7 +13,10 @@ import torch
 
 import oracle.medusa_oracle as O
 from synth import gen, inputs as I
-from helpers import (ATTN_ATOL, SMALL, check_logits, oracle_tree, pick_logits, pick_sub_h)
+from helpers import (ATTN_ATOL, SMALL, check_logits, oracle_tree, pick_logits, pick_nucleus_inputs, pick_sub_h,
+                     pick_uniforms)
+
+TOP_P = 0.8   # the pages' default
 
 pytestmark = pytest.mark.gpu
 
@@ -201,7 +204,10 @@ def test_tree_attention_edges(mb, dev, variant):
         _attention_case(mb, dev, w)
 
 
-def _posterior_case(mb, w, mode, agreement=None):
+MODES = {"greedy": 0, "typical": 1, "nucleus": 2}
+
+
+def _posterior_case(mb, w, mode, agreement=None, sampled=False):
     from synth.workloads import shrink
     if agreement is not None:
         w = shrink(w, agreement=agreement)
@@ -209,18 +215,22 @@ def _posterior_case(mb, w, mode, agreement=None):
     sub_h, u, z = pick_sub_h(w)
     ids, _ = O.topk_desc(z, w.topk)
     toks, cand, _ = O.build_tree(tr, I.root_tokens(w), ids, w.prefix_lens())
-    _, logits = pick_logits(w, tr, toks, cand)
-    ref = O.evaluate_posterior(tr, logits, cand, mode, w.temperature, w.eps, w.alpha)
+    if mode == "nucleus":
+        _, logits, uni = pick_nucleus_inputs(w, tr, toks, cand, TOP_P, sampled)
+    else:
+        _, logits = pick_logits(w, tr, toks, cand)
+        uni = pick_uniforms(w, tr, logits, cand, mode, TOP_P)[1] if sampled else None
+    ref = O.evaluate_posterior(tr, logits, cand, mode, w.temperature, w.eps, w.alpha, TOP_P, uni)
     tree = _tree(mb, w)
     c = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
     B, D1 = w.B, tree.D + 1
     out = {k: torch.full(s, -9, dtype=torch.int32, device="cuda") for k, s in
            [("best", (B,)), ("alen", (B,)), ("acc", (B, D1)), ("next", (B,))]}
     ws = mb.workspace(mb.medusa_posterior_workspace_size(tree, B))
-    mb.medusa_evaluate_posterior(tree, torch.from_numpy(logits).cuda(), c(cand),
-                                 mb.MEDUSA_TYPICAL if mode == "typical" else mb.MEDUSA_GREEDY,
+    mb.medusa_evaluate_posterior(tree, torch.from_numpy(logits).cuda(), c(cand), MODES[mode],
                                  out["best"], out["alen"], out["acc"], out["next"], ws,
-                                 temperature=w.temperature, eps=w.eps, alpha=w.alpha)
+                                 temperature=w.temperature, eps=w.eps, alpha=w.alpha, top_p=TOP_P,
+                                 uniforms=None if uni is None else torch.from_numpy(uni.astype(np.float32)).cuda())
     torch.cuda.synchronize()
     assert np.array_equal(_np(out["best"]), ref["best_path"])
     assert np.array_equal(_np(out["alen"]), ref["accept_len"])
@@ -240,14 +250,30 @@ def test_posterior(mb, name, mode):
     _posterior_case(mb, w, mode)
 
 
+@pytest.mark.parametrize("name", sorted(SMALL))
+@pytest.mark.parametrize("mode,sampled", [("nucleus", False), ("nucleus", True), ("typical", True)])
+def test_posterior_nucleus_and_sampled(mb, name, mode, sampled):
+    """Nucleus acceptance (top_p 0.8) and the next token drawn with a caller uniform."""
+    _posterior_case(mb, SMALL[name], mode, sampled=sampled)
+
+
 @pytest.mark.parametrize("V", [40001, 65540])
-@pytest.mark.parametrize("mode", ["greedy", "typical"])
-def test_posterior_vocab_shapes(mb, V, mode):
+@pytest.mark.parametrize("mode,sampled", [("greedy", False), ("typical", False), ("nucleus", True),
+                                          ("typical", True)])
+def test_posterior_vocab_shapes(mb, V, mode, sampled):
     # V = 40001: rows not 16-byte aligned (one logit per load), more than one
     # 32768-logit chunk per row; V = 65540: 16-byte loads over three chunks.
     from synth.workloads import shrink
     w = shrink(SMALL["b3_small"], name=f"b3_V{V}", V=V, modes=(mode,))
-    _posterior_case(mb, w, mode)
+    _posterior_case(mb, w, mode, sampled=sampled)
+
+
+@pytest.mark.parametrize("mode,sampled", [("nucleus", False), ("nucleus", True), ("typical", True)])
+def test_posterior_vicuna7b_shape(mb, mode, sampled):
+    """The posterior alone at the Vicuna-7B step's shape (64 tree tokens, V 32000)."""
+    from synth.workloads import WORKLOADS, shrink
+    w = shrink(WORKLOADS["vicuna7b_bs1_L1024"], name="v7b_post", d=256, layers=1, H=1, prefix=16)
+    _posterior_case(mb, w, mode, sampled=sampled)
 
 
 @pytest.mark.parametrize("agreement,expect", [(0.0, "none"), (1.0, "leaf")])
@@ -305,18 +331,26 @@ def test_accept_kv_overlap_worked_example(mb, dev):
     assert np.array_equal(_np(t["k_cache"].view(torch.int16)).view(np.uint16), k2)
 
 
-@pytest.mark.parametrize("name", sorted(SMALL))
-def test_step(mb, dev, name):
-    """medusa_step end to end against the oracle's S1..S7."""
+STEP_CASES = [(n, SMALL[n].modes[-1], False) for n in sorted(SMALL)] + [
+    ("v7b_small", "nucleus", True), ("v13b_small", "nucleus", False), ("b3_small", "typical", True)]
+
+
+@pytest.mark.parametrize("name,mode,sampled", STEP_CASES, ids=[f"{n}-{m}{'-sampled' if s else ''}"
+                                                               for n, m, s in STEP_CASES])
+def test_step(mb, dev, name, mode, sampled):
+    """medusa_step end to end against the oracle's S1..S7 (S6 and S7 share one launch)."""
     w = SMALL[name]
-    mode = w.modes[-1]
     tr = oracle_tree(w)
     sub_h, u, z = pick_sub_h(w)
     ids, _ = O.topk_desc(z, w.topk)
     lens = w.prefix_lens()
     toks, cand, pos = O.build_tree(tr, I.root_tokens(w), ids, lens)
-    sub_l, logits = pick_logits(w, tr, toks, cand)
-    post = O.evaluate_posterior(tr, logits, cand, mode, w.temperature, w.eps, w.alpha)
+    if mode == "nucleus":
+        sub_l, logits, uni = pick_nucleus_inputs(w, tr, toks, cand, TOP_P, sampled)
+    else:
+        sub_l, logits = pick_logits(w, tr, toks, cand)
+        uni = pick_uniforms(w, tr, logits, cand, mode, TOP_P)[1] if sampled else None
+    post = O.evaluate_posterior(tr, logits, cand, mode, w.temperature, w.eps, w.alpha, TOP_P, uni)
     q = I.values(I.queries(w))
     kc_raw, vc_raw = I.kv_cache(w, "k"), I.kv_cache(w, "v")
     scale = O.attention_scale(w.hd)
@@ -327,8 +361,9 @@ def test_step(mb, dev, name):
     t = dev.materialise(w, sub_h=sub_h, sub_logits=sub_l)
     t["base_logits"].copy_(torch.from_numpy(logits))
     dev.tree_outputs(t, w.B, tree.T, tree.P, tree.D)
-    args = mb.make_step_args(tree, t, mb.MEDUSA_TYPICAL if mode == "typical" else mb.MEDUSA_GREEDY,
-                             w.temperature, w.eps, w.alpha)
+    if uni is not None:
+        t["uniforms"] = torch.from_numpy(uni.astype(np.float32)).cuda()
+    args = mb.make_step_args(tree, t, MODES[mode], w.temperature, w.eps, w.alpha, top_p=TOP_P)
     ws = mb.workspace(mb.medusa_step_workspace_size(args))
     mb.medusa_step(args, ws)
     torch.cuda.synchronize()

@@ -523,18 +523,29 @@ def test_nucleus_and_sampling_special_cases():
 
 
 def check_sampling_guards(O):
-    # nucleus boundary: probabilities [0.5, 0.3, 0.2]; at top_p 0.8 the boundary mass is exactly top_p
-    z = np.log(np.array([[[0.5, 0.3, 0.2]]]))
-    assert not O.nucleus_margin_ok(z, 1.0, 0.8)
-    assert O.nucleus_margin_ok(z, 1.0, 0.7)                    # 0.5 < 0.7 - 1e-4 and 0.8 > 0.7 + 1e-4
-    assert not O.nucleus_margin_ok(z, 1.0, 0.5 + 5e-5)         # the mass before the last member is too close
+    rel = O.NUCLEUS_REL
+    # nucleus boundary of one distribution [0.5, 0.3, 0.2]
+    assert not O.nucleus_cut_ok([0.5, 0.3, 0.2], 0.8)                 # the mass through the last member is top_p
+    assert O.nucleus_cut_ok([0.5, 0.3, 0.2], 0.7)
+    assert not O.nucleus_cut_ok([0.5, 0.3, 0.2], 0.5 + rel / 2)       # the mass before the last member is too close
+    assert O.nucleus_cut_ok([0.5, 0.3, 0.2], 0.5 + 2 * rel)
     # the last member and the first token left out tie: which one is in depends on rounding
-    assert not O.nucleus_margin_ok(np.log(np.array([[[0.4, 0.3, 0.3]]])), 1.0, 0.6)
-    assert O.nucleus_margin_ok(np.log(np.array([[[0.4, 0.4, 0.2]]])), 1.0, 0.6)    # a tie inside the nucleus is harmless
+    assert not O.nucleus_cut_ok([0.4, 0.3, 0.3], 0.6)
+    assert O.nucleus_cut_ok([0.4, 0.4, 0.2], 0.6)                     # a tie inside the nucleus is harmless
+    # tree edges: one-edge tree whose child token (id 0) has mass 0.5 ranking before it
+    tr = O.tree_tables([(0,)], 1, 1)
+    _, cand, _ = O.build_tree(tr, np.array([3]), np.array([[[0]]]), np.array([0]))
+    z = np.zeros((1, 2, 3))
+    z[0, 0] = np.log([0.3, 0.5, 0.2])
+    assert O.nucleus_margin_ok(tr, z, cand, 1.0, 0.5 + 2 * rel)
+    assert not O.nucleus_margin_ok(tr, z, cand, 1.0, 0.5 + rel / 2)
+    assert not O.nucleus_margin_ok(tr, z, cand, 1.0, 0.5 - rel / 2)
+    z[0, 1] = np.log([0.5, 0.3, 0.2])                                  # the leaf's row is no parent
+    assert O.nucleus_margin_ok(tr, z, cand, 1.0, 0.5 + 2 * rel)
     # the draw's interval: weights [1, 3], u * 4 = 1 exactly is a boundary
     assert not O.sample_margin_ok([1.0, 3.0], 0.25)
-    assert not O.sample_margin_ok([1.0, 3.0], 0.25 - 1e-5)
-    assert O.sample_margin_ok([1.0, 3.0], 0.25 + 1e-3) and O.sample_margin_ok([1.0, 3.0], 0.1)
+    assert not O.sample_margin_ok([1.0, 3.0], 0.25 - rel / 8)
+    assert O.sample_margin_ok([1.0, 3.0], 0.25 + rel) and O.sample_margin_ok([1.0, 3.0], 0.1)
 
 
 def test_sampling_guards():
