@@ -36,7 +36,7 @@
 #include <cfloat>
 #include <cstdint>
 
-#include "common.cuh"
+#include "heads_common.cuh"
 
 namespace medusa {
 namespace {
@@ -277,32 +277,6 @@ struct WarpFold {
     }
   }
 };
-
-// Warp 0: insert (v, id) into the sorted list (lv, lid, *cnt) of capacity topk.
-__device__ __forceinline__ void list_insert(float* lv, int* lid, int* cnt_p, int topk, float v, int id,
-                                            int lane) {
-  const int cnt = *cnt_p;
-  float ev = -FLT_MAX;
-  int ei = -1;
-  if (lane < cnt) {
-    ev = lv[lane];
-    ei = lid[lane];
-  }
-  const bool before = lane < cnt && ranks_before(ev, ei, v, id);
-  const int pos = __popc(__ballot_sync(0xffffffffu, before));
-  const float pv = __shfl_up_sync(0xffffffffu, ev, 1);
-  const int pi = __shfl_up_sync(0xffffffffu, ei, 1);
-  __syncwarp();
-  if (pos < topk && lane < topk && lane >= pos && lane <= cnt) {
-    lv[lane] = (lane == pos) ? v : pv;
-    lid[lane] = (lane == pos) ? id : pi;
-  }
-  __syncwarp();
-  if (lane == 0 && pos < topk && cnt < topk) *cnt_p = cnt + 1;
-  __syncwarp();
-}
-
-constexpr int kMergeRegs = 16;   // candidates per lane held in registers by the merge
 
 // Shared-memory carve-up of one CTA (offsets in bytes; stages first, 128-byte aligned).
 struct Layout {
@@ -622,9 +596,7 @@ __global__ void __launch_bounds__(heads_threads<NB, VPT, R>(), 1) heads_kernel(c
   __syncthreads();
   if (flag[0] != 2) return;
 
-  // Last CTA: merge the published lists of every (sequence, head).  The
-  // candidates of one list are loaded once; each of the topk rounds picks
-  // the best candidate that ranks strictly after the previous pick.
+  // Last CTA: merge the published lists of every (sequence, head).
   __threadfence();
   const int NW = blockDim.x >> 5;
   for (int li = warp; li < a.nb * a.K; li += NW) {
@@ -632,56 +604,10 @@ __global__ void __launch_bounds__(heads_threads<NB, VPT, R>(), 1) heads_kernel(c
     const int hk_lo = k * a.V;
     const int c_lo = part_of(hk_lo, n2, G);
     const int c_hi = part_of(hk_lo + a.V - 1, n2, G);
-    const int ncand = (c_hi - c_lo + 1) * a.topk;
     const size_t base = ((static_cast<size_t>(b) * a.K + k) * G + c_lo) * a.topk;
-    float cv[kMergeRegs];
-    int ci[kMergeRegs];
-#pragma unroll
-    for (int m = 0; m < kMergeRegs; ++m) {
-      const int i = lane + 32 * m;
-      cv[m] = -FLT_MAX;
-      ci[m] = -1;
-      if (i < ncand) {
-        cv[m] = __ldcg(a.cand_vals + base + i);
-        ci[m] = __ldcg(a.cand_ids + base + i);
-      }
-    }
-    float prev_v = FLT_MAX;
-    int prev_i = -1;
-    for (int r = 0; r < a.topk; ++r) {
-      float bv = -FLT_MAX;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int m = 0; m < kMergeRegs; ++m)
-        if (ci[m] >= 0 && ranks_before(prev_v, prev_i, cv[m], ci[m]) && ranks_before(cv[m], ci[m], bv, bi)) {
-          bv = cv[m];
-          bi = ci[m];
-        }
-      for (int i = lane + 32 * kMergeRegs; i < ncand; i += 32) {   // large lists only
-        const float v = __ldcg(a.cand_vals + base + i);
-        const int id = __ldcg(a.cand_ids + base + i);
-        if (id >= 0 && ranks_before(prev_v, prev_i, v, id) && ranks_before(v, id, bv, bi)) {
-          bv = v;
-          bi = id;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ranks_before(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if (lane == 0) {
-        const size_t o = (static_cast<size_t>(a.b0 + b) * a.K + k) * a.topk + r;
-        a.topk_ids[o] = bi;
-        a.topk_vals[o] = bv;
-      }
-      prev_v = bv;
-      prev_i = bi;
-    }
+    const size_t o = (static_cast<size_t>(a.b0 + b) * a.K + k) * a.topk;
+    merge_candidates(a.cand_vals + base, a.cand_ids + base, (c_hi - c_lo + 1) * a.topk, a.topk, a.topk_ids + o,
+                     a.topk_vals + o, lane);
   }
   __syncthreads();
   if (tid == 0) {
@@ -691,27 +617,9 @@ __global__ void __launch_bounds__(heads_threads<NB, VPT, R>(), 1) heads_kernel(c
   }
   if (a.do_build) {
     // S4 from the final top-k (this CTA's merge above and the earlier batch
-    // groups' launches): the flat list [root, head 1 top-k, ..., head K
-    // top-k] gathered through tree_indices and retrieve, and the positions.
-    const TreeDev& t = a.build.t;
-    const int per_b = 2 * t.T + t.P * (t.D + 1);
-    for (int g = tid; g < a.B * per_b; g += blockDim.x) {
-      const int b = g / per_b;
-      int o = g - b * per_b;
-      auto flat = [&](int fi) -> int32_t {
-        return fi == 0 ? a.build.root_tokens[b] : a.topk_ids[(static_cast<size_t>(b) * t.K) * t.topk + (fi - 1)];
-      };
-      if (o < t.T) {
-        a.build.tree_tokens[b * t.T + o] = flat(t.tree_indices[o]);
-      } else if (o < 2 * t.T) {
-        o -= t.T;
-        a.build.position_ids[b * t.T + o] = a.build.seq_lens[b] + t.depth[o];
-      } else {
-        o -= 2 * t.T;
-        const int node = t.retrieve[o];
-        a.build.candidates[static_cast<size_t>(b) * t.P * (t.D + 1) + o] = node < 0 ? -1 : flat(t.tree_indices[node]);
-      }
-    }
+    // groups' launches).
+    __syncthreads();
+    build_tree_block(a.build, a.B, a.topk_ids);
   }
 }
 
@@ -783,12 +691,17 @@ cudaError_t dispatch_nb(const HeadsArgs& a, const Plan& p, cudaStream_t stream) 
 }  // namespace
 
 size_t heads_workspace_bytes(int B, int d, int V, int K, int topk) {
-  (void)V;
   const int G = sm_count();
   size_t off = align_up(static_cast<size_t>(B) * K * d * sizeof(float), 256);
   off += align_up(static_cast<size_t>(kMaxNB) * K * G * topk * sizeof(float), 256);
   off += align_up(static_cast<size_t>(kMaxNB) * K * G * topk * sizeof(int32_t), 256);
   off += 256;  // counters
+  // Batches the tensor-core kernel may take (bf16 with d a multiple of 128;
+  // the size does not depend on the dtype, so it is reserved either way).
+  if (heads_tc_supported(B, d, MEDUSA_BF16)) {
+    const size_t tc = heads_tc_workspace_bytes(B, d, V, K, topk);
+    if (tc > off) off = tc;
+  }
   return off;
 }
 
@@ -796,6 +709,9 @@ medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, cons
                              int B, int d, int V, int K, int topk, medusa_dtype_t dtype,
                              float* head_logits, int32_t* topk_ids, float* topk_vals, void* ws,
                              cudaStream_t stream, const TreeBuild* build) {
+  // Two or more sequences: the tensor cores, weights read once per 16 sequences.
+  if (heads_tc_supported(B, d, dtype))
+    return launch_heads_tc(h, W1, b1, Wout, B, d, V, K, topk, head_logits, topk_ids, topk_vals, ws, stream, build);
   const int G = sm_count();
   HeadsArgs a{};
   a.h = h;

@@ -69,6 +69,14 @@ medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, cons
                              float* head_logits, int32_t* topk_ids, float* topk_vals, void* ws,
                              cudaStream_t stream, const TreeBuild* build = nullptr);
 
+// The tensor-core heads (heads_tc.cu) for 2..16 sequences per pass, bf16, d a
+// multiple of 128; launch_heads dispatches to it.
+bool heads_tc_supported(int B, int d, medusa_dtype_t dtype);
+size_t heads_tc_workspace_bytes(int B, int d, int V, int K, int topk);
+medusa_status_t launch_heads_tc(const void* h, const void* W1, const void* b1, const void* Wout, int B, int d, int V,
+                                int K, int topk, float* head_logits, int32_t* topk_ids, float* topk_vals, void* ws,
+                                cudaStream_t stream, const TreeBuild* build);
+
 medusa_status_t launch_build_tree(const TreeDev& t, int B, const int32_t* root_tokens,
                                   const int32_t* topk_ids, const int32_t* seq_lens,
                                   int32_t* tree_tokens, int32_t* candidates,
