@@ -41,6 +41,9 @@ def parse():
     p.add_argument("--no-graph", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--shrink", default=None,
+                   help="a smaller variant of the workload for profiling one kernel on a small case, "
+                        "e.g. layers=1 (comma-separated field=value; the line's config names the variant)")
     return p.parse_args()
 
 
@@ -493,6 +496,9 @@ def main():
     a = parse()
     from synth import workloads as W
     w = W.get(a.workload or W.BENCH_WORKLOAD)
+    if a.shrink:
+        kv = dict(x.split("=") for x in a.shrink.split(","))
+        w = W.shrink(w, name=f"{w.name}[{a.shrink}]", **{k: int(v) for k, v in kv.items()})
     if a.impl == "reference":
         return run_reference(a, w)
     return run_ours(a, w)

@@ -11,20 +11,24 @@
 //
 // Two persistent launches, one CTA per SM:
 //  * phase 1 multiplies W1 (K heads of d x d) by h.  h is bf16, so its B
-//    operand is exact (N = B, padded to 16 columns).  The K*d/128 row tiles
-//    of 128 rows are cut along d into S parts so that every CTA gets about
-//    eight equal units; each part's fp32 accumulator goes to the workspace
-//    and, for each quarter of a tile's rows, the last part to finish (a
-//    counter per tile quarter) sums the parts in part order, applies the
+//    operand is exact (N = B, padded to 16 columns); the epilogue applies the
 //    residual block and writes u as a bf16 pair (high part, and the remainder
 //    rounded to bf16: about 16 significant bits of the fp32 u) for phase 2.
 //  * phase 2 multiplies Wout (K heads of V x d) by those pairs (N = 2B: the
 //    products of the high parts and of the remainders accumulate in separate
-//    fp32 columns and are added in the epilogue).  Each CTA takes a contiguous
-//    range of 128-row tiles; each epilogue warp keeps a running top-k per
-//    sequence; when the head changes the four warps' lists are merged into
-//    the CTA's list for that head; the last CTA to finish merges the CTAs'
-//    lists and (inside medusa_step) builds the tree.
+//    fp32 columns and are added in the epilogue); each epilogue warp keeps a
+//    running top-k per sequence; when the head changes the four warps' lists
+//    are merged into the CTA's list for that head; the last CTA to finish
+//    merges the CTAs' lists and (inside medusa_step) builds the tree.
+//  Work split: a phase is a sequence of tiles (128 rows of one head) of
+//  d/64/kKPS ring stages each.  In phase 1 every CTA takes an equal
+//  contiguous range of stages, so the HBM stream is balanced to one stage; a
+//  tile cut by a range boundary is shared by two or three CTAs: each stores
+//  its fp32 partial accumulator, and for each quarter of the tile's rows the
+//  last CTA to finish (a counter per tile quarter) sums the partials in CTA
+//  order and runs the epilogue.  Phase 2 splits at whole tiles (balanced to
+//  one tile), so each logit is a single accumulation whose order does not
+//  depend on V or on the split.
 //    Phase 2 is launched with programmatic dependent launch: its producer
 //    streams the first weight tiles before it waits for phase 1's pairs.
 //
@@ -45,12 +49,14 @@ namespace medusa {
 namespace {
 
 constexpr int kTileRows = 128;               // weight rows per tile (MMA M)
-constexpr int kKStep = 64;                   // weight columns per stage (one 128-byte swizzle row)
-constexpr int kWBytes = kTileRows * 128;     // 16 KB of weights per stage
+constexpr int kKStep = 64;                   // weight columns per block (one 128-byte swizzle row)
+constexpr int kKPS = 4;                       // blocks per ring stage (one TMA box per operand)
+constexpr int kWBlock = kTileRows * 128;     // 16 KB of weights per block
+constexpr int kWBytes = kKPS * kWBlock;      // weights per stage
 constexpr int kThreads = 256;                // warps 0 producer, 1 MMA, 2-3 idle, 4-7 epilogue
 constexpr int kMaxB = 16;                    // sequences per pass (N = 2B <= 32)
 constexpr int kMaxStages = 12;
-constexpr int kRingBytes = 200 * 1024;
+constexpr int kSmemMax = 232448;             // dynamic shared memory per CTA
 constexpr int kEpiWarps = 4;
 constexpr uint32_t kTmemCols = 64;           // two accumulators of up to 32 columns
 
@@ -59,16 +65,17 @@ struct HTArgs {
   int d, V, K, topk;
   int rows;               // rows per head of this phase's matrix (d or V)
   int tph;                // tiles per head: ceil(rows / 128)
-  int S;                  // parts per tile (phase 1; 1 in phase 2)
-  int units;              // K * tph * S
-  int ksteps;             // d / 64
+  int nst;                // ring stages per tile: d / 64 / kKPS
+  int W;                  // stages of the phase: K * tph * nst
+  int gran;               // stages per unit of the split (1, or nst: whole tiles)
+  int ksteps;             // d / 64 (a multiple of kKPS)
   int G;                  // CTAs
   int NS;                 // ring stages
   const uint16_t* h;      // [Btot, d]
   const uint16_t* b1;     // [K, d]
   uint16_t* X2;           // [K, 2B, d]: row 2b the high parts of u[b], row 2b+1 the remainders
-  float* part;            // [units, 128, B] phase-1 partial sums
-  unsigned* tile_cnt;     // [K * tph * 4] parts finished per tile quarter (self-resetting)
+  float* part;            // [G, 2, 128, N] partial accumulators of the first / last tile of each CTA
+  unsigned* tile_cnt;     // [K * tph * 4] partials finished per tile quarter (self-resetting)
   float* head_logits;     // nullable [Btot, K, V]
   int32_t* topk_ids;      // [Btot, K, topk]
   float* topk_vals;
@@ -91,33 +98,39 @@ struct Bars {
 
 // Dynamic shared memory: the ring (per stage 16 KB of weights, then the
 // activation box), the barrier block, then the epilogue's top-k lists.
-__host__ __device__ inline int x_bytes(int npad) { return npad * 128; }
+__host__ __device__ inline int x_bytes(int npad) { return kKPS * npad * 128; }
 __host__ __device__ inline int stage_bytes(int npad) { return kWBytes + x_bytes(npad); }
 __host__ __device__ inline int lists_bytes(int B, int topk) { return kEpiWarps * B * (2 * topk + 1) * 4; }
 __host__ __device__ inline int smem_bytes(int NS, int npad, int B, int topk) {
   return 1024 + NS * stage_bytes(npad) + 1024 + lists_bytes(B, topk);
 }
 
-__device__ __forceinline__ int unit_lo(int c, int units, int G) {
-  return static_cast<int>(static_cast<long long>(units) * c / G);
+// First stage of CTA c's range, and the CTA whose range holds stage st
+// (ranges are equal shares of the W / gran units of gran stages each).
+__device__ __forceinline__ int stage_lo(int c, const HTArgs& a) {
+  return a.gran * static_cast<int>(static_cast<long long>(a.W / a.gran) * c / a.G);
 }
-__device__ __forceinline__ int unit_owner(int u, int units, int G) {
-  return static_cast<int>((static_cast<long long>(u + 1) * G - 1) / units);
+__device__ __forceinline__ int stage_owner(int st, const HTArgs& a) {
+  return static_cast<int>((static_cast<long long>(st / a.gran + 1) * a.G - 1) / (a.W / a.gran));
 }
 
 struct Unit {
-  int tile, s, head, row0, k0, k1;   // k-steps [k0, k1)
+  int tile, head, row0, k0, k1;   // column blocks [k0, k1) of one tile, whole stages
 };
 
-__device__ __forceinline__ Unit unit_info(const HTArgs& a, int u) {
-  Unit x;
-  x.tile = u / a.S;
-  x.s = u - x.tile * a.S;
+// The next unit of a CTA's stage range: the stages from `st` to the end of
+// the range or of the tile, whichever comes first.
+__device__ __forceinline__ bool next_unit(const HTArgs& a, int& st, int st_hi, Unit& x) {
+  if (st >= st_hi) return false;
+  x.tile = st / a.nst;
+  const int t0 = x.tile * a.nst;
+  const int e = st_hi < t0 + a.nst ? st_hi : t0 + a.nst;
   x.head = x.tile / a.tph;
   x.row0 = (x.tile - x.head * a.tph) * kTileRows;
-  x.k0 = static_cast<int>(static_cast<long long>(a.ksteps) * x.s / a.S);
-  x.k1 = static_cast<int>(static_cast<long long>(a.ksteps) * (x.s + 1) / a.S);
-  return x;
+  x.k0 = (st - t0) * kKPS;
+  x.k1 = (e - t0) * kKPS;
+  st = e;
+  return true;
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Bars* bs, int* status) {
@@ -140,12 +153,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int NS = a.NS;
-  constexpr int kSB = kWBytes + kNpad * 128;
+  constexpr int kSB = kWBytes + kKPS * kNpad * 128;
   Bars* bs = reinterpret_cast<Bars*>(smem + NS * kSB);
   float* lv_all = reinterpret_cast<float*>(smem + NS * kSB + 1024);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x;
-  const int u_lo = unit_lo(cta, a.units, a.G), u_hi = unit_lo(cta + 1, a.units, a.G);
+  const int st_lo = stage_lo(cta, a), st_hi = stage_lo(cta + 1, a);
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -184,23 +197,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto flush = [&]() {
         wait_prior_grids();
         for (int i = 0; i < npend; ++i)
-          tc::tma_load_3d(smem + pend_slot[i] * kSB + kWBytes, &x_map, pend_k[i] * kKStep, 0, pend_head[i],
+          tc::tma_load_4d(smem + pend_slot[i] * kSB + kWBytes, &x_map, 0, 0, pend_k[i], pend_head[i],
                           &bs->full[pend_slot[i]]);
         npend = 0;
         x_ready = true;
       };
       int g = 0;
-      for (int u = u_lo; u < u_hi && !bs->abort; ++u) {
-        const Unit x = unit_info(a, u);
-        for (int j = x.k0; j < x.k1; ++j, ++g) {
+      Unit x;
+      for (int st = st_lo; !bs->abort && next_unit(a, st, st_hi, x);) {
+        for (int j = x.k0; j < x.k1; j += kKPS, ++g) {
           const int slot = g % NS;
           if (!x_ready && npend == NS) flush();
           if (g >= NS && !wait_or_abort(&bs->empty[slot], ((g / NS) - 1) & 1, bs, a.status)) break;
           mbar_arrive_expect_tx(&bs->full[slot], kSB);
-          tc::tma_load_3d_hint(smem + slot * kSB, &w_map, j * kKStep, x.row0, x.head, &bs->full[slot], pol);
+          tc::tma_load_4d_hint(smem + slot * kSB, &w_map, 0, x.row0, j, x.head, &bs->full[slot], pol);
           const int xh = kPhase == 1 ? 0 : x.head;
           if (x_ready) {
-            tc::tma_load_3d(smem + slot * kSB + kWBytes, &x_map, j * kKStep, 0, xh, &bs->full[slot]);
+            tc::tma_load_4d(smem + slot * kSB + kWBytes, &x_map, 0, 0, j, xh, &bs->full[slot]);
           } else {
             pend_slot[npend] = slot;
             pend_k[npend] = j;
@@ -220,14 +233,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = tc::idesc_bf16_f32(kTileRows, kNpad, 0);
       const uint32_t sbase = smem_u32(smem);
       int g = 0, n = 0;
-      for (int u = u_lo; u < u_hi && !bs->abort; ++u, ++n) {
-        const Unit x = unit_info(a, u);
+      Unit x;
+      for (int st = st_lo; !bs->abort && next_unit(a, st, st_hi, x); ++n) {
         const int buf = n & 1;
         if (n >= 2 && !wait_or_abort(&bs->acc_empty[buf], ((n >> 1) - 1) & 1, bs, a.status)) break;
         tc::fence_after_sync();
         const uint32_t d = tmem + buf * kNpad;
         bool ok = true;
-        for (int j = x.k0; j < x.k1; ++j, ++g) {
+        for (int j = x.k0; j < x.k1; j += kKPS, ++g) {
           const int slot = g % NS;
           if (!wait_or_abort(&bs->full[slot], (g / NS) & 1, bs, a.status)) {
             ok = false;
@@ -236,11 +249,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::fence_after_sync();
           const uint32_t wa = sbase + slot * kSB, xa = wa + kWBytes;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = tc::smem_desc_sw128(wa + kk * 32, 16, 1024);
-            const uint64_t bd = tc::smem_desc_sw128(xa + kk * 32, 16, 1024);
-            tc::mma_ss(d, ad, bd, idesc, (j > x.k0 || kk > 0) ? 1u : 0u);
-          }
+          for (int c = 0; c < kKPS; ++c)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = tc::smem_desc_sw128(wa + c * kWBlock + kk * 32, 16, 1024);
+              const uint64_t bd = tc::smem_desc_sw128(xa + c * kNpad * 128 + kk * 32, 16, 1024);
+              tc::mma_ss(d, ad, bd, idesc, (j > x.k0 || c > 0 || kk > 0) ? 1u : 0u);
+            }
           tc::mma_commit(&bs->empty[slot]);
         }
         if (!ok) break;
@@ -322,8 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     if (kPhase == 2) reset_lists();
     int n = 0;
-    for (int u = u_lo; u < u_hi; ++u, ++n) {
-      const Unit x = unit_info(a, u);
+    Unit x;
+    for (int st = st_lo; next_unit(a, st, st_hi, x); ++n) {
       if constexpr (kPhase == 2) {
         if (x.head != cur_head) {
           if (cur_head >= 0) flush(cur_head);
@@ -347,38 +362,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&bs->acc_empty[buf]);
 
-      if constexpr (kPhase == 1) {
-        const int i = x.row0 + r;   // output feature of head x.head (d is a multiple of 128)
-        if (a.S > 1) {
-          // Publish this part; for each quarter of the tile's rows the last
-          // part to finish sums all the parts, in part order.
-          float* mine = a.part + (static_cast<size_t>(u) * kTileRows + r) * B;
+      // A tile shared with other CTAs: store this CTA's partial accumulator;
+      // for each quarter of the rows the last CTA to finish sums the partials
+      // in CTA order and runs the epilogue.
+      const int ncol = kPhase == 1 ? B : 2 * B;
+      const int t0 = x.tile * a.nst;
+      const int c_first = stage_owner(t0, a), c_last = stage_owner(t0 + a.nst - 1, a);
+      if (c_first != c_last) {
+        const int slot = x.tile == st_lo / a.nst ? 0 : 1;
+        float* mine = a.part + ((static_cast<size_t>(cta) * 2 + slot) * kTileRows + r) * ncol;
+#pragma unroll
+        for (int b = 0; b < kNpad; ++b)
+          if (b < ncol) mine[b] = acc[b];
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          unsigned* cnt = &a.tile_cnt[x.tile * kEpiWarps + q];
+          last = atom_add_acq_rel_gpu(cnt, 1u) == static_cast<unsigned>(c_last - c_first);
+          if (last) *cnt = 0u;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) continue;
+        __threadfence();
+        float sum[kNpad];
+#pragma unroll
+        for (int b = 0; b < kNpad; ++b) sum[b] = 0.f;
+        for (int c = c_first; c <= c_last; ++c) {
+          const int sl = x.tile == stage_lo(c, a) / a.nst ? 0 : 1;
+          const float* pc = a.part + ((static_cast<size_t>(c) * 2 + sl) * kTileRows + r) * ncol;
 #pragma unroll
           for (int b = 0; b < kNpad; ++b)
-            if (b < B) mine[b] = acc[b];
-          __threadfence();
-          __syncwarp();
-          int last = 0;
-          if (lane == 0) {
-            unsigned* cnt = &a.tile_cnt[x.tile * kEpiWarps + q];
-            last = atom_add_acq_rel_gpu(cnt, 1u) == static_cast<unsigned>(a.S - 1);
-            if (last) *cnt = 0u;
-          }
-          last = __shfl_sync(0xffffffffu, last, 0);
-          if (!last) continue;
-          __threadfence();
-          float sum[kNpad];
-#pragma unroll
-          for (int b = 0; b < kNpad; ++b) sum[b] = 0.f;
-          for (int s = 0; s < a.S; ++s) {
-            const float* ps = a.part + ((static_cast<size_t>(x.tile) * a.S + s) * kTileRows + r) * B;
-#pragma unroll
-            for (int b = 0; b < kNpad; ++b)
-              if (b < B) sum[b] += (s == x.s) ? acc[b] : __ldcg(ps + b);
-          }
-#pragma unroll
-          for (int b = 0; b < kNpad; ++b) acc[b] = sum[b];
+            if (b < ncol) sum[b] += (c == cta) ? acc[b] : __ldcg(pc + b);
         }
+#pragma unroll
+        for (int b = 0; b < kNpad; ++b) acc[b] = sum[b];
+      }
+      if constexpr (kPhase == 1) {
+        const int i = x.row0 + r;   // output feature of head x.head (d is a multiple of 128)
         const float bias = __uint_as_float(static_cast<uint32_t>(a.b1[static_cast<size_t>(x.head) * a.d + i]) << 16);
         uint16_t* x2 = a.X2 + static_cast<size_t>(x.head) * 2 * B * a.d + i;
 #pragma unroll
@@ -439,11 +460,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (!bs->flag) return;
   __threadfence();
-  const int per_head = a.tph * a.S;
+  const int per_head = a.tph * a.nst;
   for (int lidx = warp; lidx < a.B * a.K; lidx += kThreads / 32) {
     const int b = lidx / a.K, k = lidx - b * a.K;
-    const int c_lo = unit_owner(k * per_head, a.units, a.G);
-    const int c_hi = unit_owner((k + 1) * per_head - 1, a.units, a.G);
+    const int c_lo = stage_owner(k * per_head, a);
+    const int c_hi = stage_owner((k + 1) * per_head - 1, a);
     const size_t base = ((static_cast<size_t>(b) * a.K + k) * a.G + c_lo) * a.topk;
     const size_t o = (static_cast<size_t>(a.b0 + b) * a.K + k) * a.topk;
     merge_candidates(a.cand_vals + base, a.cand_ids + base, (c_hi - c_lo + 1) * a.topk, a.topk, a.topk_ids + o,
@@ -459,25 +480,18 @@ struct Layout {
   size_t x2, part, tile_cnt, cand_v, cand_i, done, total;
 };
 
-int parts_per_tile(int K, int d, int G) {
-  const int tiles = K * (d / kTileRows);
-  const int want = (8 * G + tiles - 1) / tiles;
-  const int ks = d / kKStep;
-  return want < 1 ? 1 : (want > ks ? ks : want);
-}
-
-Layout make_layout(int B, int d, int K, int topk, int G) {
+Layout make_layout(int B, int d, int V, int K, int topk, int G) {
   const int nb = B < kMaxB ? B : kMaxB;
-  const int S = parts_per_tile(K, d, G);
-  const size_t units1 = static_cast<size_t>(K) * (d / kTileRows) * S;
+  const size_t tiles1 = static_cast<size_t>(K) * (d / kTileRows);
+  const size_t tiles2 = static_cast<size_t>(K) * ((V + kTileRows - 1) / kTileRows);
   Layout l{};
   size_t o = 0;
   l.x2 = o;
   o += align_up(static_cast<size_t>(K) * 2 * nb * d * 2, 256);
   l.part = o;
-  o += align_up(units1 * kTileRows * nb * 4, 256);
+  o += align_up(static_cast<size_t>(G) * 2 * kTileRows * 2 * nb * 4, 256);
   l.tile_cnt = o;
-  o += align_up(static_cast<size_t>(K) * (d / kTileRows) * kEpiWarps * 4, 256);
+  o += align_up((tiles1 > tiles2 ? tiles1 : tiles2) * kEpiWarps * 4, 256);
   const size_t nc = static_cast<size_t>(nb) * K * G * topk;
   l.cand_v = o;
   o += align_up(nc * 4, 256);
@@ -499,13 +513,17 @@ cudaError_t launch_phase(const CUtensorMap& wm, const CUtensorMap& xm, const HTA
   return launch_kernel(fn, dim3(grid), dim3(kThreads), static_cast<size_t>(smem), stream, pdl, wm, xm, a);
 }
 
-bool encode3(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid,
+// A [outer][mid][inner] bf16 array as a 4-D map {64 columns, mid rows, inner/64
+// blocks, outer} (the block dimension has the 128-byte stride, so one box of
+// {64, box_mid, kKPS, 1} lands as kKPS consecutive canonical 128-byte-swizzled
+// tiles of box_mid rows each).
+bool encode4(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid,
              uint64_t outer, uint32_t box_mid) {
-  const cuuint64_t dims[3] = {inner, mid, outer};
-  const cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kKStep), box_mid, 1};
-  const cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kKStep), mid, inner / kKStep, outer};
+  const cuuint64_t strides[3] = {inner * 2, kKStep * 2, inner * mid * 2};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(kKStep), box_mid, static_cast<cuuint32_t>(kKPS), 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -518,7 +536,7 @@ bool heads_tc_supported(int B, int d, medusa_dtype_t dtype) {
 
 size_t heads_tc_workspace_bytes(int B, int d, int V, int K, int topk) {
   (void)V;
-  return make_layout(B, d, K, topk, sm_count()).total;
+  return make_layout(B, d, V, K, topk, sm_count()).total;
 }
 
 medusa_status_t launch_heads_tc(const void* h, const void* W1, const void* b1, const void* Wout, int B, int d, int V,
@@ -527,7 +545,7 @@ medusa_status_t launch_heads_tc(const void* h, const void* W1, const void* b1, c
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!enc) return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_heads_topk: cuTensorMapEncodeTiled unavailable");
   const int G = sm_count();
-  const Layout l = make_layout(B, d, K, topk, G);
+  const Layout l = make_layout(B, d, V, K, topk, G);
   unsigned char* w = static_cast<unsigned char*>(ws);
   HTArgs a{};
   a.Btot = B;
@@ -559,15 +577,16 @@ medusa_status_t launch_heads_tc(const void* h, const void* W1, const void* b1, c
       HTArgs p = a;
       p.rows = d;
       p.tph = d / kTileRows;
-      p.S = parts_per_tile(K, d, G);
-      p.units = K * p.tph * p.S;
+      p.nst = d / kKStep / kKPS;
+      p.W = K * p.tph * p.nst;
+      p.gran = 1;
       const int npad = 16;   // B <= 16 columns of h
-      p.NS = kRingBytes / stage_bytes(npad);
+      p.NS = (kSmemMax - smem_bytes(0, npad, 0, topk)) / stage_bytes(npad);
       if (p.NS > kMaxStages) p.NS = kMaxStages;
-      p.G = p.units < G ? p.units : G;
+      p.G = p.W < G ? p.W : G;
       CUtensorMap wm, xm;
-      if (!encode3(enc, &wm, W1, d, d, K, kTileRows) ||
-          !encode3(enc, &xm, static_cast<const uint16_t*>(h) + static_cast<size_t>(b0) * d, d, nb, 1, npad))
+      if (!encode4(enc, &wm, W1, d, d, K, kTileRows) ||
+          !encode4(enc, &xm, static_cast<const uint16_t*>(h) + static_cast<size_t>(b0) * d, d, nb, 1, npad))
         return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_heads_topk: phase-1 tensor map rejected");
       const cudaError_t e = launch_phase<1, 16>(wm, xm, p, p.G, stream, false);
       if (e != cudaSuccess) return cuda_fail("medusa_heads_topk: tensor-core phase 1 launch", e);
@@ -577,14 +596,17 @@ medusa_status_t launch_heads_tc(const void* h, const void* W1, const void* b1, c
       HTArgs p = a;
       p.rows = V;
       p.tph = (V + kTileRows - 1) / kTileRows;
-      p.S = 1;
-      p.units = K * p.tph;
+      p.nst = d / kKStep / kKPS;
+      p.W = K * p.tph * p.nst;
+      // Whole tiles: every logit is one accumulation over d in the same order
+      // whatever V is, so vocabulary shards reproduce the unsplit logits.
+      p.gran = p.nst;
       const int npad = 2 * nb <= 16 ? 16 : 32;
-      p.NS = kRingBytes / stage_bytes(npad);
+      p.NS = (kSmemMax - smem_bytes(0, npad, nb, topk)) / stage_bytes(npad);
       if (p.NS > kMaxStages) p.NS = kMaxStages;
-      p.G = p.units < G ? p.units : G;
+      p.G = K * p.tph < G ? K * p.tph : G;
       CUtensorMap wm, xm;
-      if (!encode3(enc, &wm, Wout, d, V, K, kTileRows) || !encode3(enc, &xm, a.X2, d, 2 * nb, K, npad))
+      if (!encode4(enc, &wm, Wout, d, V, K, kTileRows) || !encode4(enc, &xm, a.X2, d, 2 * nb, K, npad))
         return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_heads_topk: phase-2 tensor map rejected");
       const cudaError_t e = npad == 16 ? launch_phase<2, 16>(wm, xm, p, p.G, stream, true)
                                        : launch_phase<2, 32>(wm, xm, p, p.G, stream, true);
