@@ -109,6 +109,21 @@ int medusa_abi_version(void);
  * device.  *detail receives a kernel-specific code (may be NULL). */
 medusa_status_t medusa_device_status(int32_t* status, int32_t* detail, int clear);
 
+/* Test hook of the failure-detection path; not for production use.  Later
+ * launches of the batch-1 / fp32 heads kernel (medusa_heads_topk with B = 1,
+ * or fp32 weights) wait, between the residual block and the vocabulary
+ * projection, for extra_arrivals more CTAs than the launch has, so with
+ * extra_arrivals > 0 that wait cannot be satisfied, and that wait gives up
+ * after limit_ns (0: the default of about 2 s).  A wait that gives up sets
+ * the device status (MEDUSA_ERR_TIMEOUT, detail 1 for this wait), the
+ * kernel's other roles stop waiting as soon as they see it, its copies in
+ * flight land, and it returns without writing the top-k; zero the workspace
+ * before the next call.
+ * medusa_test_heads_wait(0, 0) restores the defaults.  Process-wide.
+ * Errors: INVALID_ARG unless 0 <= extra_arrivals <= 1024 and limit_ns >= 0.
+ * The pages have no counterpart. */
+medusa_status_t medusa_test_heads_wait(int extra_arrivals, long long limit_ns);
+
 /* ------------------------------------------------------------------------ */
 /* Candidate tree                                                            */
 /* ------------------------------------------------------------------------ */

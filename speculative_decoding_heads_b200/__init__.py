@@ -47,7 +47,7 @@ MAX_T, MAX_K, MAX_TOPK, MAX_B, MAX_SHARDS = 256, 16, 32, 64, 64
 
 # Every symbol the header declares (checked by the CPU tests).
 EXPORTED = [
-    "medusa_last_error", "medusa_abi_version", "medusa_device_status",
+    "medusa_last_error", "medusa_abi_version", "medusa_device_status", "medusa_test_heads_wait",
     "medusa_tree_choices_ranksum", "medusa_tree_create", "medusa_tree_destroy",
     "medusa_tree_info", "medusa_tree_tables",
     "medusa_heads_workspace_size", "medusa_heads_topk", "medusa_heads_topk_noalloc",
@@ -101,6 +101,7 @@ def _sig(name, restype, argtypes):
 _sig("medusa_last_error", ctypes.c_char_p, [])
 _sig("medusa_abi_version", _i32, [])
 _sig("medusa_device_status", _i32, [_pi32, _pi32, _i32])
+_sig("medusa_test_heads_wait", _i32, [_i32, ctypes.c_longlong])
 _sig("medusa_tree_choices_ranksum", _i32, [_i32, _i32, _i32, _pi32, _pi32])
 _sig("medusa_tree_create", _i32, [_pi32, _pi32, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp)])
 _sig("medusa_tree_destroy", None, [_vp])
@@ -230,6 +231,12 @@ def device_status(clear: bool = True) -> Tuple[int, int]:
     st, det = ctypes.c_int32(0), ctypes.c_int32(0)
     _check(_lib.medusa_device_status(ctypes.byref(st), ctypes.byref(det), int(clear)))
     return st.value, det.value
+
+
+def medusa_test_heads_wait(extra_arrivals: int, limit_ns: int):
+    """Test hook of the failure-detection path (see the C header): (1, 10**6) makes the batch-1 heads
+    kernel's wait between its two phases run out after 1 ms; (0, 0) restores the defaults."""
+    _check(_lib.medusa_test_heads_wait(int(extra_arrivals), int(limit_ns)))
 
 
 # ---------------------------------------------------------------------------

@@ -33,6 +33,7 @@
 //    entry.  At the end each CTA publishes its lists, and the last CTA to
 //    finish merges them (k rounds of a warp arg-max over the published
 //    candidates) and resets the counters for the next call.
+#include <atomic>
 #include <cfloat>
 #include <cstdint>
 
@@ -78,6 +79,8 @@ struct HeadsArgs {
   int p1_max;             // most phase-1 rows of any CTA
   int do_build;           // 1: the last CTA also builds the candidate tree (S4) for all B sequences
   TreeBuild build;
+  unsigned s1_extra;      // arrivals the S1 -> S2 wait expects beyond the G CTAs (0; a test sets 1)
+  unsigned long long s1_limit_ns;   // bound on the S1 -> S2 wait (the other waits take kSpinLimitNs)
 };
 
 template <typename TW>
@@ -246,6 +249,18 @@ __device__ __forceinline__ void pack_x(const float* f, uint64_t* xp) {
 
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
 
+// Waits for the phase with the given parity; gives up after limit_ns, or as
+// soon as another role of the CTA has aborted (*abort == 1), and returns false.
+__device__ __forceinline__ bool wait_or_quit(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                             unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0 && (*abort == 1 || globaltimer_ns() - t0 > limit_ns)) return false;
+  }
+}
+
 // CTA of row r when n rows are split evenly over G CTAs (inverse of part_lo).
 __device__ __forceinline__ int part_of(int r, int n, int G) {
   return static_cast<int>((static_cast<long long>(r + 1) * G - 1) / n);
@@ -375,7 +390,7 @@ __global__ void __launch_bounds__(heads_threads<NB, VPT, R>(), 1) heads_kernel(c
       int s = 0;
       for (; pc.phase != 3; ++s) {
         const int slot = s % NS;
-        if (s >= NS && !mbar_wait(&empty[slot], static_cast<uint32_t>(((s / NS) - 1) & 1))) {
+        if (s >= NS && !wait_or_quit(&empty[slot], static_cast<uint32_t>(((s / NS) - 1) & 1), flag, kSpinLimitNs)) {
           set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsStageWait);
           flag[0] = 1;
           break;
@@ -422,7 +437,7 @@ __global__ void __launch_bounds__(heads_threads<NB, VPT, R>(), 1) heads_kernel(c
       const int khead = cc.head;   // uniform per stage
       if (cc.phase == 2 && khead != cur_head2) {
         if (!u_ok) {
-          if (!mbar_wait(u_ready, 0u)) {
+          if (!wait_or_quit(u_ready, 0u, flag, kSpinLimitNs)) {
             set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsS1Wait);
             flag[0] = 1;
           }
@@ -442,7 +457,7 @@ __global__ void __launch_bounds__(heads_threads<NB, VPT, R>(), 1) heads_kernel(c
             }
           }
       }
-      if (!mbar_wait(&full[slot], static_cast<uint32_t>((s / NS) & 1))) {
+      if (!wait_or_quit(&full[slot], static_cast<uint32_t>((s / NS) & 1), flag, kSpinLimitNs)) {
         set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsStageWait);
         flag[0] = 1;
       }
@@ -474,7 +489,7 @@ __global__ void __launch_bounds__(heads_threads<NB, VPT, R>(), 1) heads_kernel(c
       if (lane == 0) mbar_arrive_cta(&empty[slot]);   // this warp is done with the stage's bytes
       int idx = 0;
       WarpFold<RNB, 16>::run(acc, lane, idx);
-      if (s >= NS && !mbar_wait(&pfree[slot], static_cast<uint32_t>(((s / NS) - 1) & 1))) {
+      if (s >= NS && !wait_or_quit(&pfree[slot], static_cast<uint32_t>(((s / NS) - 1) & 1), flag, kSpinLimitNs)) {
         set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsStageWait);
         flag[0] = 1;
         break;
@@ -506,8 +521,8 @@ __global__ void __launch_bounds__(heads_threads<NB, VPT, R>(), 1) heads_kernel(c
       if (lane == 0) {
         atom_add_release_gpu(&a.counters[0], 1u);
         const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire_gpu(&a.counters[0]) < static_cast<unsigned>(G)) {
-          if (globaltimer_ns() - t0 > kSpinLimitNs) {
+        while (ld_acquire_gpu(&a.counters[0]) < static_cast<unsigned>(G) + a.s1_extra) {
+          if (globaltimer_ns() - t0 > a.s1_limit_ns) {
             set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsS1Wait);
             flag[0] = 1;
             break;
@@ -523,7 +538,7 @@ __global__ void __launch_bounds__(heads_threads<NB, VPT, R>(), 1) heads_kernel(c
     cursor_start<R>(cc, a, p1_lo, p1_hi, p2_lo, p2_hi);
     for (int s = 0; cc.phase != 3; ++s) {
       const int slot = s % NS;
-      if (!mbar_wait(&pready[slot], static_cast<uint32_t>((s / NS) & 1))) {
+      if (!wait_or_quit(&pready[slot], static_cast<uint32_t>((s / NS) & 1), flag, kSpinLimitNs)) {
         set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailHeadsStageWait);
         flag[0] = 1;
       }
@@ -688,6 +703,10 @@ cudaError_t dispatch_nb(const HeadsArgs& a, const Plan& p, cudaStream_t stream) 
   return dispatch_vpt<TW, 4>(a, p, stream);
 }
 
+// Test hook of the failure-detection path (medusa_test_heads_wait).
+std::atomic<unsigned> g_test_s1_extra{0};
+std::atomic<unsigned long long> g_test_limit_ns{0};
+
 }  // namespace
 
 size_t heads_workspace_bytes(int B, int d, int V, int K, int topk) {
@@ -739,6 +758,9 @@ medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, cons
   a.G = G;
   a.nvec = (dtype == MEDUSA_BF16) ? d / 8 : d / 4;
   a.p1_max = static_cast<int>((static_cast<long long>(K) * d + G - 1) / G) + 1;
+  a.s1_extra = g_test_s1_extra.load();
+  const unsigned long long lim = g_test_limit_ns.load();
+  a.s1_limit_ns = lim ? lim : kSpinLimitNs;
   for (int b0 = 0; b0 < B; b0 += kMaxNB) {
     a.b0 = b0;
     a.nb = (B - b0) < kMaxNB ? (B - b0) : kMaxNB;
@@ -756,3 +778,11 @@ medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, cons
 }
 
 }  // namespace medusa
+
+extern "C" medusa_status_t medusa_test_heads_wait(int extra_arrivals, long long limit_ns) {
+  if (extra_arrivals < 0 || extra_arrivals > 1024 || limit_ns < 0)
+    return medusa::fail(MEDUSA_ERR_INVALID_ARG, "medusa_test_heads_wait: extra_arrivals in [0, 1024], limit_ns >= 0");
+  medusa::g_test_s1_extra.store(static_cast<unsigned>(extra_arrivals));
+  medusa::g_test_limit_ns.store(static_cast<unsigned long long>(limit_ns));
+  return MEDUSA_OK;
+}
