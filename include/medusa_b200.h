@@ -371,6 +371,71 @@ medusa_status_t medusa_accept_kv(const medusa_tree_t* tree, int layers, int B, i
                                  const int32_t* accept_len, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* The base model's forward over the tree tokens (tree_decoding)             */
+/* ------------------------------------------------------------------------ */
+
+/* One LLaMA (Vicuna) decoder layer's weights, bf16 device pointers, hd = 128
+ * (H = D / 128 heads), F the feed-forward width (multiples of 128):
+ *   attn_norm, mlp_norm [D]   RMSNorm weights (eps 1e-6)
+ *   wqkv  [3D, D]  the rows of Wq, Wk and Wv (out x in) in that order, each
+ *                  head's 128 rows packed so that row 2j is feature j and row
+ *                  2j+1 feature j + 64 (the two features one rotary pair turns)
+ *   wo    [D, D]   output projection
+ *   wgu   [2F, D]  gate and up projections interleaved: row 2j is W_gate row
+ *                  j, row 2j+1 is W_up row j
+ *   wdown [D, F]   down projection
+ * The packing only reorders rows; medusa_decoder_pack_rows gives the order. */
+typedef struct medusa_decoder_layer {
+  const void* attn_norm;
+  const void* wqkv;
+  const void* wo;
+  const void* mlp_norm;
+  const void* wgu;
+  const void* wdown;
+} medusa_decoder_layer_t;
+
+typedef struct medusa_decoder {
+  int layers, D, F, V;
+  const void* embed;                    /* [V, D] bf16 */
+  const medusa_decoder_layer_t* layer;  /* HOST array of `layers` entries (device pointers inside) */
+  const void* final_norm;               /* [D] bf16 */
+  const void* lm_head;                  /* [V, D] bf16, no bias */
+} medusa_decoder_t;
+
+/* Host.  The source row of every packed row: for which = 0 (wqkv, D rows of
+ * one of Wq / Wk / Wv; apply it to each of the three) out[r] = the row of
+ * the unpacked matrix that packed row r holds (r < D); for which = 1 (wgu,
+ * 2F rows) out[r] = j for W_gate row j (r = 2j) and F + j for W_up row j
+ * (r = 2j + 1), indexing the unpacked [W_gate; W_up].  INVALID_ARG unless D
+ * (which 0) is a multiple of 128 and n > 0. */
+medusa_status_t medusa_decoder_pack_rows(int which, int n, int32_t* out);
+
+size_t medusa_tree_decode_workspace_size(const medusa_tree_t* tree, const medusa_decoder_t* model, int B);
+
+/* The base model's forward over the T tree tokens of each of B sequences
+ * ["Medusa API参考", 核心功能函数: tree_decoding (medusa_position_ids =
+ * prefix length + depth, the tree mask, the cached K/V); "基于 Medusa 头的投机
+ * 解码架构", 性能基准测试: Vicuna bases]: embedding of tree_tokens [B, T], for
+ * every layer l (x the fp32 residual stream of the B*T tokens)
+ *   x += Wo . tree_attention(RoPE(Wq n), RoPE(Wk n), Wv n),  n = RMSNorm(x)
+ *   x += Wdown (SiLU(Wgate n) * (Wup n)),                   n = RMSNorm(x)
+ * with RoPE at position seq_lens[b] + depth(node) (pair i with i + 64, base
+ * 10000), the tree's own k and v written to cache rows seq_lens[b] + node of
+ * layer l (caches [layers, B, H, Lcap, 128] bf16; rows below seq_lens[b]
+ * hold the prefix), attention as medusa_tree_attention; then
+ *   logits [B*T, V] fp32 = lm_head . RMSNorm(x),   hidden [B*T, D] fp32 = x
+ * (hidden may be NULL).  The normalised activations, q/k/v, the attention
+ * output and the SwiGLU activation are rounded to bf16 between the products
+ * (fp32 accumulation).  Requires seq_lens[b] + T <= Lcap (a violation sets
+ * MEDUSA_ERR_DEVICE_CHECK); a token outside [0, V) sets
+ * MEDUSA_ERR_DEVICE_CHECK.  Every matrix product streams its weights once
+ * per 64 tree tokens.  Pointers 16-byte aligned. */
+medusa_status_t medusa_tree_decode(const medusa_tree_t* tree, const medusa_decoder_t* model, int B,
+                                   const int32_t* tree_tokens, void* k_cache, void* v_cache, int Lcap,
+                                   const int32_t* seq_lens, float* logits, float* hidden, void* workspace,
+                                   size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* The whole step                                                            */
 /* ------------------------------------------------------------------------ */
 

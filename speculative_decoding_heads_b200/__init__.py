@@ -56,6 +56,7 @@ EXPORTED = [
     "medusa_tree_attention_split", "medusa_attention_combine", "medusa_attention_rescale",
     "medusa_posterior_workspace_size", "medusa_evaluate_posterior",
     "medusa_accept_kv",
+    "medusa_decoder_pack_rows", "medusa_tree_decode_workspace_size", "medusa_tree_decode",
     "medusa_step_workspace_size", "medusa_step",
 ]
 
@@ -91,6 +92,17 @@ class StepArgs(ctypes.Structure):
     ]
 
 
+class DecoderLayer(ctypes.Structure):
+    """Mirror of ``medusa_decoder_layer_t`` (device pointers)."""
+    _fields_ = [("attn_norm", _vp), ("wqkv", _vp), ("wo", _vp), ("mlp_norm", _vp), ("wgu", _vp), ("wdown", _vp)]
+
+
+class DecoderModel(ctypes.Structure):
+    """Mirror of ``medusa_decoder_t``."""
+    _fields_ = [("layers", _i32), ("D", _i32), ("F", _i32), ("V", _i32), ("embed", _vp),
+                ("layer", ctypes.POINTER(DecoderLayer)), ("final_norm", _vp), ("lm_head", _vp)]
+
+
 def _sig(name, restype, argtypes):
     fn = getattr(_lib, name)
     fn.restype = restype
@@ -123,6 +135,10 @@ _sig("medusa_posterior_workspace_size", _sz, [_vp, _i32])
 _sig("medusa_evaluate_posterior", _i32,
      [_vp, _i32, _i32, _vp, _vp, _i32, _f32, _f32, _f32, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _sig("medusa_accept_kv", _i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp])
+_sig("medusa_decoder_pack_rows", _i32, [_i32, _i32, _pi32])
+_sig("medusa_tree_decode_workspace_size", _sz, [_vp, ctypes.POINTER(DecoderModel), _i32])
+_sig("medusa_tree_decode", _i32, [_vp, ctypes.POINTER(DecoderModel), _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp,
+                                   _sz, _vp])
 _sig("medusa_step_workspace_size", _sz, [ctypes.POINTER(StepArgs)])
 _sig("medusa_step", _i32, [ctypes.POINTER(StepArgs), _vp, _sz, _vp])
 
@@ -453,6 +469,78 @@ def medusa_accept_kv(tree: Tree, k_cache, v_cache, seq_lens, best_path, accept_l
     _check(_lib.medusa_accept_kv(tree.handle, layers, B, H, hd, _dtype(k_cache), _p(k_cache),
                                  _p(v_cache), Lcap, _p(seq_lens), _p(best_path), _p(accept_len),
                                  _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# the base model's forward over the tree tokens
+# ---------------------------------------------------------------------------
+
+
+def medusa_decoder_pack_rows(which: int, n: int) -> List[int]:
+    """Source row of every packed row (which 0: one of Wq/Wk/Wv with n = D rows; which 1: [W_gate;
+    W_up] with n = 2F rows), as the C call documents."""
+    out = (ctypes.c_int32 * n)()
+    _check(_lib.medusa_decoder_pack_rows(int(which), int(n), out))
+    return list(out)
+
+
+class Decoder:
+    """A base model for ``medusa_tree_decode``: bf16 device tensors, hd = 128.
+
+    ``layers`` is a list of dicts with attn_norm [D], Wq, Wk, Wv, Wo [D, D], mlp_norm [D],
+    W_gate, W_up [F, D], W_down [D, F] (out x in); they are packed here (a row reordering, done
+    once when the model is set up) into the layout the kernels read."""
+
+    def __init__(self, embed, layers, final_norm, lm_head):
+        V, D = embed.shape
+        F = layers[0]["W_gate"].shape[0]
+        dev = embed.device
+        iq = torch.tensor(medusa_decoder_pack_rows(0, D), dtype=torch.long, device=dev)
+        igu = torch.tensor(medusa_decoder_pack_rows(1, 2 * F), dtype=torch.long, device=dev)
+        bf = lambda t: t.to(device=dev, dtype=torch.bfloat16).contiguous()
+        self.tensors = []
+        for ly in layers:
+            wqkv = torch.cat([bf(ly["Wq"])[iq], bf(ly["Wk"])[iq], bf(ly["Wv"])[iq]], 0).contiguous()
+            wgu = torch.cat([bf(ly["W_gate"]), bf(ly["W_up"])], 0)[igu].contiguous()
+            self.tensors.append(dict(attn_norm=bf(ly["attn_norm"]), wqkv=wqkv, wo=bf(ly["Wo"]),
+                                     mlp_norm=bf(ly["mlp_norm"]), wgu=wgu, wdown=bf(ly["W_down"])))
+        self.embed, self.final_norm, self.lm_head = bf(embed), bf(final_norm), bf(lm_head)
+        self.D, self.F, self.V = D, F, V
+        arr = (DecoderLayer * len(layers))()
+        for i, t in enumerate(self.tensors):
+            for k, v in t.items():
+                _spec(k, v, v.shape, torch.bfloat16)
+                setattr(arr[i], k, _p(v).value)
+        self._layers = arr
+        self.c = DecoderModel(len(layers), D, F, V, _p(self.embed).value, arr, _p(self.final_norm).value,
+                              _p(self.lm_head).value)
+
+
+def medusa_tree_decode_workspace_size(tree: Tree, model: Decoder, B: int) -> int:
+    return int(_lib.medusa_tree_decode_workspace_size(tree.handle, ctypes.byref(model.c), int(B)))
+
+
+def medusa_tree_decode(tree: Tree, model: Decoder, tree_tokens, k_cache, v_cache, seq_lens, logits, ws,
+                       hidden=None, stream=None):
+    """The base model's forward over the tree tokens: tree_tokens [B, T] int32; caches
+    [layers, B, H, Lcap, 128] bf16 (the tree's k/v are written at rows seq_lens[b] + node);
+    logits [B*T, V] fp32; hidden [B*T, D] fp32 (optional, the residual stream after the last layer)."""
+    _require(tree_tokens.dim() == 2 and tree_tokens.shape[1] == tree.T, "tree_tokens must be [B, T]")
+    B = tree_tokens.shape[0]
+    D, V, H = model.D, model.V, model.D // 128
+    _spec("tree_tokens", tree_tokens, (B, tree.T), torch.int32)
+    _require(k_cache.dim() == 5, "caches must be [layers, B, H, Lcap, 128]")
+    Lcap = k_cache.shape[3]
+    shape = (len(model.tensors), B, H, Lcap, 128)
+    _spec("k_cache", k_cache, shape, torch.bfloat16)
+    _spec("v_cache", v_cache, shape, torch.bfloat16)
+    _spec("seq_lens", seq_lens, (B,), torch.int32)
+    _spec("logits", logits, (B * tree.T, V), torch.float32)
+    if hidden is not None:
+        _spec("hidden", hidden, (B * tree.T, D), torch.float32)
+    nbytes = _nbytes("ws", ws)
+    _check(_lib.medusa_tree_decode(tree.handle, ctypes.byref(model.c), B, _p(tree_tokens), _p(k_cache), _p(v_cache),
+                                   Lcap, _p(seq_lens), _p(logits), _p(hidden), _p(ws), nbytes, _stream(stream)))
 
 
 def make_step_args(tree: Tree, t: dict, mode: int, temperature=0.0, eps=0.09, alpha=0.3,

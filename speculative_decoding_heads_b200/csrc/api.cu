@@ -342,6 +342,69 @@ extern "C" medusa_status_t medusa_accept_kv(const medusa_tree_t* tree, int layer
                           accept_len, stream);
 }
 
+// ---- the base model's forward over the tree -------------------------------
+
+extern "C" medusa_status_t medusa_decoder_pack_rows(int which, int n, int32_t* out) {
+  const char* fn = "medusa_decoder_pack_rows";
+  if (!out || n <= 0 || (which != 0 && which != 1)) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": arguments");
+  if (which == 0) {
+    if (n % 128 != 0) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": D must be a multiple of 128");
+    for (int r = 0; r < n; ++r) {
+      const int head = r / 128, lr = r % 128;
+      out[r] = head * 128 + (lr >> 1) + (lr & 1) * 64;
+    }
+  } else {
+    if (n % 2 != 0) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": 2F rows");
+    for (int r = 0; r < n; ++r) out[r] = (r & 1) ? n / 2 + (r >> 1) : (r >> 1);
+  }
+  return MEDUSA_OK;
+}
+
+static medusa_status_t check_decoder(const medusa_tree_t* tree, const medusa_decoder_t* m, int B, const char* fn) {
+  medusa_status_t st = check_tree(tree, fn);
+  if (st != MEDUSA_OK) return st;
+  if (!m || !m->layer || !m->embed || !m->final_norm || !m->lm_head)
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null model pointer");
+  if (m->layers < 1 || m->D < 128 || m->D % 128 != 0 || m->F < 128 || m->F % 128 != 0 || m->V < 1 || B < 1 ||
+      B > MEDUSA_MAX_B)
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": layers, D, F, V or B out of range");
+  if (static_cast<long long>(B) * tree->T > (1 << 20))
+    return fail(MEDUSA_ERR_UNSUPPORTED, std::string(fn) + ": too many tree tokens");
+  for (int l = 0; l < m->layers; ++l) {
+    const medusa_decoder_layer_t& y = m->layer[l];
+    if (!y.attn_norm || !y.wqkv || !y.wo || !y.mlp_norm || !y.wgu || !y.wdown)
+      return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null layer pointer");
+    if (!aligned16(y.wqkv) || !aligned16(y.wo) || !aligned16(y.wgu) || !aligned16(y.wdown))
+      return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": misaligned weights");
+  }
+  if (!aligned16(m->embed) || !aligned16(m->lm_head)) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": misaligned");
+  return MEDUSA_OK;
+}
+
+extern "C" size_t medusa_tree_decode_workspace_size(const medusa_tree_t* tree, const medusa_decoder_t* m, int B) {
+  if (!tree || !m || B < 1 || sm_count() <= 0) return 0;
+  return decoder_workspace_bytes(B * tree->T, m->D, m->F, m->V);
+}
+
+extern "C" medusa_status_t medusa_tree_decode(const medusa_tree_t* tree, const medusa_decoder_t* m, int B,
+                                              const int32_t* tree_tokens, void* k_cache, void* v_cache, int Lcap,
+                                              const int32_t* seq_lens, float* logits, float* hidden,
+                                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const char* fn = "medusa_tree_decode";
+  medusa_status_t st = check_decoder(tree, m, B, fn);
+  if (st != MEDUSA_OK) return st;
+  if (!tree_tokens || !k_cache || !v_cache || !seq_lens || !logits || !workspace)
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (Lcap < tree->T) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": Lcap smaller than the tree");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(logits) || (hidden && !aligned16(hidden)) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": misaligned pointer");
+  if (workspace_bytes < decoder_workspace_bytes(B * tree->T, m->D, m->F, m->V))
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": workspace too small");
+  return launch_tree_decode(tree->dev, m, B, tree_tokens, k_cache, v_cache, Lcap, seq_lens, logits, hidden, workspace,
+                            stream);
+}
+
 // ---- the whole step ------------------------------------------------------
 
 namespace {

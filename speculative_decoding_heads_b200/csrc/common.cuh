@@ -18,6 +18,9 @@ enum DeviceDetail : int {
   kDetailAcceptSeqLen = 5,    // accept_kv: seq_lens[b] + T > Lcap or bad accept_len
   kDetailPosteriorArgs = 6,   // posterior: a candidate token outside [0, V)
   kDetailPosteriorWait = 7,   // step: the compaction waited for a sequence's walk in vain
+  kDetailDecoderWait = 8,     // tree decode: a matrix product's copy or product never completed
+  kDetailDecoderToken = 9,    // tree decode: a tree token outside [0, V)
+  kDetailDecoderSeqLen = 10,  // tree decode: seq_lens[b] + T > Lcap
 };
 
 // Address of the current device's status word ([0] status, [1] detail).

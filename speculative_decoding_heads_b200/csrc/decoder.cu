@@ -1,0 +1,521 @@
+// The base model's forward over the tree tokens (tree_decoding): the step
+// either side of tree attention.  "Medusa API参考：核心函数与类详解", 核心功能函数:
+// tree_decoding runs the base model once over every tree token at the tree's
+// position ids (prefix length + depth) under the tree mask, against the
+// cached K/V, and its logits feed evaluate_posterior; "基于 Medusa 头的投机解码架构",
+// 性能基准测试: the base models are Vicuna (LLaMA) 7B/13B/33B.  The layer is the
+// LLaMA decoder layer: RMSNorm, Q/K/V with rotary embedding (pair i with
+// i + hd/2, base 10000), tree attention, output projection and residual,
+// RMSNorm, SwiGLU feed-forward and residual; then a final RMSNorm and the LM
+// head.
+//
+// Every matrix product here is weights x (at most 64 tree tokens): the
+// weights stream from HBM once per pass of 64 tokens, as the A operand of
+// M = 128, N = 64, K = 16 tcgen05 products (TMA boxes of 128 rows x 2 x 64
+// columns, 128-byte swizzle, no multicast), the tokens' activations are the
+// B operand, and the fp32 accumulators live in tensor memory.  The W/64/2
+// ring stages of a product are split evenly over the CTAs (stream-K); a tile
+// of 128 rows cut by a range boundary is summed, per quarter of its rows, by
+// the last CTA to finish it, in CTA order.  The epilogue is fused per
+// product:
+//   QKV     rotary embedding of q and k at position L_b + depth, q to its
+//           buffer, k and v into the cache rows L_b + node
+//   RESID   x += product (the fp32 residual stream)
+//   SWIGLU  act = SiLU(gate) * up, bf16
+//   LOGITS  fp32 logits
+// For QKV and SWIGLU the rows of the packed weights interleave the two rows
+// an output needs (q/k features i and i + hd/2; gate and up of one feature),
+// so the pair sits in lanes 2j and 2j + 1 of one warp.
+#include <cfloat>
+#include <cudaTypedefs.h>
+
+#include "tcgen05.cuh"
+
+namespace medusa {
+namespace {
+
+constexpr int kTileRows = 128;
+constexpr int kKStep = 64;
+constexpr int kKPS = 2;                        // column blocks per ring stage
+constexpr int kN = 64;                         // tokens per pass (MMA N)
+constexpr int kWBlock = kTileRows * 128;       // 16 KB
+constexpr int kXBlock = kN * 128;              // 8 KB
+constexpr int kSB = kKPS * (kWBlock + kXBlock);   // 48 KB per stage
+constexpr int kNS = 4;
+constexpr int kThreads = 256;                  // warps 0 producer, 1 MMA, 4-7 epilogue
+constexpr uint32_t kTmemCols = 128;            // two accumulators of 64 columns
+constexpr int kSmem = 1024 + kNS * kSB + 1024;
+constexpr float kRmsEps = 1e-6f;
+
+enum Mode : int { kQKV = 0, kResid = 1, kSwiGLU = 2, kLogits = 3 };
+
+struct GemmArgs {
+  int rows;               // weight rows
+  int kdim;               // reduction length (a multiple of 128)
+  int tiles, nst, W, G;   // tiles of 128 rows, stages per tile, all stages, CTAs
+  int tok0, ntok;         // this pass: tokens tok0 .. tok0 + 63 (clipped to ntok)
+  float* part;            // [G, 2, 128, 64]
+  unsigned* tile_cnt;     // [tiles * 4]
+  int* status;
+  // QKV
+  uint16_t* q_out;        // [ntok, H, 128]
+  uint16_t* k_cache;      // this layer: [B, H, Lcap, 128]
+  uint16_t* v_cache;
+  const int32_t* seq_lens;
+  const int32_t* depth;   // [T]
+  int T, H, Lcap;
+  // RESID
+  float* x;               // [ntok, rows]
+  // SWIGLU
+  uint16_t* act;          // [ntok, rows / 2]
+  // LOGITS
+  float* logits;          // [ntok, rows]
+};
+
+struct Bars {
+  uint64_t full[kNS], empty[kNS];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ int stage_lo(int c, const GemmArgs& a) {
+  return static_cast<int>(static_cast<long long>(a.W) * c / a.G);
+}
+__device__ __forceinline__ int stage_owner(int st, const GemmArgs& a) {
+  return static_cast<int>((static_cast<long long>(st + 1) * a.G - 1) / a.W);
+}
+
+struct Unit {
+  int tile, k0, k1;   // column blocks [k0, k1) of one tile
+};
+
+__device__ __forceinline__ bool next_unit(const GemmArgs& a, int& st, int st_hi, Unit& x) {
+  if (st >= st_hi) return false;
+  x.tile = st / a.nst;
+  const int t0 = x.tile * a.nst;
+  const int e = st_hi < t0 + a.nst ? st_hi : t0 + a.nst;
+  x.k0 = (st - t0) * kKPS;
+  x.k1 = (e - t0) * kKPS;
+  st = e;
+  return true;
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Bars* bs, int* status) {
+  if (bs->abort) return false;
+  if (mbar_wait(bar, parity)) return true;
+  set_device_status(status, MEDUSA_ERR_TIMEOUT, kDetailDecoderWait);
+  bs->abort = 1;
+  return false;
+}
+
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
+__device__ __forceinline__ float bf(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
+
+// The epilogue of one finished tile row (all 64 token columns in acc).
+template <int kMode>
+__device__ __forceinline__ void epilogue_row(const GemmArgs& a, int tile, int r, int lane, const float (&acc)[kN]) {
+  const int nvalid = a.ntok - a.tok0 < kN ? a.ntok - a.tok0 : kN;
+  if constexpr (kMode == kQKV) {
+    const int which = tile / a.H, h = tile - which * a.H;   // 0 q, 1 k, 2 v; head h
+    const int j = r >> 1;                                   // pair index (frequency)
+    const int feat = j + (r & 1) * 64;                      // feature within the head
+    // rotation frequency base^(-2j/128), angle reduced in double
+    const double inv = exp2(-static_cast<double>(2 * j) / 128.0 * 13.287712379549449);   // log2(10000)
+    for (int c = 0; c < kN; ++c) {
+      const float own = acc[c];
+      const float other = __shfl_xor_sync(0xffffffffu, own, 1);
+      if (c >= nvalid) continue;
+      const int n = a.tok0 + c;
+      const int b = n / a.T, node = n - b * a.T;
+      const int L = a.seq_lens[b];
+      if (L < 0 || L + a.T > a.Lcap) {   // the tree's rows would not fit in the cache
+        set_device_status(a.status, MEDUSA_ERR_DEVICE_CHECK, kDetailDecoderSeqLen);
+        continue;
+      }
+      float out = own;
+      if (which < 2) {
+        const double ang = static_cast<double>(L + a.depth[node]) * inv;
+        const double red = ang - 6.283185307179586 * rint(ang / 6.283185307179586);
+        float sn, cs;
+        sincosf(static_cast<float>(red), &sn, &cs);
+        out = (r & 1) ? other * sn + own * cs : own * cs - other * sn;
+      }
+      const uint16_t v = f32_to_bf16_rne(out);
+      if (which == 0) {
+        a.q_out[(static_cast<size_t>(n) * a.H + h) * 128 + feat] = v;
+      } else {
+        uint16_t* cache = which == 1 ? a.k_cache : a.v_cache;
+        cache[((static_cast<size_t>(b) * a.H + h) * a.Lcap + L + node) * 128 + feat] = v;
+      }
+    }
+  } else if constexpr (kMode == kSwiGLU) {
+    const int j = tile * 64 + (r >> 1);   // output feature
+    for (int c = 0; c < kN; ++c) {
+      const float own = acc[c];
+      const float up = __shfl_xor_sync(0xffffffffu, own, 1);
+      if (c >= nvalid || (r & 1) || 2 * j >= a.rows) continue;
+      a.act[static_cast<size_t>(a.tok0 + c) * (a.rows / 2) + j] = f32_to_bf16_rne(silu(own) * up);
+    }
+  } else {
+    const int f = tile * kTileRows + r;
+    if (f >= a.rows) return;
+    for (int c = 0; c < nvalid; ++c) {
+      const size_t o = static_cast<size_t>(a.tok0 + c) * a.rows + f;
+      if constexpr (kMode == kResid) {
+        a.x[o] += acc[c];
+      } else {
+        a.logits[o] = acc[c];
+      }
+    }
+  }
+  (void)lane;
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+    wgemm_kernel(const __grid_constant__ CUtensorMap w_map, const __grid_constant__ CUtensorMap x_map,
+                 const GemmArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bs = reinterpret_cast<Bars*>(smem + kNS * kSB);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cta = blockIdx.x;
+  const int st_lo = stage_lo(cta, a), st_hi = stage_lo(cta + 1, a);
+
+  if (tid == 0) {
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&bs->full[s], 1);
+      mbar_init(&bs->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bs->acc_full[b], 1);
+      mbar_init(&bs->acc_empty[b], 4);
+    }
+    mbar_init(&bs->mma_done, 1);
+    bs->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&bs->tmem_base, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bs->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::prefetch_tensormap(&w_map);
+      tc::prefetch_tensormap(&x_map);
+      const uint64_t pol = l2_evict_first_policy();
+      int g = 0;
+      Unit x;
+      for (int st = st_lo; !bs->abort && next_unit(a, st, st_hi, x);) {
+        for (int j = x.k0; j < x.k1; j += kKPS, ++g) {
+          const int slot = g % kNS;
+          if (g >= kNS && !wait_or_abort(&bs->empty[slot], ((g / kNS) - 1) & 1, bs, a.status)) break;
+          mbar_arrive_expect_tx(&bs->full[slot], kSB);
+          unsigned char* sd = smem + slot * kSB;
+          tc::tma_load_4d_hint(sd, &w_map, 0, x.tile * kTileRows, j, 0, &bs->full[slot], pol);
+          tc::tma_load_4d(sd + kKPS * kWBlock, &x_map, 0, a.tok0, j, 0, &bs->full[slot]);
+        }
+      }
+      for (int t = g - kNS < 0 ? 0 : g - kNS; t < g; ++t) mbar_wait(&bs->full[t % kNS], (t / kNS) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16_f32(kTileRows, kN, 0);
+      const uint32_t sbase = smem_u32(smem);
+      int g = 0, n = 0;
+      Unit x;
+      for (int st = st_lo; !bs->abort && next_unit(a, st, st_hi, x); ++n) {
+        const int buf = n & 1;
+        if (n >= 2 && !wait_or_abort(&bs->acc_empty[buf], ((n >> 1) - 1) & 1, bs, a.status)) break;
+        tc::fence_after_sync();
+        const uint32_t d = tmem + buf * kN;
+        bool ok = true;
+        for (int j = x.k0; j < x.k1; j += kKPS, ++g) {
+          const int slot = g % kNS;
+          if (!wait_or_abort(&bs->full[slot], (g / kNS) & 1, bs, a.status)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t wa = sbase + slot * kSB, xa = wa + kKPS * kWBlock;
+#pragma unroll
+          for (int c = 0; c < kKPS; ++c)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = tc::smem_desc_sw128(wa + c * kWBlock + kk * 32, 16, 1024);
+              const uint64_t bd = tc::smem_desc_sw128(xa + c * kXBlock + kk * 32, 16, 1024);
+              tc::mma_ss(d, ad, bd, idesc, (j > x.k0 || c > 0 || kk > 0) ? 1u : 0u);
+            }
+          tc::mma_commit(&bs->empty[slot]);
+        }
+        if (!ok) break;
+        tc::mma_commit(&bs->acc_full[buf]);
+      }
+      tc::mma_commit(&bs->mma_done);
+      mbar_wait(&bs->mma_done, 0);
+    }
+  } else if (warp >= 4) {
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    const int r = 32 * q + lane;
+    int n = 0;
+    Unit x;
+    for (int st = st_lo; next_unit(a, st, st_hi, x); ++n) {
+      const int buf = n & 1;
+      if (!wait_or_abort(&bs->acc_full[buf], (n >> 1) & 1, bs, a.status)) break;
+      tc::fence_after_sync();
+      float acc[kN];
+      tc::tmem_ld32(tmem + lane_off + buf * kN, acc);
+      tc::tmem_ld32(tmem + lane_off + buf * kN + 32, acc + 32);
+      tc::tmem_wait_ld();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bs->acc_empty[buf]);
+      const int t0 = x.tile * a.nst;
+      const int c_first = stage_owner(t0, a), c_last = stage_owner(t0 + a.nst - 1, a);
+      if (c_first != c_last) {
+        // A tile shared with other CTAs: the last to finish sums the partials in CTA order.
+        const int slot = x.tile == st_lo / a.nst ? 0 : 1;
+        float* mine = a.part + ((static_cast<size_t>(cta) * 2 + slot) * kTileRows + r) * kN;
+#pragma unroll
+        for (int c = 0; c < kN; c += 4)
+          *reinterpret_cast<float4*>(mine + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          unsigned* cnt = &a.tile_cnt[x.tile * 4 + q];
+          last = atom_add_acq_rel_gpu(cnt, 1u) == static_cast<unsigned>(c_last - c_first);
+          if (last) *cnt = 0u;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) continue;
+        __threadfence();
+        float sum[kN];
+#pragma unroll
+        for (int c = 0; c < kN; ++c) sum[c] = 0.f;
+        for (int cc = c_first; cc <= c_last; ++cc) {
+          const int sl = x.tile == stage_lo(cc, a) / a.nst ? 0 : 1;
+          const float* pc = a.part + ((static_cast<size_t>(cc) * 2 + sl) * kTileRows + r) * kN;
+#pragma unroll
+          for (int c = 0; c < kN; c += 4) {
+            const float4 v = cc == cta ? make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3])
+                                       : __ldcg(reinterpret_cast<const float4*>(pc + c));
+            sum[c] += v.x;
+            sum[c + 1] += v.y;
+            sum[c + 2] += v.z;
+            sum[c + 3] += v.w;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < kN; ++c) acc[c] = sum[c];
+      }
+      epilogue_row<kMode>(a, x.tile, r, lane, acc);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---- small kernels ------------------------------------------------------------
+
+// x[n] = embed[tokens[n]] (bf16 -> fp32), n over the B*T tree tokens.
+__global__ void embed_kernel(const int32_t* tokens, const uint16_t* embed, int D, int V, float* x, int* status) {
+  const int n = blockIdx.x;
+  const int tok = tokens[n];
+  if (tok < 0 || tok >= V) {
+    if (threadIdx.x == 0) set_device_status(status, MEDUSA_ERR_DEVICE_CHECK, kDetailDecoderToken);
+    for (int i = threadIdx.x; i < D; i += blockDim.x) x[static_cast<size_t>(n) * D + i] = 0.f;
+    return;
+  }
+  for (int i = threadIdx.x; i < D; i += blockDim.x)
+    x[static_cast<size_t>(n) * D + i] = bf(embed[static_cast<size_t>(tok) * D + i]);
+}
+
+// y[n] = bf16(x[n] / sqrt(mean(x[n]^2) + eps) * w), one CTA per token.
+__global__ void rmsnorm_kernel(const float* x, const uint16_t* w, int D, uint16_t* y) {
+  __shared__ float red[32];
+  const int n = blockIdx.x;
+  const float* xr = x + static_cast<size_t>(n) * D;
+  float s = 0.f;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) s = fmaf(xr[i], xr[i], s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  const float inv = rsqrtf(red[0] / static_cast<float>(D) + kRmsEps);
+  for (int i = threadIdx.x; i < D; i += blockDim.x)
+    y[static_cast<size_t>(n) * D + i] = f32_to_bf16_rne(xr[i] * inv * bf(w[i]));
+}
+
+__global__ void to_bf16_kernel(const float* x, size_t n, uint16_t* y) {
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    y[i] = f32_to_bf16_rne(x[i]);
+}
+
+bool encode_w(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, uint64_t kdim,
+              uint64_t rows, uint32_t box_rows) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kKStep), rows, kdim / kKStep, 1};
+  const cuuint64_t strides[3] = {kdim * 2, kKStep * 2, kdim * rows * 2};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(kKStep), box_rows, static_cast<cuuint32_t>(kKPS), 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Scratch of the matrix products: tile counters, then [G, 2, 128, 64] partials.
+size_t gemm_scratch_bytes(int D, int F, int V) {
+  int rows = 3 * D;
+  if (2 * F > rows) rows = 2 * F;
+  if (V > rows) rows = V;
+  const int tiles = (rows + kTileRows - 1) / kTileRows;
+  const int G = sm_count() > 0 ? sm_count() : 1;
+  return align_up(static_cast<size_t>(tiles) * 16, 256) + align_up(static_cast<size_t>(G) * 2 * kTileRows * kN * 4, 256);
+}
+
+template <int kMode>
+medusa_status_t gemm(const void* Wt, const uint16_t* X, GemmArgs a, void* ws, cudaStream_t stream) {
+  auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
+  if (!enc) return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_tree_decode: cuTensorMapEncodeTiled unavailable");
+  const int G = sm_count();
+  a.tiles = (a.rows + kTileRows - 1) / kTileRows;
+  a.nst = a.kdim / kKStep / kKPS;
+  a.W = a.tiles * a.nst;
+  a.G = a.W < G ? a.W : G;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  a.tile_cnt = reinterpret_cast<unsigned*>(w);
+  a.part = reinterpret_cast<float*>(w + align_up(static_cast<size_t>(a.tiles) * 4 * 4, 256));
+  a.status = device_status_ptr();
+  CUtensorMap wm, xm;
+  if (!encode_w(enc, &wm, Wt, a.kdim, a.rows, kTileRows) || !encode_w(enc, &xm, X, a.kdim, a.ntok, kN))
+    return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_tree_decode: tensor map rejected");
+  auto fn = wgemm_kernel<kMode>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  for (a.tok0 = 0; e == cudaSuccess && a.tok0 < a.ntok; a.tok0 += kN)
+    e = launch_kernel(fn, dim3(a.G), dim3(kThreads), static_cast<size_t>(kSmem), stream, false, wm, xm, a);
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_tree_decode: matrix-product launch", e);
+}
+
+}  // namespace
+
+size_t decoder_workspace_bytes(int ntok, int D, int F, int V) {
+  // The products' scratch; then x fp32, xn bf16, q bf16, attention fp32 and bf16, act bf16.
+  size_t o = gemm_scratch_bytes(D, F, V);
+  o += align_up(static_cast<size_t>(ntok) * D * 4, 256);       // x
+  o += align_up(static_cast<size_t>(ntok) * D * 2, 256);       // xn
+  o += align_up(static_cast<size_t>(ntok) * D * 2, 256);       // q (bf16, [ntok, H, 128])
+  o += align_up(static_cast<size_t>(ntok) * D * 4, 256);       // attention output fp32
+  o += align_up(static_cast<size_t>(ntok) * D * 2, 256);       // attention output bf16
+  o += align_up(static_cast<size_t>(ntok) * F * 2, 256);       // act
+  return o;
+}
+
+medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, int B, const int32_t* tree_tokens,
+                                   void* k_cache, void* v_cache, int Lcap, const int32_t* seq_lens,
+                                   float* logits, float* hidden, void* ws, cudaStream_t stream) {
+  const int D = m->D, F = m->F, V = m->V, H = D / 128;
+  const int ntok = B * t.T;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  size_t o = gemm_scratch_bytes(D, F, V);
+  void* gws = w;
+  float* x = reinterpret_cast<float*>(w + o);
+  o += align_up(static_cast<size_t>(ntok) * D * 4, 256);
+  uint16_t* xn = reinterpret_cast<uint16_t*>(w + o);
+  o += align_up(static_cast<size_t>(ntok) * D * 2, 256);
+  uint16_t* qb = reinterpret_cast<uint16_t*>(w + o);
+  o += align_up(static_cast<size_t>(ntok) * D * 2, 256);
+  float* att = reinterpret_cast<float*>(w + o);
+  o += align_up(static_cast<size_t>(ntok) * D * 4, 256);
+  uint16_t* attb = reinterpret_cast<uint16_t*>(w + o);
+  o += align_up(static_cast<size_t>(ntok) * D * 2, 256);
+  uint16_t* act = reinterpret_cast<uint16_t*>(w + o);
+  int* status = device_status_ptr();
+  const size_t slab = static_cast<size_t>(B) * H * Lcap * 128;   // one layer of one cache, elements
+  const float scale = 1.0f / sqrtf(128.0f);
+
+  embed_kernel<<<ntok, 256, 0, stream>>>(tree_tokens, static_cast<const uint16_t*>(m->embed), D, V, x, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("medusa_tree_decode: embedding launch", e);
+  for (int l = 0; l < m->layers; ++l) {
+    const medusa_decoder_layer_t& ly = m->layer[l];
+    uint16_t* kc = static_cast<uint16_t*>(k_cache) + static_cast<size_t>(l) * slab;
+    uint16_t* vc = static_cast<uint16_t*>(v_cache) + static_cast<size_t>(l) * slab;
+    rmsnorm_kernel<<<ntok, 256, 0, stream>>>(x, static_cast<const uint16_t*>(ly.attn_norm), D, xn);
+    GemmArgs g{};
+    g.ntok = ntok;
+    g.rows = 3 * D;
+    g.kdim = D;
+    g.q_out = qb;
+    g.k_cache = kc;
+    g.v_cache = vc;
+    g.seq_lens = seq_lens;
+    g.depth = t.depth;
+    g.T = t.T;
+    g.H = H;
+    g.Lcap = Lcap;
+    medusa_status_t st = gemm<kQKV>(ly.wqkv, xn, g, gws, stream);
+    if (st != MEDUSA_OK) return st;
+    st = launch_attention(t, 1, B, H, 128, MEDUSA_BF16, qb, kc, vc, Lcap, seq_lens, scale, att, nullptr, stream);
+    if (st != MEDUSA_OK) return st;
+    to_bf16_kernel<<<2 * sm_count(), 256, 0, stream>>>(att, static_cast<size_t>(ntok) * D, attb);
+    g = GemmArgs{};
+    g.ntok = ntok;
+    g.rows = D;
+    g.kdim = D;
+    g.x = x;
+    st = gemm<kResid>(ly.wo, attb, g, gws, stream);
+    if (st != MEDUSA_OK) return st;
+    rmsnorm_kernel<<<ntok, 256, 0, stream>>>(x, static_cast<const uint16_t*>(ly.mlp_norm), D, xn);
+    g = GemmArgs{};
+    g.ntok = ntok;
+    g.rows = 2 * F;
+    g.kdim = D;
+    g.act = act;
+    st = gemm<kSwiGLU>(ly.wgu, xn, g, gws, stream);
+    if (st != MEDUSA_OK) return st;
+    g = GemmArgs{};
+    g.ntok = ntok;
+    g.rows = D;
+    g.kdim = F;
+    g.x = x;
+    st = gemm<kResid>(ly.wdown, act, g, gws, stream);
+    if (st != MEDUSA_OK) return st;
+  }
+  if (hidden) {
+    e = cudaMemcpyAsync(hidden, x, static_cast<size_t>(ntok) * D * 4, cudaMemcpyDeviceToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail("medusa_tree_decode: hidden copy", e);
+  }
+  rmsnorm_kernel<<<ntok, 256, 0, stream>>>(x, static_cast<const uint16_t*>(m->final_norm), D, xn);
+  GemmArgs g{};
+  g.ntok = ntok;
+  g.rows = V;
+  g.kdim = D;
+  g.logits = logits;
+  medusa_status_t st = gemm<kLogits>(m->lm_head, xn, g, gws, stream);
+  if (st != MEDUSA_OK) return st;
+  e = cudaGetLastError();
+  return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_tree_decode: launch", e);
+}
+
+}  // namespace medusa

@@ -129,6 +129,12 @@ medusa_status_t launch_attention_rescale(int G, int rank, size_t rows, int hd, c
 medusa_status_t launch_topk_merge(const float* vals, const int32_t* ids, const int32_t* row0, int G, int B,
                                   int K, int topk, float* out_vals, int32_t* out_ids, cudaStream_t stream);
 
+// The tree-token forward of the base model (decoder.cu).
+size_t decoder_workspace_bytes(int ntok, int D, int F, int V);
+medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, int B, const int32_t* tree_tokens,
+                                   void* k_cache, void* v_cache, int Lcap, const int32_t* seq_lens,
+                                   float* logits, float* hidden, void* ws, cudaStream_t stream);
+
 // cuTensorMapEncodeTiled (PFN_cuTensorMapEncodeTiled_v12000), or null.
 void* tensor_map_encoder();
 

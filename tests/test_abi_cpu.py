@@ -105,3 +105,19 @@ def test_ranksum_rejects_too_many_nodes(mb):
         mb.medusa_tree_choices_ranksum(2, 2, 7)          # only 6 tuples exist
     with pytest.raises(mb.MedusaError):
         mb.medusa_tree_choices_ranksum(5, 10, 256)       # T would exceed 256
+
+
+def test_decoder_pack_rows(mb):
+    # q/k/v: within each head of 128 rows, row 2j holds feature j and row 2j+1 feature j + 64
+    rows = mb.medusa_decoder_pack_rows(0, 256)
+    assert sorted(rows) == list(range(256))
+    for r in range(256):
+        head, lr = divmod(r, 128)
+        assert rows[r] == head * 128 + (lr // 2 if lr % 2 == 0 else 64 + lr // 2)
+    # gate/up: row 2j is gate row j, row 2j+1 is up row j (index F + j of [W_gate; W_up])
+    F = 384
+    gu = mb.medusa_decoder_pack_rows(1, 2 * F)
+    assert sorted(gu) == list(range(2 * F))
+    assert gu[:4] == [0, F, 1, F + 1] and gu[-1] == 2 * F - 1
+    with pytest.raises(mb.MedusaError):
+        mb.medusa_decoder_pack_rows(0, 100)
