@@ -41,6 +41,8 @@ def parse():
     p.add_argument("--no-graph", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-decode", action="store_true",
+                   help="skip the timing of the base model's forward over the tree (tree_decoding)")
     p.add_argument("--shrink", default=None,
                    help="a smaller variant of the workload for profiling one kernel on a small case, "
                         "e.g. layers=1 (comma-separated field=value; the line's config names the variant)")
@@ -445,6 +447,11 @@ def run_ours(a, w):
         e_ms_max = reduce_max(statistics.mean(e_ms), world, "cuda")
         e2e = {"value": e_ms_max * 1e3, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    # ---- the base model's forward over the tree (tree_decoding) -------
+    decode = None
+    if not a.no_decode and w.dtype == "bf16" and w.hd == 128 and w.d // 128 == w.H and w.d in VICUNA_FFN:
+        decode = time_tree_decode(a, w, t, tree, mb, stream, peak, world)
+
     # ---- CPU baseline (rank 0, N = 1 only) -----------------------------
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -476,10 +483,92 @@ def run_ours(a, w):
                      "algorithmic_bytes_per_launch": head_bytes},
         "attention_roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
                                "frac": attn_gbs / peak, "algorithmic_bytes_per_launch": kv_bytes},
+        "tree_decode": decode,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * a.steps, "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# Feed-forward width of the Vicuna (LLaMA) base models by hidden size.
+VICUNA_FFN = {4096: 11008, 5120: 13824, 6656: 17920}
+
+
+def time_tree_decode(a, w, t, tree, mb, stream, peak, world):
+    """The base model's forward over the step's tree tokens (every layer of the workload's shape,
+    random bf16 weights from the counter-based generator), timed alone and inside a full
+    verification step (heads, tree, forward, posterior, compaction).  Overwrites the tree rows of
+    the caches, so it runs after every other measurement."""
+    import torch
+    from synth import device, gen
+    D, F, V, H = w.d, VICUNA_FFN[w.d], w.V, w.H
+    bf = torch.bfloat16
+
+    def rnd(shape, tid, sigma):
+        x = torch.empty(shape, dtype=bf, device="cuda")
+        device.fill_normal(x, w.seed, tid, sigma)
+        return x
+
+    s = D ** -0.5
+    layers = []
+    for l in range(w.layers):
+        tid = gen.TID_DECODER + 9 * l
+        layers.append({"attn_norm": rnd((D,), tid, 0.1) + 1.0, "Wq": rnd((D, D), tid + 1, s),
+                       "Wk": rnd((D, D), tid + 2, s), "Wv": rnd((D, D), tid + 3, s), "Wo": rnd((D, D), tid + 4, s),
+                       "mlp_norm": rnd((D,), tid + 5, 0.1) + 1.0, "W_gate": rnd((F, D), tid + 6, s),
+                       "W_up": rnd((F, D), tid + 7, s), "W_down": rnd((D, F), tid + 8, F ** -0.5)})
+    tid = gen.TID_DECODER + 9 * w.layers
+    model = mb.Decoder(rnd((V, D), tid, 1.0), layers, rnd((D,), tid + 1, 0.1) + 1.0, rnd((V, D), tid + 2, s))
+    del layers
+    torch.cuda.synchronize()
+    ntok = w.B * w.T
+    logits = torch.empty((ntok, V), device="cuda")
+    ws = mb.workspace(mb.medusa_tree_decode_workspace_size(tree, model, w.B))
+    lens = t["seq_lens0"]
+
+    def fwd():
+        mb.medusa_tree_decode(tree, model, t["tree_tokens"], t["k_cache"], t["v_cache"], lens, logits, ws)
+
+    def full_step():
+        # the whole verification step with the base model's forward producing the base logits
+        t["seq_lens"].copy_(lens)
+        hws = t["_hws"]
+        mb.medusa_heads_topk(t["h"], t["W1"], t["b1"], t["Wout"], w.topk, t["topk_ids"], t["topk_vals"], hws)
+        mb.medusa_build_tree(tree, t["root_tokens"], t["topk_ids"], t["seq_lens"], t["tree_tokens"],
+                             t["candidates"], t["position_ids"])
+        mb.medusa_tree_decode(tree, model, t["tree_tokens"], t["k_cache"], t["v_cache"], t["seq_lens"], logits, ws)
+        mb.medusa_evaluate_posterior(tree, logits.view(w.B, w.T, V), t["candidates"], mb.MEDUSA_GREEDY, t["best_path"],
+                                     t["accept_len"], t["accepted_tokens"], t["next_token"], t["_pws"])
+        mb.medusa_accept_kv(tree, t["k_cache"], t["v_cache"], t["seq_lens"], t["best_path"], t["accept_len"])
+
+    t["_hws"] = mb.workspace(mb.medusa_heads_workspace_size(w.B, w.d, w.V, w.K, w.topk))
+    t["_pws"] = mb.workspace(mb.medusa_posterior_workspace_size(tree, w.B))
+    res = {}
+    with torch.cuda.stream(stream):
+        for name, fn in (("forward", fwd), ("full_step", full_step)):
+            for _ in range(max(3, a.warmup)):
+                fn()
+            torch.cuda.synchronize()
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(a.steps + 1)]
+            evs[0].record(stream)
+            for i in range(a.steps):
+                fn()
+                evs[i + 1].record(stream)
+            torch.cuda.synchronize()
+            xs = sorted(evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(a.steps))
+            res[name] = {"median": statistics.median(xs), "min": xs[0], "p90": xs[min(a.steps - 1, int(0.9 * (a.steps - 1)))]}
+    st, det = mb.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} detail {det} after the tree-decode timing")
+    wbytes = sum(x.numel() * 2 for ly in model.tensors for x in ly.values()) + model.lm_head.numel() * 2
+    kv_bytes = 2 * w.layers * w.H * w.hd * int((w.prefix_lens() + w.T).sum()) * 2
+    fwd_us = res["forward"]["median"]
+    return {"layers": w.layers, "D": D, "F": F, "V": V, "tokens": ntok, "weights_bytes": wbytes, "kv_bytes": kv_bytes,
+            "forward_us": res["forward"], "full_step_us": res["full_step"],
+            "forward_gbs": (wbytes + kv_bytes) / (fwd_us * 1e-6) / 1e9,
+            "forward_frac": (wbytes + kv_bytes) / (fwd_us * 1e-6) / 1e9 / peak,
+            "note": "random bf16 weights of the base model's shape; the full step's acceptance is meaningless "
+                    "with random weights, so tokens per step are not reported"}
 
 
 def kernel_revision():

@@ -375,7 +375,7 @@ medusa_status_t medusa_accept_kv(const medusa_tree_t* tree, int layers, int B, i
 /* ------------------------------------------------------------------------ */
 
 /* One LLaMA (Vicuna) decoder layer's weights, bf16 device pointers, hd = 128
- * (H = D / 128 heads), F the feed-forward width (multiples of 128):
+ * (H = D / 128 heads, D <= 8192), F the feed-forward width (multiples of 128):
  *   attn_norm, mlp_norm [D]   RMSNorm weights (eps 1e-6)
  *   wqkv  [3D, D]  the rows of Wq, Wk and Wv (out x in) in that order, each
  *                  head's 128 rows packed so that row 2j is feature j and row

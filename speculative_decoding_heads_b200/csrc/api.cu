@@ -365,8 +365,8 @@ static medusa_status_t check_decoder(const medusa_tree_t* tree, const medusa_dec
   if (st != MEDUSA_OK) return st;
   if (!m || !m->layer || !m->embed || !m->final_norm || !m->lm_head)
     return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null model pointer");
-  if (m->layers < 1 || m->D < 128 || m->D % 128 != 0 || m->F < 128 || m->F % 128 != 0 || m->V < 1 || B < 1 ||
-      B > MEDUSA_MAX_B)
+  if (m->layers < 1 || m->D < 128 || m->D % 128 != 0 || m->D > 8192 || m->F < 128 || m->F % 128 != 0 || m->V < 1 ||
+      B < 1 || B > MEDUSA_MAX_B)
     return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": layers, D, F, V or B out of range");
   if (static_cast<long long>(B) * tree->T > (1 << 20))
     return fail(MEDUSA_ERR_UNSUPPORTED, std::string(fn) + ": too many tree tokens");
@@ -374,10 +374,12 @@ static medusa_status_t check_decoder(const medusa_tree_t* tree, const medusa_dec
     const medusa_decoder_layer_t& y = m->layer[l];
     if (!y.attn_norm || !y.wqkv || !y.wo || !y.mlp_norm || !y.wgu || !y.wdown)
       return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": null layer pointer");
-    if (!aligned16(y.wqkv) || !aligned16(y.wo) || !aligned16(y.wgu) || !aligned16(y.wdown))
+    if (!aligned16(y.wqkv) || !aligned16(y.wo) || !aligned16(y.wgu) || !aligned16(y.wdown) ||
+        !aligned16(y.attn_norm) || !aligned16(y.mlp_norm))
       return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": misaligned weights");
   }
-  if (!aligned16(m->embed) || !aligned16(m->lm_head)) return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": misaligned");
+  if (!aligned16(m->embed) || !aligned16(m->lm_head) || !aligned16(m->final_norm))
+    return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": misaligned");
   return MEDUSA_OK;
 }
 

@@ -78,6 +78,10 @@ struct Bars {
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
+  // QKV: for each token c of the pass, its rotary position and its cache row
+  // offset ((b H) Lcap + L + node) 128 (-1: no valid cache row)
+  int pos[kN];
+  long long crow[kN];
 };
 
 __device__ __forceinline__ int stage_lo(int c, const GemmArgs& a) {
@@ -113,64 +117,71 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ba
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
 __device__ __forceinline__ float bf(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
 
-// The epilogue of one finished tile row (all 64 token columns in acc).
+// The epilogue of one finished tile row, for the 32 token columns c0 ..
+// c0 + 31 (in acc).  Every global load comes before the stores, so the loads
+// of the 32 tokens overlap.
+constexpr int kHalf = 32;
 template <int kMode>
-__device__ __forceinline__ void epilogue_row(const GemmArgs& a, int tile, int r, int lane, const float (&acc)[kN]) {
+__device__ __forceinline__ void epilogue_half(const GemmArgs& a, const Bars* bs, int tile, int r, int c0,
+                                              const float (&acc)[kHalf]) {
   const int nvalid = a.ntok - a.tok0 < kN ? a.ntok - a.tok0 : kN;
   if constexpr (kMode == kQKV) {
     const int which = tile / a.H, h = tile - which * a.H;   // 0 q, 1 k, 2 v; head h
     const int j = r >> 1;                                   // pair index (frequency)
     const int feat = j + (r & 1) * 64;                      // feature within the head
-    // rotation frequency base^(-2j/128), angle reduced in double
-    const double inv = exp2(-static_cast<double>(2 * j) / 128.0 * 13.287712379549449);   // log2(10000)
-    for (int c = 0; c < kN; ++c) {
-      const float own = acc[c];
+    // rotation frequency base^(-2j/128) with base 10000, angle reduced in double
+    const double inv = exp2(-static_cast<double>(2 * j) / 128.0 * 13.287712379549449);
+    uint16_t* cache = which == 1 ? a.k_cache : a.v_cache;
+#pragma unroll 4
+    for (int i = 0; i < kHalf; ++i) {
+      const int c = c0 + i;
+      const float own = acc[i];
       const float other = __shfl_xor_sync(0xffffffffu, own, 1);
-      if (c >= nvalid) continue;
-      const int n = a.tok0 + c;
-      const int b = n / a.T, node = n - b * a.T;
-      const int L = a.seq_lens[b];
-      if (L < 0 || L + a.T > a.Lcap) {   // the tree's rows would not fit in the cache
-        set_device_status(a.status, MEDUSA_ERR_DEVICE_CHECK, kDetailDecoderSeqLen);
-        continue;
-      }
+      const long long row = bs->crow[c];
+      if (c >= nvalid || row < 0) continue;
       float out = own;
       if (which < 2) {
-        const double ang = static_cast<double>(L + a.depth[node]) * inv;
-        const double red = ang - 6.283185307179586 * rint(ang / 6.283185307179586);
+        const double ang = static_cast<double>(bs->pos[c]) * inv;
+        const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
         float sn, cs;
         sincosf(static_cast<float>(red), &sn, &cs);
         out = (r & 1) ? other * sn + own * cs : own * cs - other * sn;
       }
       const uint16_t v = f32_to_bf16_rne(out);
       if (which == 0) {
-        a.q_out[(static_cast<size_t>(n) * a.H + h) * 128 + feat] = v;
+        a.q_out[(static_cast<size_t>(a.tok0 + c) * a.H + h) * 128 + feat] = v;
       } else {
-        uint16_t* cache = which == 1 ? a.k_cache : a.v_cache;
-        cache[((static_cast<size_t>(b) * a.H + h) * a.Lcap + L + node) * 128 + feat] = v;
+        cache[row + static_cast<long long>(h) * a.Lcap * 128 + feat] = v;
       }
     }
   } else if constexpr (kMode == kSwiGLU) {
     const int j = tile * 64 + (r >> 1);   // output feature
-    for (int c = 0; c < kN; ++c) {
-      const float own = acc[c];
+    const bool writer = !(r & 1) && 2 * j < a.rows;
+    uint16_t* dst = a.act + static_cast<size_t>(a.tok0 + c0) * (a.rows / 2) + j;
+#pragma unroll
+    for (int i = 0; i < kHalf; ++i) {
+      const float own = acc[i];
       const float up = __shfl_xor_sync(0xffffffffu, own, 1);
-      if (c >= nvalid || (r & 1) || 2 * j >= a.rows) continue;
-      a.act[static_cast<size_t>(a.tok0 + c) * (a.rows / 2) + j] = f32_to_bf16_rne(silu(own) * up);
+      if (c0 + i < nvalid && writer) dst[static_cast<size_t>(i) * (a.rows / 2)] = f32_to_bf16_rne(silu(own) * up);
     }
+  } else if constexpr (kMode == kResid) {
+    const int f = tile * kTileRows + r;
+    if (f >= a.rows) return;
+    float* xr = a.x + static_cast<size_t>(a.tok0 + c0) * a.rows + f;
+    float old[kHalf];
+#pragma unroll
+    for (int i = 0; i < kHalf; ++i) old[i] = c0 + i < nvalid ? xr[static_cast<size_t>(i) * a.rows] : 0.f;
+#pragma unroll
+    for (int i = 0; i < kHalf; ++i)
+      if (c0 + i < nvalid) xr[static_cast<size_t>(i) * a.rows] = old[i] + acc[i];
   } else {
     const int f = tile * kTileRows + r;
     if (f >= a.rows) return;
-    for (int c = 0; c < nvalid; ++c) {
-      const size_t o = static_cast<size_t>(a.tok0 + c) * a.rows + f;
-      if constexpr (kMode == kResid) {
-        a.x[o] += acc[c];
-      } else {
-        a.logits[o] = acc[c];
-      }
-    }
+    float* lr = a.logits + static_cast<size_t>(a.tok0 + c0) * a.rows + f;
+#pragma unroll
+    for (int i = 0; i < kHalf; ++i)
+      if (c0 + i < nvalid) lr[static_cast<size_t>(i) * a.rows] = acc[i];
   }
-  (void)lane;
 }
 
 template <int kMode>
@@ -202,28 +213,69 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tmem_alloc(&bs->tmem_base, kTmemCols);
     tc::tmem_relinquish();
   }
+  if constexpr (kMode == kQKV) {
+    for (int c = tid; c < kN; c += kThreads) {
+      const int n = a.tok0 + c;
+      int p = 0;
+      long long row = -1;
+      if (n < a.ntok) {
+        const int b = n / a.T, node = n - b * a.T;
+        const int L = a.seq_lens[b];
+        if (L < 0 || L + a.T > a.Lcap) {   // the tree's rows would not fit in the cache
+          set_device_status(a.status, MEDUSA_ERR_DEVICE_CHECK, kDetailDecoderSeqLen);
+        } else {
+          p = L + a.depth[node];
+          row = (static_cast<long long>(b) * a.H * a.Lcap + L + node) * 128;
+        }
+      }
+      bs->pos[c] = p;
+      bs->crow[c] = row;
+    }
+  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = bs->tmem_base;
+  allow_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
       tc::prefetch_tensormap(&w_map);
       tc::prefetch_tensormap(&x_map);
       const uint64_t pol = l2_evict_first_policy();
+      // The weights do not depend on the previous kernel: the first stages'
+      // weight tiles load before waiting for it, their activations after.
+      bool x_ready = false;
+      int pend_slot[kNS], pend_k[kNS];
+      int npend = 0;
+      auto flush = [&]() {
+        wait_prior_grids();
+        for (int i = 0; i < npend; ++i)
+          tc::tma_load_4d(smem + pend_slot[i] * kSB + kKPS * kWBlock, &x_map, 0, a.tok0, pend_k[i], 0,
+                          &bs->full[pend_slot[i]]);
+        npend = 0;
+        x_ready = true;
+      };
       int g = 0;
       Unit x;
       for (int st = st_lo; !bs->abort && next_unit(a, st, st_hi, x);) {
         for (int j = x.k0; j < x.k1; j += kKPS, ++g) {
           const int slot = g % kNS;
+          if (!x_ready && npend == kNS) flush();
           if (g >= kNS && !wait_or_abort(&bs->empty[slot], ((g / kNS) - 1) & 1, bs, a.status)) break;
           mbar_arrive_expect_tx(&bs->full[slot], kSB);
           unsigned char* sd = smem + slot * kSB;
           tc::tma_load_4d_hint(sd, &w_map, 0, x.tile * kTileRows, j, 0, &bs->full[slot], pol);
-          tc::tma_load_4d(sd + kKPS * kWBlock, &x_map, 0, a.tok0, j, 0, &bs->full[slot]);
+          if (x_ready) {
+            tc::tma_load_4d(sd + kKPS * kWBlock, &x_map, 0, a.tok0, j, 0, &bs->full[slot]);
+          } else {
+            pend_slot[npend] = slot;
+            pend_k[npend] = j;
+            ++npend;
+          }
         }
       }
+      if (!x_ready) flush();
       for (int t = g - kNS < 0 ? 0 : g - kNS; t < g; ++t) mbar_wait(&bs->full[t % kNS], (t / kNS) & 1);
     }
   } else if (warp == 1) {
@@ -266,28 +318,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
     const int r = 32 * q + lane;
+    wait_prior_grids();   // the residual stream and the outputs of the kernels before
     int n = 0;
     Unit x;
     for (int st = st_lo; next_unit(a, st, st_hi, x); ++n) {
       const int buf = n & 1;
       if (!wait_or_abort(&bs->acc_full[buf], (n >> 1) & 1, bs, a.status)) break;
       tc::fence_after_sync();
-      float acc[kN];
-      tc::tmem_ld32(tmem + lane_off + buf * kN, acc);
-      tc::tmem_ld32(tmem + lane_off + buf * kN + 32, acc + 32);
-      tc::tmem_wait_ld();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&bs->acc_empty[buf]);
+      const uint32_t tacc = tmem + lane_off + buf * kN;
       const int t0 = x.tile * a.nst;
       const int c_first = stage_owner(t0, a), c_last = stage_owner(t0 + a.nst - 1, a);
-      if (c_first != c_last) {
-        // A tile shared with other CTAs: the last to finish sums the partials in CTA order.
+      const bool split = c_first != c_last;
+      bool mine_last = true;
+      if (split) {
+        // A tile shared with other CTAs: store this part; the last to finish
+        // sums the parts in CTA order.
         const int slot = x.tile == st_lo / a.nst ? 0 : 1;
         float* mine = a.part + ((static_cast<size_t>(cta) * 2 + slot) * kTileRows + r) * kN;
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          float acc[kHalf];
+          tc::tmem_ld32(tacc + hh * kHalf, acc);
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kN; c += 4)
-          *reinterpret_cast<float4*>(mine + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+          for (int c = 0; c < kHalf; c += 4)
+            *reinterpret_cast<float4*>(mine + hh * kHalf + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+        }
         __threadfence();
         __syncwarp();
         int last = 0;
@@ -296,29 +352,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           last = atom_add_acq_rel_gpu(cnt, 1u) == static_cast<unsigned>(c_last - c_first);
           if (last) *cnt = 0u;
         }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (!last) continue;
-        __threadfence();
-        float sum[kN];
-#pragma unroll
-        for (int c = 0; c < kN; ++c) sum[c] = 0.f;
-        for (int cc = c_first; cc <= c_last; ++cc) {
-          const int sl = x.tile == stage_lo(cc, a) / a.nst ? 0 : 1;
-          const float* pc = a.part + ((static_cast<size_t>(cc) * 2 + sl) * kTileRows + r) * kN;
-#pragma unroll
-          for (int c = 0; c < kN; c += 4) {
-            const float4 v = cc == cta ? make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3])
-                                       : __ldcg(reinterpret_cast<const float4*>(pc + c));
-            sum[c] += v.x;
-            sum[c + 1] += v.y;
-            sum[c + 2] += v.z;
-            sum[c + 3] += v.w;
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < kN; ++c) acc[c] = sum[c];
+        mine_last = __shfl_sync(0xffffffffu, last, 0) != 0;
+        if (mine_last) __threadfence();
       }
-      epilogue_row<kMode>(a, x.tile, r, lane, acc);
+      if (mine_last) {
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          float acc[kHalf];
+          tc::tmem_ld32(tacc + hh * kHalf, acc);
+          tc::tmem_wait_ld();
+          if (split) {
+            float sum[kHalf];
+#pragma unroll
+            for (int c = 0; c < kHalf; ++c) sum[c] = 0.f;
+            for (int cc = c_first; cc <= c_last; ++cc) {
+              const int sl = x.tile == stage_lo(cc, a) / a.nst ? 0 : 1;
+              const float* pc = a.part + ((static_cast<size_t>(cc) * 2 + sl) * kTileRows + r) * kN + hh * kHalf;
+#pragma unroll
+              for (int c = 0; c < kHalf; c += 4) {
+                const float4 v = cc == cta ? make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3])
+                                           : __ldcg(reinterpret_cast<const float4*>(pc + c));
+                sum[c] += v.x;
+                sum[c + 1] += v.y;
+                sum[c + 2] += v.z;
+                sum[c + 3] += v.w;
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < kHalf; ++c) acc[c] = sum[c];
+          }
+          epilogue_half<kMode>(a, bs, x.tile, r, hh * kHalf, acc);
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bs->acc_empty[buf]);
     }
   }
   tc::fence_before_sync();
@@ -333,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // x[n] = embed[tokens[n]] (bf16 -> fp32), n over the B*T tree tokens.
 __global__ void embed_kernel(const int32_t* tokens, const uint16_t* embed, int D, int V, float* x, int* status) {
+  allow_dependents();
   const int n = blockIdx.x;
   const int tok = tokens[n];
   if (tok < 0 || tok >= V) {
@@ -344,30 +413,55 @@ __global__ void embed_kernel(const int32_t* tokens, const uint16_t* embed, int D
     x[static_cast<size_t>(n) * D + i] = bf(embed[static_cast<size_t>(tok) * D + i]);
 }
 
-// y[n] = bf16(x[n] / sqrt(mean(x[n]^2) + eps) * w), one CTA per token.
-__global__ void rmsnorm_kernel(const float* x, const uint16_t* w, int D, uint16_t* y) {
-  __shared__ float red[32];
-  const int n = blockIdx.x;
-  const float* xr = x + static_cast<size_t>(n) * D;
+// y[n] = bf16(x[n] / sqrt(mean(x[n]^2) + eps) * w), one CTA per token: the
+// row is loaded once (16-byte loads, kept in registers), reduced, scaled.
+constexpr int kNormThreads = 256;
+constexpr int kNormVec = 8;   // float4 per thread: rows of up to 8192 values
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* x, const uint16_t* w, int D, uint16_t* y) {
+  __shared__ float red[kNormThreads / 32];
+  wait_prior_grids();
+  allow_dependents();
+  const int n = blockIdx.x, tid = threadIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(n) * D);
+  const int nv = D / 4;
+  float4 v[kNormVec];
   float s = 0.f;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) s = fmaf(xr[i], xr[i], s);
+#pragma unroll
+  for (int i = 0; i < kNormVec; ++i) {
+    const int k = tid + i * kNormThreads;
+    v[i] = k < nv ? xr[k] : make_float4(0.f, 0.f, 0.f, 0.f);
+    s = fmaf(v[i].x, v[i].x, fmaf(v[i].y, v[i].y, fmaf(v[i].z, v[i].z, fmaf(v[i].w, v[i].w, s))));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  if ((tid & 31) == 0) red[tid >> 5] = s;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    float t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+  float t = 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    if (threadIdx.x == 0) red[0] = t;
+  for (int i = 0; i < kNormThreads / 32; ++i) t += red[i];
+  const float inv = rsqrtf(t / static_cast<float>(D) + kRmsEps);
+  uint2* yr = reinterpret_cast<uint2*>(y + static_cast<size_t>(n) * D);
+  const uint2* wr = reinterpret_cast<const uint2*>(w);
+#pragma unroll
+  for (int i = 0; i < kNormVec; ++i) {
+    const int k = tid + i * kNormThreads;
+    if (k < nv) {
+      const uint2 ww = wr[k];
+      const float w0 = __uint_as_float(ww.x << 16), w1 = __uint_as_float(ww.x & 0xffff0000u);
+      const float w2 = __uint_as_float(ww.y << 16), w3 = __uint_as_float(ww.y & 0xffff0000u);
+      uint2 o;
+      o.x = static_cast<uint32_t>(f32_to_bf16_rne(v[i].x * inv * w0)) |
+            (static_cast<uint32_t>(f32_to_bf16_rne(v[i].y * inv * w1)) << 16);
+      o.y = static_cast<uint32_t>(f32_to_bf16_rne(v[i].z * inv * w2)) |
+            (static_cast<uint32_t>(f32_to_bf16_rne(v[i].w * inv * w3)) << 16);
+      yr[k] = o;
+    }
   }
-  __syncthreads();
-  const float inv = rsqrtf(red[0] / static_cast<float>(D) + kRmsEps);
-  for (int i = threadIdx.x; i < D; i += blockDim.x)
-    y[static_cast<size_t>(n) * D + i] = f32_to_bf16_rne(xr[i] * inv * bf(w[i]));
 }
 
 __global__ void to_bf16_kernel(const float* x, size_t n, uint16_t* y) {
+  wait_prior_grids();
+  allow_dependents();
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
     y[i] = f32_to_bf16_rne(x[i]);
@@ -413,7 +507,7 @@ medusa_status_t gemm(const void* Wt, const uint16_t* X, GemmArgs a, void* ws, cu
   auto fn = wgemm_kernel<kMode>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   for (a.tok0 = 0; e == cudaSuccess && a.tok0 < a.ntok; a.tok0 += kN)
-    e = launch_kernel(fn, dim3(a.G), dim3(kThreads), static_cast<size_t>(kSmem), stream, false, wm, xm, a);
+    e = launch_kernel(fn, dim3(a.G), dim3(kThreads), static_cast<size_t>(kSmem), stream, true, wm, xm, a);
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_tree_decode: matrix-product launch", e);
 }
 
@@ -461,7 +555,9 @@ medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, 
     const medusa_decoder_layer_t& ly = m->layer[l];
     uint16_t* kc = static_cast<uint16_t*>(k_cache) + static_cast<size_t>(l) * slab;
     uint16_t* vc = static_cast<uint16_t*>(v_cache) + static_cast<size_t>(l) * slab;
-    rmsnorm_kernel<<<ntok, 256, 0, stream>>>(x, static_cast<const uint16_t*>(ly.attn_norm), D, xn);
+    e = launch_kernel(rmsnorm_kernel, dim3(ntok), dim3(kNormThreads), 0, stream, true, static_cast<const float*>(x),
+                      static_cast<const uint16_t*>(ly.attn_norm), D, xn);
+    if (e != cudaSuccess) return cuda_fail("medusa_tree_decode: RMSNorm launch", e);
     GemmArgs g{};
     g.ntok = ntok;
     g.rows = 3 * D;
@@ -478,7 +574,9 @@ medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, 
     if (st != MEDUSA_OK) return st;
     st = launch_attention(t, 1, B, H, 128, MEDUSA_BF16, qb, kc, vc, Lcap, seq_lens, scale, att, nullptr, stream);
     if (st != MEDUSA_OK) return st;
-    to_bf16_kernel<<<2 * sm_count(), 256, 0, stream>>>(att, static_cast<size_t>(ntok) * D, attb);
+    e = launch_kernel(to_bf16_kernel, dim3(2 * sm_count()), dim3(256), 0, stream, true, static_cast<const float*>(att),
+                      static_cast<size_t>(ntok) * D, attb);
+    if (e != cudaSuccess) return cuda_fail("medusa_tree_decode: conversion launch", e);
     g = GemmArgs{};
     g.ntok = ntok;
     g.rows = D;
@@ -486,7 +584,9 @@ medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, 
     g.x = x;
     st = gemm<kResid>(ly.wo, attb, g, gws, stream);
     if (st != MEDUSA_OK) return st;
-    rmsnorm_kernel<<<ntok, 256, 0, stream>>>(x, static_cast<const uint16_t*>(ly.mlp_norm), D, xn);
+    e = launch_kernel(rmsnorm_kernel, dim3(ntok), dim3(kNormThreads), 0, stream, true, static_cast<const float*>(x),
+                      static_cast<const uint16_t*>(ly.mlp_norm), D, xn);
+    if (e != cudaSuccess) return cuda_fail("medusa_tree_decode: RMSNorm launch", e);
     g = GemmArgs{};
     g.ntok = ntok;
     g.rows = 2 * F;
@@ -506,7 +606,9 @@ medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, 
     e = cudaMemcpyAsync(hidden, x, static_cast<size_t>(ntok) * D * 4, cudaMemcpyDeviceToDevice, stream);
     if (e != cudaSuccess) return cuda_fail("medusa_tree_decode: hidden copy", e);
   }
-  rmsnorm_kernel<<<ntok, 256, 0, stream>>>(x, static_cast<const uint16_t*>(m->final_norm), D, xn);
+  e = launch_kernel(rmsnorm_kernel, dim3(ntok), dim3(kNormThreads), 0, stream, true, static_cast<const float*>(x),
+                    static_cast<const uint16_t*>(m->final_norm), D, xn);
+  if (e != cudaSuccess) return cuda_fail("medusa_tree_decode: RMSNorm launch", e);
   GemmArgs g{};
   g.ntok = ntok;
   g.rows = V;

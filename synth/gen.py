@@ -65,6 +65,7 @@ TID_ROOT = 9
 TID_PLANT = 10
 TID_SEQLEN = 11
 TID_UNIFORM = 12          # one draw per sequence for the sampled next token
+TID_DECODER = 1 << 20     # base-model weights: TID_DECODER + 9 * layer + matrix index; embed, final norm, LM head after
 SUBSEED_STRIDE = 64
 
 _CHUNK = 1 << 22
