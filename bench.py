@@ -218,6 +218,77 @@ class OracleSample:
         return t_full + t_sample * self.scale_slices
 
 
+def expected_launches(w, T):
+    """Kernel launches of one medusa_step by the library's launch plan: the heads
+    (one launch per group of <= 4 sequences on the CUDA cores at batch 1 or
+    fp32, two per pass of <= 16 sequences on the tensor cores), tree attention
+    (one launch, two when a tree above 64 tokens leaves 1-64 rows after its
+    128-row groups) and the posterior with the compaction (one)."""
+    if w.dtype == "bf16" and w.B >= 2 and w.d % 128 == 0:
+        heads = 2 * ((w.B + 15) // 16)
+    else:
+        heads = (w.B + 3) // 4
+    attn = 1
+    if w.dtype == "bf16" and w.hd == 128 and T > 64 and 0 < T % 128 <= 64:
+        attn = 2
+    return heads + attn + 1
+
+
+def _kernel_short_name(mangled):
+    """The innermost identifier of an Itanium-mangled kernel name (the kernel's own name)."""
+    if not mangled.startswith("_Z"):
+        return mangled
+    i, last = 2, mangled
+    if i < len(mangled) and mangled[i] == "N":
+        i += 1
+    while i < len(mangled) and mangled[i].isdigit():
+        j = i
+        while j < len(mangled) and mangled[j].isdigit():
+            j += 1
+        n = int(mangled[i:j])
+        last = mangled[j:j + n]
+        i = j + n
+    return last
+
+
+def graph_kernels(g):
+    """Names of the kernel nodes of a captured CUDA graph (kept with keep_graph=True), in
+    node order; None when the driver API cannot be queried."""
+    try:
+        from cuda.bindings import driver as drv
+        graph = drv.CUgraph(int(g.raw_cuda_graph()))
+        err, _, n = drv.cuGraphGetNodes(graph, 0)
+        if err != drv.CUresult.CUDA_SUCCESS:
+            return None
+        err, nodes, n = drv.cuGraphGetNodes(graph, n)
+        if err != drv.CUresult.CUDA_SUCCESS:
+            return None
+        names = []
+        for node in nodes:
+            err, ty = drv.cuGraphNodeGetType(node)
+            if err != drv.CUresult.CUDA_SUCCESS:
+                return None
+            if ty != drv.CUgraphNodeType.CU_GRAPH_NODE_TYPE_KERNEL:
+                continue
+            name = "?"
+            try:
+                err, p = drv.cuGraphKernelNodeGetParams(node)
+                if err == drv.CUresult.CUDA_SUCCESS:
+                    if int(p.func):
+                        err, nm = drv.cuFuncGetName(p.func)
+                    else:
+                        err, nm = drv.cuKernelGetName(p.kern)
+                    if err == drv.CUresult.CUDA_SUCCESS:
+                        name = _kernel_short_name(nm.decode() if isinstance(nm, bytes) else str(nm))
+            except Exception:
+                pass
+            names.append(name)
+        return names
+    except Exception as ex:
+        print(f"# graph node query failed: {ex}", file=sys.stderr)
+        return None
+
+
 def reduce_max(x, world, device):
     """The largest of a per-rank scalar over all ranks (every rank receives it)."""
     if world <= 1:
@@ -302,8 +373,8 @@ def run_ours(a, w):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
-    # heads (+ tree build) per group of <= 4 sequences, attention, posterior with the KV compaction
-    launches_per_step = (w.B + 3) // 4 + 1 + 1
+    launches_per_step = expected_launches(w, tree.T)
+    kernels = None
 
     def step():
         t["seq_lens"].copy_(t["seq_lens0"])
@@ -320,10 +391,14 @@ def run_ours(a, w):
     graph = None
     if not a.no_graph:
         try:
-            g = torch.cuda.CUDAGraph()
+            g = torch.cuda.CUDAGraph(keep_graph=True)
             with torch.cuda.graph(g, stream=stream):
                 step()
+            g.instantiate()
             graph = g
+            kernels = graph_kernels(g)
+            if kernels is not None:
+                launches_per_step = len(kernels)
             with torch.cuda.stream(stream):
                 for _ in range(a.warmup):
                     graph.replay()
@@ -358,22 +433,31 @@ def run_ours(a, w):
         raise RuntimeError(f"device status {st} detail {det} after the timed region")
 
     # ---- per-step distribution, graph replay and eager launches side by side ----
-    def per_step(fn, k):
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(k + 1)]
+    def per_step_pair(fns, k):
+        # The launch forms alternate step by step, so clock and power drift
+        # over the run affects both alike.
+        evs = {n: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+               for n in fns}
         with torch.cuda.stream(stream):
-            evs[0].record(stream)
             for i in range(k):
-                fn()
-                evs[i + 1].record(stream)
+                for n, fn in fns.items():
+                    evs[n][i][0].record(stream)
+                    fn()
+                    evs[n][i][1].record(stream)
         torch.cuda.synchronize()
-        xs = sorted(evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(k))
-        return {"mean": statistics.mean(xs), "median": statistics.median(xs), "min": xs[0],
-                "p90": xs[min(k - 1, int(round(0.9 * (k - 1))))], "n": k}
+        out = {}
+        for n in fns:
+            xs = sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in evs[n])
+            out[n] = {"mean": statistics.mean(xs), "median": statistics.median(xs), "min": xs[0],
+                      "p90": xs[min(k - 1, int(round(0.9 * (k - 1))))], "n": k}
+        return out
 
     dist_steps = max(a.steps, 20)
-    step_us = {"eager": per_step(step, dist_steps)}
+    forms = {"eager": step}
     if graph is not None:
-        step_us["graph"] = per_step(graph.replay, dist_steps)
+        forms["graph"] = graph.replay
+    step_us = per_step_pair(forms, dist_steps)
+    step_us["note"] = "graph and eager steps alternate"
 
     # ---- per-stage breakdown (eager, CUDA events on the launching stream) ----
     peak, peak_kind = load_peaks()
@@ -420,6 +504,15 @@ def run_ours(a, w):
         if tj.get("workload") == w.name and tj.get("kernel_rev") == kernel_revision():
             traffic = tj.get("dram_bytes_per_launch")
 
+    peak_desc = (f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                 else "fallback 6650 GB/s")
+    heads_line = {"bound": "hbm", "kernel": "heads_topk", "achieved": heads_gbs, "peak": peak, "peak_kind": peak_desc,
+                  "unit": "GB/s", "frac": heads_gbs / peak, "traffic": traffic,
+                  "algorithmic_bytes_per_launch": head_bytes}
+    attn_line = {"bound": "hbm", "kernel": "tree_attention", "achieved": attn_gbs, "peak": peak,
+                 "peak_kind": peak_desc, "unit": "GB/s", "frac": attn_gbs / peak, "traffic": None,
+                 "algorithmic_bytes_per_launch": kv_bytes}
+
     # ---- end to end through the public API with host buffers ----------
     e2e = None
     if not a.no_e2e:
@@ -431,15 +524,14 @@ def run_ours(a, w):
         vt = torch.stack([t["v_cache"][:, b, :, int(lens[b]):int(lens[b]) + w.T] for b in range(w.B)], 1)
         host_in["k_tree"], host_in["v_tree"] = pin(kt), pin(vt)
         host_out = {k: torch.empty_like(t[k], device="cpu").pin_memory()
-                    for k in ("best_path", "accept_len", "accepted_tokens", "next_token")}
-        dev_map = dict(t)
+                    for k in ("best_path", "accept_len", "accepted_tokens", "next_token", "seq_lens")}
         h2d = sum(x.numel() * x.element_size() for x in host_in.values())
         d2h = sum(x.numel() * x.element_size() for x in host_out.values())
         e_ms = []
         for i in range(a.warmup + a.steps):
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s0.record(stream)
-            mb.medusa_step_from_host(args, ws, host_in, dev_map, host_out, stream)
+            mb.medusa_step_host(args, ws, host_in, host_out, stream)
             s1.record(stream)
             s1.synchronize()
             if i >= a.warmup:
@@ -477,14 +569,16 @@ def run_ours(a, w):
         "tree_tokens_per_s": world * w.B * w.T / (us * 1e-6),
         "stage_us": stage,
         "step_us": step_us,
-        "roofline": {"bound": "hbm", "kernel": "heads_topk", "achieved": heads_gbs, "peak": peak,
-                     "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                     else "fallback 6650 GB/s", "unit": "GB/s", "frac": heads_gbs / peak, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": head_bytes},
-        "attention_roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
-                               "frac": attn_gbs / peak, "algorithmic_bytes_per_launch": kv_bytes},
+        # `roofline` is the dominant kernel's (the larger per-call stage time).
+        "roofline": heads_line if stage["heads_topk"] >= stage["tree_attention"] else attn_line,
+        "heads_roofline": heads_line,
+        "attention_roofline": attn_line,
         "tree_decode": decode,
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * a.steps, "clocks": clocks,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * a.steps,
+        "launches_per_step": {"count": launches_per_step,
+                              "source": "kernel nodes of the captured step graph" if kernels is not None
+                              else "launch plan", "kernels": kernels},
+        "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
     return 0

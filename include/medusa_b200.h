@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define MEDUSA_ABI_VERSION 4
+#define MEDUSA_ABI_VERSION 5
 #define MEDUSA_MAX_T 256     /* tree tokens including the root */
 #define MEDUSA_MAX_K 16      /* heads (so tree depth <= 16) */
 #define MEDUSA_MAX_TOPK 32   /* candidates per head */
@@ -490,6 +490,49 @@ size_t medusa_step_workspace_size(const medusa_step_args_t* args);
  * before anything is enqueued. */
 medusa_status_t medusa_step(const medusa_step_args_t* args, void* workspace,
                             size_t workspace_bytes, cudaStream_t stream);
+
+/* Per-step inputs and results of medusa_step_host, in host memory.  Every
+ * pointer is host memory (page-locked, for copies that overlap the step;
+ * pageable memory works but the driver stages it) or NULL: a NULL input is
+ * already in its device buffer of the step's args, a NULL result is not
+ * read back.  A device or managed pointer here is INVALID_ARG. */
+typedef struct medusa_step_host_io {
+  const void* h;                  /* [B, d] dtype -> args->h */
+  const int32_t* root_tokens;     /* [B] -> args->root_tokens */
+  const int32_t* seq_lens;        /* [B] -> args->seq_lens; read on the host during the call to place
+                                   * the tree rows; required when k_tree or v_tree is given */
+  const float* uniforms;          /* [B] -> args->uniforms (which must then be non-NULL) */
+  const void* q;                  /* [layers, B, T, H, hd] dtype -> args->q */
+  const void* k_tree;             /* [layers, B, H, T, hd] dtype: the tree tokens' own key and value */
+  const void* v_tree;             /*   rows, copied to cache rows seq_lens[b] .. seq_lens[b] + T - 1 */
+  const float* base_logits;       /* [B, T, V] -> args->base_logits */
+  int32_t* best_path;             /* [B] */
+  int32_t* accept_len;            /* [B] */
+  int32_t* accepted_tokens;       /* [B, D + 1] */
+  int32_t* next_token;            /* [B] */
+  int32_t* seq_lens_out;          /* [B]: the lengths after the step */
+  cudaStream_t copy_stream;       /* second stream for q, the tree's K/V rows and base_logits, or NULL */
+} medusa_step_host_io_t;
+
+/* medusa_step with its per-step inputs copied in from host memory and its
+ * results copied back (the end-to-end form of the step: "Medusa API参考",
+ * MedusaModelABC medusa_generate calls the verification once per generated
+ * block and reads the accepted tokens on the host).  Enqueued in this order:
+ * h, root_tokens, seq_lens and uniforms on stream; q, k_tree / v_tree (one
+ * 3-D copy per sequence into the caches) and then base_logits on
+ * copy_stream, after all work enqueued earlier on stream; the step, which
+ * waits for copy_stream right before tree attention and right before the
+ * posterior, so the copies overlap the heads; the results on stream.  With
+ * copy_stream NULL every copy goes on stream ahead of the step.  Returns
+ * once all of it is enqueued: synchronise stream before reading the host
+ * results or reusing the host inputs.  args->attn_inputs_ready and
+ * posterior_inputs_ready must be NULL (this call supplies its own events).
+ * Every check of medusa_step, and of io (host pointers, seq_lens[b] + T <=
+ * Lcap on the host copy), happens before anything is enqueued.  Not
+ * capturable in a CUDA graph (it reads seq_lens on the host and creates
+ * events). */
+medusa_status_t medusa_step_host(const medusa_step_args_t* args, const medusa_step_host_io_t* io,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

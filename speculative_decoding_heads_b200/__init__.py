@@ -26,7 +26,7 @@ if not os.path.exists(LIB_PATH):
         "`python -m speculative_decoding_heads_b200._build` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
-ABI_VERSION = 4   # layout of medusa_step_args_t (StepArgs below) and of every signature
+ABI_VERSION = 5   # layout of medusa_step_args_t (StepArgs below) and of every signature
 _lib.medusa_abi_version.restype = ctypes.c_int
 if _lib.medusa_abi_version() != ABI_VERSION:
     raise ImportError(f"{LIB_PATH} has ABI version {_lib.medusa_abi_version()}, this binding needs "
@@ -57,7 +57,7 @@ EXPORTED = [
     "medusa_posterior_workspace_size", "medusa_evaluate_posterior",
     "medusa_accept_kv",
     "medusa_decoder_pack_rows", "medusa_tree_decode_workspace_size", "medusa_tree_decode",
-    "medusa_step_workspace_size", "medusa_step",
+    "medusa_step_workspace_size", "medusa_step", "medusa_step_host",
 ]
 
 _vp = ctypes.c_void_p
@@ -90,6 +90,14 @@ class StepArgs(ctypes.Structure):
         ("attn_inputs_ready", _vp), ("posterior_inputs_ready", _vp),
         ("top_p", _f32), ("uniforms", _vp),
     ]
+
+
+class StepHostIO(ctypes.Structure):
+    """Mirror of ``medusa_step_host_io_t`` (host pointers)."""
+    _fields_ = [("h", _vp), ("root_tokens", _vp), ("seq_lens", _vp), ("uniforms", _vp), ("q", _vp),
+                ("k_tree", _vp), ("v_tree", _vp), ("base_logits", _vp),
+                ("best_path", _vp), ("accept_len", _vp), ("accepted_tokens", _vp), ("next_token", _vp),
+                ("seq_lens_out", _vp), ("copy_stream", _vp)]
 
 
 class DecoderLayer(ctypes.Structure):
@@ -141,6 +149,7 @@ _sig("medusa_tree_decode", _i32, [_vp, ctypes.POINTER(DecoderModel), _i32, _vp, 
                                    _sz, _vp])
 _sig("medusa_step_workspace_size", _sz, [ctypes.POINTER(StepArgs)])
 _sig("medusa_step", _i32, [ctypes.POINTER(StepArgs), _vp, _sz, _vp])
+_sig("medusa_step_host", _i32, [ctypes.POINTER(StepArgs), ctypes.POINTER(StepHostIO), _vp, _sz, _vp])
 
 
 class MedusaError(RuntimeError):
@@ -577,6 +586,8 @@ def make_step_args(tree: Tree, t: dict, mode: int, temperature=0.0, eps=0.09, al
     a.mode = int(mode)
     a.temperature, a.eps, a.alpha = float(temperature), float(eps), float(alpha)
     a.top_p = float(top_p)
+    a._shape = {"B": B, "d": a.d, "V": V, "T": T, "D": tree.D, "layers": layers, "H": H, "hd": hd,
+                "dtype": t["h"].dtype}
     if t.get("uniforms") is not None:
         _spec("uniforms", t["uniforms"], (B,), torch.float32)
         a.uniforms = _p(t["uniforms"]).value
@@ -592,62 +603,49 @@ def medusa_step(args: StepArgs, ws, stream=None):
     _check(_lib.medusa_step(ctypes.byref(args), _p(ws), nbytes, _stream(stream)))
 
 
-def medusa_step_from_host(args: StepArgs, ws, host_in: dict, dev: dict, host_out: dict, stream=None,
-                          copy_stream=None):
-    """One step through the public API with host buffers.
+def medusa_step_host(args: StepArgs, ws, host_in: dict, host_out: dict, stream=None, copy_stream=None):
+    """One step through ``medusa_step_host`` with host buffers.
 
-    Copies every per-step input from pinned host memory (``host_in``: name ->
-    pinned tensor, copied into ``dev[name]``; the tree's own K/V rows are
-    given as ``k_tree``/``v_tree`` [layers, B, H, T, hd] and scattered into
-    the caches at each sequence's current length), runs ``medusa_step`` and
-    reads the results back into the pinned ``host_out`` tensors.
-
-    The heads need only h, the root tokens and the lengths, which go first
-    on ``stream``; q, the tree's K/V rows and then the base logits go on
-    ``copy_stream`` (a second stream, created on first use when omitted)
-    while the heads run, and the step waits for them (through
-    ``attn_inputs_ready`` / ``posterior_inputs_ready``) only before tree
-    attention and before the posterior.  The caller synchronises ``stream``.
-    """
+    ``host_in`` maps input names to host tensors (page-locked for copies that
+    overlap the step): ``h``, ``root_tokens``, ``seq_lens``, ``uniforms``,
+    ``q``, ``base_logits``, and the tree tokens' own key / value rows as
+    ``k_tree`` / ``v_tree`` [layers, B, H, T, hd], which the library places
+    at each sequence's length in the caches.  ``host_out`` maps result names
+    (``best_path``, ``accept_len``, ``accepted_tokens``, ``next_token``,
+    ``seq_lens``) to host tensors the results are copied into.  Absent inputs
+    are already on the device; absent results are not copied.  The copies of
+    q, the tree rows and the base logits go on ``copy_stream`` (created on
+    first use when omitted) while the heads run.  The caller synchronises
+    ``stream`` before reading ``host_out``."""
+    sh = args._shape
+    B, T, D = sh["B"], sh["T"], sh["D"]
+    shapes = {"h": ((B, sh["d"]), sh["dtype"]), "root_tokens": ((B,), torch.int32),
+              "seq_lens": ((B,), torch.int32), "uniforms": ((B,), torch.float32),
+              "q": ((sh["layers"], B, T, sh["H"], sh["hd"]), sh["dtype"]),
+              "k_tree": ((sh["layers"], B, sh["H"], T, sh["hd"]), sh["dtype"]),
+              "v_tree": ((sh["layers"], B, sh["H"], T, sh["hd"]), sh["dtype"]),
+              "base_logits": ((B, T, sh["V"]), torch.float32),
+              "best_path": ((B,), torch.int32), "accept_len": ((B,), torch.int32),
+              "accepted_tokens": ((B, D + 1), torch.int32), "next_token": ((B,), torch.int32)}
+    io = StepHostIO()
+    for group, names in ((host_in, ("h", "root_tokens", "seq_lens", "uniforms", "q", "k_tree", "v_tree",
+                                    "base_logits")),
+                         (host_out, ("best_path", "accept_len", "accepted_tokens", "next_token", "seq_lens"))):
+        extra = set(group) - set(names)
+        _require(not extra, f"medusa_step_host: unknown buffers {sorted(extra)}")
+        for name in names:
+            x = group.get(name)
+            if x is None:
+                continue
+            shape, dtype = shapes[name]
+            _spec(name, x, shape, dtype)
+            _require(not x.is_cuda, f"medusa_step_host: {name} must be a host tensor")
+            setattr(io, "seq_lens_out" if group is host_out and name == "seq_lens" else name, x.data_ptr())
     s = stream or torch.cuda.current_stream()
     if copy_stream is None:
         if getattr(args, "_copy_stream", None) is None:
             args._copy_stream = torch.cuda.Stream()
         copy_stream = args._copy_stream
-    if getattr(args, "_events", None) is None:
-        args._events = (torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event())
-    ev_start, ev_attn, ev_post = args._events
-    early = ("h", "root_tokens", "seq_lens")
-    with torch.cuda.stream(s):
-        for name in early:
-            if name in host_in:
-                dev[name].copy_(host_in[name], non_blocking=True)
-        ev_start.record(s)   # everything earlier on `stream` (the previous step) comes first
-    with torch.cuda.stream(copy_stream):
-        copy_stream.wait_event(ev_start)
-        if "q" in host_in:
-            dev["q"].copy_(host_in["q"], non_blocking=True)
-        if "k_tree" in host_in:
-            lens = host_in["seq_lens"]
-            T = host_in["k_tree"].shape[3]
-            for b in range(lens.shape[0]):
-                L = int(lens[b])
-                dev["k_cache"][:, b, :, L:L + T, :].copy_(host_in["k_tree"][:, b], non_blocking=True)
-                dev["v_cache"][:, b, :, L:L + T, :].copy_(host_in["v_tree"][:, b], non_blocking=True)
-        for name, src in host_in.items():
-            if name not in early and name not in ("q", "k_tree", "v_tree", "base_logits"):
-                dev[name].copy_(src, non_blocking=True)
-        ev_attn.record(copy_stream)
-        if "base_logits" in host_in:
-            dev["base_logits"].copy_(host_in["base_logits"], non_blocking=True)
-        ev_post.record(copy_stream)
-    args.attn_inputs_ready = ctypes.c_void_p(ev_attn.cuda_event)
-    args.posterior_inputs_ready = ctypes.c_void_p(ev_post.cuda_event)
-    try:
-        with torch.cuda.stream(s):
-            medusa_step(args, ws, s)
-            for name, dst in host_out.items():
-                dst.copy_(dev[name], non_blocking=True)
-    finally:
-        args.attn_inputs_ready = None
-        args.posterior_inputs_ready = None
+    io.copy_stream = copy_stream.cuda_stream
+    nbytes = _nbytes("ws", ws)
+    _check(_lib.medusa_step_host(ctypes.byref(args), ctypes.byref(io), _p(ws), nbytes, _stream(s)))

@@ -429,8 +429,7 @@ extern "C" size_t medusa_step_workspace_size(const medusa_step_args_t* args) {
   return step_layout(args).total;
 }
 
-extern "C" medusa_status_t medusa_step(const medusa_step_args_t* a, void* workspace, size_t workspace_bytes,
-                                       cudaStream_t stream) {
+medusa_status_t medusa::check_step(const medusa_step_args_t* a, const void* workspace, size_t workspace_bytes) {
   if (!a) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_step: args is null");
   medusa_status_t st = check_tree(a->tree, "medusa_step");
   if (st != MEDUSA_OK) return st;
@@ -439,9 +438,8 @@ extern "C" medusa_status_t medusa_step(const medusa_step_args_t* a, void* worksp
   if (!workspace) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_step: workspace is null");
   const StepLayout l = step_layout(a);
   if (workspace_bytes < l.total) return fail(MEDUSA_ERR_INVALID_ARG, "medusa_step: workspace too small");
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  unsigned char* ws = static_cast<unsigned char*>(const_cast<void*>(workspace));
   void* ws_heads = ws;
-  void* ws_attn = ws + l.heads;
   void* ws_post = ws + l.heads + l.attn;
   // Validate every stage before launching any of them.
   st = check_heads(a->h, a->W1, a->b1, a->Wout, a->B, a->d, a->V, a->K, a->topk, a->dtype, a->head_logits,
@@ -455,9 +453,19 @@ extern "C" medusa_status_t medusa_step(const medusa_step_args_t* a, void* worksp
   st = check_posterior(a->tree, a->B, a->V, a->base_logits, a->candidates, a->mode, a->temperature, a->eps, a->alpha,
                        a->top_p, a->best_path, a->accept_len, a->accepted_tokens, a->next_token, ws_post, l.post);
   if (st != MEDUSA_OK) return st;
-  st = check_accept(a->tree, a->layers, a->B, a->H, a->hd, a->dtype, a->k_cache, a->v_cache, a->Lcap, a->seq_lens,
-                    a->best_path, a->accept_len);
+  return check_accept(a->tree, a->layers, a->B, a->H, a->hd, a->dtype, a->k_cache, a->v_cache, a->Lcap,
+                      a->seq_lens, a->best_path, a->accept_len);
+}
+
+extern "C" medusa_status_t medusa_step(const medusa_step_args_t* a, void* workspace, size_t workspace_bytes,
+                                       cudaStream_t stream) {
+  medusa_status_t st = check_step(a, workspace, workspace_bytes);
   if (st != MEDUSA_OK) return st;
+  const StepLayout l = step_layout(a);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  void* ws_heads = ws;
+  void* ws_attn = ws + l.heads;
+  void* ws_post = ws + l.heads + l.attn;
 
   // S1-S4 in one launch per batch group: the heads kernel's last CTA also
   // builds the candidate tree from the final top-k.

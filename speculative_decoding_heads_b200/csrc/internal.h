@@ -62,6 +62,9 @@ medusa_status_t check_heads(const void* h, const void* W1, const void* b1, const
                             int K, int topk, medusa_dtype_t dtype, const float* head_logits, const int32_t* topk_ids,
                             const float* topk_vals, const void* ws, size_t ws_bytes);
 
+// Every host-side check of medusa_step (api.cu); nothing is enqueued.
+medusa_status_t check_step(const medusa_step_args_t* args, const void* ws, size_t ws_bytes);
+
 // Kernel launchers (heads.cu, tree_kernels.cu, attention.cu, posterior.cu, accept.cu).
 size_t heads_workspace_bytes(int B, int d, int V, int K, int topk);
 medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, const void* Wout,

@@ -112,6 +112,28 @@ def test_heads_topk_wide_rows(mb, dev, B):
     _status_clean(mb)
 
 
+@pytest.mark.parametrize("B", [2, 16, 17, 33])
+def test_heads_topk_tensor_core_passes(mb, dev, B):
+    # bf16 heads from two sequences up run on the tensor cores in passes of
+    # at most 16 sequences (two launches each): B 2 is the smallest pass,
+    # 16 a full one, 17 and 33 end in a one-sequence pass.  At 33 sequences
+    # two heads of top-4 keep the gap guard satisfiable.
+    from synth.workloads import shrink
+    extra = {"K": 2, "topk": 4} if B > 17 else {}
+    w = shrink(SMALL["v13b_small"], name=f"heads_tc_B{B}", d=512, V=2100, B=B, **extra)
+    sub_h, u, z = pick_sub_h(w, max_tries=32)
+    ids_ref, vals_ref = O.topk_desc(z, w.topk)
+    t = dev.materialise(w, sub_h=sub_h)
+    ws = mb.workspace(mb.medusa_heads_workspace_size(w.B, w.d, w.V, w.K, w.topk))
+    mb.medusa_heads_topk(t["h"], t["W1"], t["b1"], t["Wout"], w.topk, t["topk_ids"], t["topk_vals"], ws,
+                         head_logits=t["head_logits"])
+    torch.cuda.synchronize()
+    assert np.array_equal(_np(t["topk_ids"]), ids_ref)
+    check_logits(_np(t["head_logits"]), z)
+    check_logits(_np(t["topk_vals"]), vals_ref)
+    _status_clean(mb)
+
+
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_build_tree(mb, dev, name):
     w = SMALL[name]
@@ -441,10 +463,11 @@ def test_device_check_on_overflowing_sequence(mb, dev):
     _status_clean(mb)
 
 
-def test_step_from_host_matches_device_step(mb, dev):
-    # The host-buffer step copies q, the tree's K/V rows and the base logits
-    # on a second stream while the heads run; the step waits for them through
-    # the two input-ready events.  Its results equal a step over device inputs.
+def test_step_host_matches_device_step(mb, dev):
+    # medusa_step_host copies q, the tree's K/V rows (one 3-D copy per
+    # sequence into the caches) and the base logits on a second stream while
+    # the heads run; the step waits for them through the two input-ready
+    # events.  Its results equal a step over device-resident inputs.
     w = SMALL["v7b_small"]
     sub_h, _, _ = pick_sub_h(w)
     tree = _tree(mb, w)
@@ -457,7 +480,7 @@ def test_step_from_host_matches_device_step(mb, dev):
     mb.medusa_step(args, ws)
     torch.cuda.synchronize()
     ref = {k: t[k].clone() for k in ("best_path", "accept_len", "accepted_tokens", "next_token", "attn_out",
-                                     "seq_lens", "k_cache")}
+                                     "seq_lens", "k_cache", "v_cache")}
     pin = lambda x: x.cpu().pin_memory()
     L = lens0.cpu()
     host_in = {"h": pin(t["h"]), "root_tokens": pin(t["root_tokens"]), "seq_lens": pin(lens0),
@@ -465,20 +488,54 @@ def test_step_from_host_matches_device_step(mb, dev):
                "k_tree": pin(torch.stack([kc0[:, b, :, int(L[b]):int(L[b]) + w.T] for b in range(w.B)], 1)),
                "v_tree": pin(torch.stack([vc0[:, b, :, int(L[b]):int(L[b]) + w.T] for b in range(w.B)], 1))}
     host_out = {k: torch.empty_like(t[k], device="cpu").pin_memory()
-                for k in ("best_path", "accept_len", "accepted_tokens", "next_token")}
-    # clobber every input and output the host step must bring back
-    for k in ("q", "base_logits", "attn_out"):
+                for k in ("best_path", "accept_len", "accepted_tokens", "next_token", "seq_lens")}
+    # clobber every input the host step must bring in, and the tree rows of the caches
+    for k in ("q", "base_logits", "attn_out", "h"):
         t[k].fill_(float("nan"))
-    for k in ("best_path", "accept_len", "accepted_tokens", "next_token"):
+    for k in ("best_path", "accept_len", "accepted_tokens", "next_token", "root_tokens"):
         t[k].fill_(-9)
-    t["k_cache"].copy_(kc0)
-    t["v_cache"].copy_(vc0)
+    t["seq_lens"].fill_(0)
+    kc, vc = kc0.clone(), vc0.clone()
+    for b in range(w.B):
+        kc[:, b, :, int(L[b]):int(L[b]) + w.T] = float("nan")
+        vc[:, b, :, int(L[b]):int(L[b]) + w.T] = float("nan")
+    t["k_cache"].copy_(kc)
+    t["v_cache"].copy_(vc)
     stream = torch.cuda.Stream()
-    mb.medusa_step_from_host(args, ws, host_in, dict(t), host_out, stream)
+    mb.medusa_step_host(args, ws, host_in, host_out, stream)
     stream.synchronize()
     for k in host_out:
         assert torch.equal(host_out[k], ref[k].cpu()), k
     assert torch.equal(t["attn_out"], ref["attn_out"])
     assert torch.equal(t["seq_lens"], ref["seq_lens"])
     assert torch.equal(t["k_cache"], ref["k_cache"])
+    assert torch.equal(t["v_cache"], ref["v_cache"])
+    _status_clean(mb)
+
+
+def test_step_host_refuses_device_buffers_and_overflow(mb, dev):
+    # io must hold host memory; a host length that would put the tree rows
+    # past Lcap is refused; both before anything is enqueued.
+    import ctypes
+    w = SMALL["v7b_small"]
+    tree = _tree(mb, w)
+    t = dev.materialise(w)
+    dev.tree_outputs(t, w.B, tree.T, tree.P, tree.D)
+    args = mb.make_step_args(tree, t, mb.MEDUSA_GREEDY)
+    ws = mb.workspace(mb.medusa_step_workspace_size(args))
+    before = {k: t[k].clone() for k in ("best_path", "seq_lens", "k_cache")}
+    io = mb.StepHostIO()
+    io.h = t["h"].data_ptr()   # device memory where host memory is required
+    st = mb._lib.medusa_step_host(ctypes.byref(args), ctypes.byref(io), ws.data_ptr(), ws.numel(),
+                                  torch.cuda.current_stream().cuda_stream)
+    assert st == mb.MEDUSA_ERR_INVALID_ARG
+    lens = torch.full((w.B,), w.Lcap - tree.T + 1, dtype=torch.int32).pin_memory()
+    kt = torch.zeros((w.layers, w.B, w.H, tree.T, w.hd), dtype=t["k_cache"].dtype).pin_memory()
+    with pytest.raises(mb.MedusaError):
+        mb.medusa_step_host(args, ws, {"seq_lens": lens, "k_tree": kt}, {})
+    with pytest.raises(ValueError):
+        mb.medusa_step_host(args, ws, {"h": t["h"]}, {})
+    torch.cuda.synchronize()
+    for k, v in before.items():
+        assert torch.equal(t[k], v), k
     _status_clean(mb)
