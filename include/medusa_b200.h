@@ -429,7 +429,7 @@ size_t medusa_tree_decode_workspace_size(const medusa_tree_t* tree, const medusa
  * (fp32 accumulation).  Requires seq_lens[b] + T <= Lcap (a violation sets
  * MEDUSA_ERR_DEVICE_CHECK); a token outside [0, V) sets
  * MEDUSA_ERR_DEVICE_CHECK.  Every matrix product streams its weights once
- * per 64 tree tokens.  Pointers 16-byte aligned. */
+ * per pass of up to 256 of the B*T tree tokens.  Pointers 16-byte aligned. */
 medusa_status_t medusa_tree_decode(const medusa_tree_t* tree, const medusa_decoder_t* model, int B,
                                    const int32_t* tree_tokens, void* k_cache, void* v_cache, int Lcap,
                                    const int32_t* seq_lens, float* logits, float* hidden, void* workspace,

@@ -9,11 +9,13 @@
 // RMSNorm, SwiGLU feed-forward and residual; then a final RMSNorm and the LM
 // head.
 //
-// Every matrix product here is weights x (at most 64 tree tokens): the
-// weights stream from HBM once per pass of 64 tokens, as the A operand of
-// M = 128, N = 64, K = 16 tcgen05 products (TMA boxes of 128 rows x 2 x 64
+// Every matrix product here is weights x (a pass of at most 256 tree
+// tokens): the weights stream from HBM once per pass, as the A operand of
+// M = 128, N = kN, K = 16 tcgen05 products (TMA boxes of 128 rows x 64
 // columns, 128-byte swizzle, no multicast), the tokens' activations are the
-// B operand, and the fp32 accumulators live in tensor memory.  The W/64/2
+// B operand, and the fp32 accumulators live in tensor memory.  A pass holds
+// 64, 128 or 256 tokens (the smallest that takes all of them, else 256); a
+// ring stage holds 2 column blocks of 64 at 64 tokens and 1 above.  The
 // ring stages of a product are split evenly over the CTAs (stream-K); a tile
 // of 128 rows cut by a range boundary is summed, per quarter of its rows, by
 // the last CTA to finish it, in CTA order.  The epilogue is fused per
@@ -36,16 +38,24 @@ namespace {
 
 constexpr int kTileRows = 128;
 constexpr int kKStep = 64;
-constexpr int kKPS = 2;                        // column blocks per ring stage
-constexpr int kN = 64;                         // tokens per pass (MMA N)
 constexpr int kWBlock = kTileRows * 128;       // 16 KB
-constexpr int kXBlock = kN * 128;              // 8 KB
-constexpr int kSB = kKPS * (kWBlock + kXBlock);   // 48 KB per stage
-constexpr int kNS = 4;
 constexpr int kThreads = 256;                  // warps 0 producer, 1 MMA, 4-7 epilogue
-constexpr uint32_t kTmemCols = 128;            // two accumulators of 64 columns
-constexpr int kSmem = 1024 + kNS * kSB + 1024;
+constexpr int kRingBytes = 196608;             // 192 KB of ring stages
+constexpr int kMaxN = 256;                     // tokens per pass, at most
 constexpr float kRmsEps = 1e-6f;
+
+// The shape of one pass of kN tokens.
+template <int kN_>
+struct Cfg {
+  static constexpr int kN = kN_;                             // tokens per pass (MMA N)
+  static constexpr int kKPS = kN_ >= 128 ? 1 : 2;            // column blocks per ring stage
+  static constexpr int kXBlock = kN_ * 128;                  // activations of one column block
+  static constexpr int kSB = kKPS * (kWBlock + kXBlock);     // bytes per stage: 48, 32, 48 KB
+  static constexpr int kNS = kRingBytes / kSB;               // stages: 4, 6, 4
+  static constexpr uint32_t kTmemCols = 2 * kN_;             // two accumulators of kN columns
+  static constexpr int kTail = 4096;                         // barriers and the token table
+  static constexpr int kSmem = 1024 + kNS * kSB + kTail;
+};
 
 enum Mode : int { kQKV = 0, kResid = 1, kSwiGLU = 2, kLogits = 3 };
 
@@ -53,8 +63,9 @@ struct GemmArgs {
   int rows;               // weight rows
   int kdim;               // reduction length (a multiple of 128)
   int tiles, nst, W, G;   // tiles of 128 rows, stages per tile, all stages, CTAs
-  int tok0, ntok;         // this pass: tokens tok0 .. tok0 + 63 (clipped to ntok)
-  float* part;            // [G, 2, 128, 64]
+  int kps;                // column blocks per ring stage
+  int tok0, ntok;         // this pass: tokens tok0 .. tok0 + kN - 1 (clipped to ntok)
+  float* part;            // [G, 2, 128, kN]
   unsigned* tile_cnt;     // [tiles * 4]
   int* status;
   // QKV
@@ -72,6 +83,7 @@ struct GemmArgs {
   float* logits;          // [ntok, rows]
 };
 
+template <int kN, int kNS>
 struct Bars {
   uint64_t full[kNS], empty[kNS];
   uint64_t acc_full[2], acc_empty[2];
@@ -100,13 +112,14 @@ __device__ __forceinline__ bool next_unit(const GemmArgs& a, int& st, int st_hi,
   x.tile = st / a.nst;
   const int t0 = x.tile * a.nst;
   const int e = st_hi < t0 + a.nst ? st_hi : t0 + a.nst;
-  x.k0 = (st - t0) * kKPS;
-  x.k1 = (e - t0) * kKPS;
+  x.k0 = (st - t0) * a.kps;
+  x.k1 = (e - t0) * a.kps;
   st = e;
   return true;
 }
 
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Bars* bs, int* status) {
+template <class BarsT>
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, BarsT* bs, int* status) {
   if (bs->abort) return false;
   if (mbar_wait(bar, parity)) return true;
   set_device_status(status, MEDUSA_ERR_TIMEOUT, kDetailDecoderWait);
@@ -121,8 +134,8 @@ __device__ __forceinline__ float bf(uint16_t v) { return __uint_as_float(static_
 // c0 + 31 (in acc).  Every global load comes before the stores, so the loads
 // of the 32 tokens overlap.
 constexpr int kHalf = 32;
-template <int kMode>
-__device__ __forceinline__ void epilogue_half(const GemmArgs& a, const Bars* bs, int tile, int r, int c0,
+template <int kMode, int kN, class BarsT>
+__device__ __forceinline__ void epilogue_half(const GemmArgs& a, const BarsT* bs, int tile, int r, int c0,
                                               const float (&acc)[kHalf]) {
   const int nvalid = a.ntok - a.tok0 < kN ? a.ntok - a.tok0 : kN;
   if constexpr (kMode == kQKV) {
@@ -184,14 +197,19 @@ __device__ __forceinline__ void epilogue_half(const GemmArgs& a, const Bars* bs,
   }
 }
 
-template <int kMode>
+template <int kMode, int kN>
 __global__ void __launch_bounds__(kThreads, 1)
     wgemm_kernel(const __grid_constant__ CUtensorMap w_map, const __grid_constant__ CUtensorMap x_map,
                  const GemmArgs a) {
+  using C = Cfg<kN>;
+  constexpr int kKPS = C::kKPS, kXBlock = C::kXBlock, kSB = C::kSB, kNS = C::kNS;
+  constexpr uint32_t kTmemCols = C::kTmemCols;
+  using BarsT = Bars<kN, kNS>;
+  static_assert(sizeof(BarsT) <= C::kTail, "barrier block too large");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars* bs = reinterpret_cast<Bars*>(smem + kNS * kSB);
+  BarsT* bs = reinterpret_cast<BarsT*>(smem + kNS * kSB);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x;
   const int st_lo = stage_lo(cta, a), st_hi = stage_lo(cta + 1, a);
@@ -336,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = x.tile == st_lo / a.nst ? 0 : 1;
         float* mine = a.part + ((static_cast<size_t>(cta) * 2 + slot) * kTileRows + r) * kN;
 #pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
+        for (int hh = 0; hh < kN / kHalf; ++hh) {
           float acc[kHalf];
           tc::tmem_ld32(tacc + hh * kHalf, acc);
           tc::tmem_wait_ld();
@@ -357,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (mine_last) {
 #pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
+        for (int hh = 0; hh < kN / kHalf; ++hh) {
           float acc[kHalf];
           tc::tmem_ld32(tacc + hh * kHalf, acc);
           tc::tmem_wait_ld();
@@ -381,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < kHalf; ++c) acc[c] = sum[c];
           }
-          epilogue_half<kMode>(a, bs, x.tile, r, hh * kHalf, acc);
+          epilogue_half<kMode, kN>(a, bs, x.tile, r, hh * kHalf, acc);
         }
       }
       tc::fence_before_sync();
@@ -468,33 +486,40 @@ __global__ void to_bf16_kernel(const float* x, size_t n, uint16_t* y) {
 }
 
 bool encode_w(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, uint64_t kdim,
-              uint64_t rows, uint32_t box_rows) {
+              uint64_t rows, uint32_t box_rows, uint32_t kps) {
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kKStep), rows, kdim / kKStep, 1};
   const cuuint64_t strides[3] = {kdim * 2, kKStep * 2, kdim * rows * 2};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(kKStep), box_rows, static_cast<cuuint32_t>(kKPS), 1};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(kKStep), box_rows, kps, 1};
   const cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Scratch of the matrix products: tile counters, then [G, 2, 128, 64] partials.
-size_t gemm_scratch_bytes(int D, int F, int V) {
+// Tokens per pass for a forward over ntok tokens: the smallest of 64, 128
+// and 256 that takes all of them, else 256.
+int tokens_per_pass(int ntok) { return ntok <= 64 ? 64 : (ntok <= 128 ? 128 : kMaxN); }
+
+// Scratch of the matrix products: tile counters, then [G, 2, 128, kN] partials.
+size_t gemm_scratch_bytes(int D, int F, int V, int ntok) {
   int rows = 3 * D;
   if (2 * F > rows) rows = 2 * F;
   if (V > rows) rows = V;
   const int tiles = (rows + kTileRows - 1) / kTileRows;
   const int G = sm_count() > 0 ? sm_count() : 1;
-  return align_up(static_cast<size_t>(tiles) * 16, 256) + align_up(static_cast<size_t>(G) * 2 * kTileRows * kN * 4, 256);
+  return align_up(static_cast<size_t>(tiles) * 16, 256) +
+         align_up(static_cast<size_t>(G) * 2 * kTileRows * tokens_per_pass(ntok) * 4, 256);
 }
 
-template <int kMode>
-medusa_status_t gemm(const void* Wt, const uint16_t* X, GemmArgs a, void* ws, cudaStream_t stream) {
+template <int kMode, int kN>
+medusa_status_t gemm_n(const void* Wt, const uint16_t* X, GemmArgs a, void* ws, cudaStream_t stream) {
+  using C = Cfg<kN>;
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!enc) return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_tree_decode: cuTensorMapEncodeTiled unavailable");
   const int G = sm_count();
+  a.kps = C::kKPS;
   a.tiles = (a.rows + kTileRows - 1) / kTileRows;
-  a.nst = a.kdim / kKStep / kKPS;
+  a.nst = a.kdim / kKStep / C::kKPS;
   a.W = a.tiles * a.nst;
   a.G = a.W < G ? a.W : G;
   unsigned char* w = static_cast<unsigned char*>(ws);
@@ -502,20 +527,30 @@ medusa_status_t gemm(const void* Wt, const uint16_t* X, GemmArgs a, void* ws, cu
   a.part = reinterpret_cast<float*>(w + align_up(static_cast<size_t>(a.tiles) * 4 * 4, 256));
   a.status = device_status_ptr();
   CUtensorMap wm, xm;
-  if (!encode_w(enc, &wm, Wt, a.kdim, a.rows, kTileRows) || !encode_w(enc, &xm, X, a.kdim, a.ntok, kN))
+  if (!encode_w(enc, &wm, Wt, a.kdim, a.rows, kTileRows, C::kKPS) ||
+      !encode_w(enc, &xm, X, a.kdim, a.ntok, kN, C::kKPS))
     return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_tree_decode: tensor map rejected");
-  auto fn = wgemm_kernel<kMode>;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  auto fn = wgemm_kernel<kMode, kN>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   for (a.tok0 = 0; e == cudaSuccess && a.tok0 < a.ntok; a.tok0 += kN)
-    e = launch_kernel(fn, dim3(a.G), dim3(kThreads), static_cast<size_t>(kSmem), stream, true, wm, xm, a);
+    e = launch_kernel(fn, dim3(a.G), dim3(kThreads), static_cast<size_t>(C::kSmem), stream, true, wm, xm, a);
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_tree_decode: matrix-product launch", e);
+}
+
+template <int kMode>
+medusa_status_t gemm(const void* Wt, const uint16_t* X, GemmArgs a, void* ws, cudaStream_t stream) {
+  switch (tokens_per_pass(a.ntok)) {
+    case 64: return gemm_n<kMode, 64>(Wt, X, a, ws, stream);
+    case 128: return gemm_n<kMode, 128>(Wt, X, a, ws, stream);
+    default: return gemm_n<kMode, kMaxN>(Wt, X, a, ws, stream);
+  }
 }
 
 }  // namespace
 
 size_t decoder_workspace_bytes(int ntok, int D, int F, int V) {
   // The products' scratch; then x fp32, xn bf16, q bf16, attention fp32 and bf16, act bf16.
-  size_t o = gemm_scratch_bytes(D, F, V);
+  size_t o = gemm_scratch_bytes(D, F, V, ntok);
   o += align_up(static_cast<size_t>(ntok) * D * 4, 256);       // x
   o += align_up(static_cast<size_t>(ntok) * D * 2, 256);       // xn
   o += align_up(static_cast<size_t>(ntok) * D * 2, 256);       // q (bf16, [ntok, H, 128])
@@ -531,7 +566,7 @@ medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, 
   const int D = m->D, F = m->F, V = m->V, H = D / 128;
   const int ntok = B * t.T;
   unsigned char* w = static_cast<unsigned char*>(ws);
-  size_t o = gemm_scratch_bytes(D, F, V);
+  size_t o = gemm_scratch_bytes(D, F, V, ntok);
   void* gws = w;
   float* x = reinterpret_cast<float*>(w + o);
   o += align_up(static_cast<size_t>(ntok) * D * 4, 256);

@@ -60,8 +60,10 @@ def _close(got, ref, what):
 
 @pytest.mark.parametrize("B,lens,choices", [
     (2, [37, 70], ("ranksum", 3, 2, 14)),        # T 15: one pass of 64 tokens
-    (4, [5, 130, 64, 0], ("ranksum", 4, 3, 20)),  # T 21: 84 tokens, two passes; an empty prefix
+    (4, [5, 130, 64, 0], ("ranksum", 4, 3, 20)),  # T 21: 84 tokens, one pass of 128; an empty prefix
     (1, [300], ("ranksum", 5, 10, 63)),           # T 64: the 7B tree, one full pass
+    (3, [10, 200, 77], ("ranksum", 5, 10, 63)),   # 192 tokens: one pass of 256
+    (5, [3, 90, 0, 41, 260], ("ranksum", 5, 10, 63)),   # 320 tokens: passes of 256 and 64 rows
 ])
 def test_tree_decode_matches_oracle(mb, B, lens, choices):
     rng = np.random.default_rng(B * 100 + len(choices))
