@@ -92,8 +92,8 @@ struct Bars {
   int abort;
   // QKV: for each token c of the pass, its rotary position and its cache row
   // offset ((b H) Lcap + L + node) 128 (-1: no valid cache row)
-  int pos[kN];
-  long long crow[kN];
+  alignas(16) int pos[kN];
+  alignas(16) long long crow[kN];
 };
 
 __device__ __forceinline__ int stage_lo(int c, const GemmArgs& a) {
@@ -127,13 +127,16 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ba
   return false;
 }
 
-__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
+// SiLU for a value that is rounded to bf16 next: the fast exponential and
+// division (a few ulp of fp32) are far inside bf16's rounding.
+__device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 __device__ __forceinline__ float bf(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
 
 // The epilogue of one finished tile row, for the 32 token columns c0 ..
 // c0 + 31 (in acc).  Every global load comes before the stores, so the loads
 // of the 32 tokens overlap.
 constexpr int kHalf = 32;
+constexpr int kPar = 3;   // partial sums of a shared tile loaded at once
 template <int kMode, int kN, class BarsT>
 __device__ __forceinline__ void epilogue_half(const GemmArgs& a, const BarsT* bs, int tile, int r, int c0,
                                               const float (&acc)[kHalf]) {
@@ -145,26 +148,52 @@ __device__ __forceinline__ void epilogue_half(const GemmArgs& a, const BarsT* bs
     // rotation frequency base^(-2j/128) with base 10000, angle reduced in double
     const double inv = exp2(-static_cast<double>(2 * j) / 128.0 * 13.287712379549449);
     uint16_t* cache = which == 1 ? a.k_cache : a.v_cache;
-#pragma unroll 4
-    for (int i = 0; i < kHalf; ++i) {
-      const int c = c0 + i;
-      const float own = acc[i];
-      const float other = __shfl_xor_sync(0xffffffffu, own, 1);
-      const long long row = bs->crow[c];
-      if (c >= nvalid || row < 0) continue;
-      float out = own;
-      if (which < 2) {
-        const double ang = static_cast<double>(bs->pos[c]) * inv;
-        const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
-        float sn, cs;
-        sincosf(static_cast<float>(red), &sn, &cs);
-        out = (r & 1) ? other * sn + own * cs : own * cs - other * sn;
+    // 16 tokens at a time: their table entries (vector loads) and partner
+    // values first, so that the 16 rotations are independent and no store
+    // sits between loads; then the stores, each under its own predicate.
+    uint16_t* const dst = which == 0 ? a.q_out + h * 128 + feat : cache + static_cast<long long>(h) * a.Lcap * 128 + feat;
+#pragma unroll
+    for (int i0 = 0; i0 < kHalf; i0 += 16) {
+      int pos[16];
+      long long row[16];
+      float other[16];
+      const int4* pp = reinterpret_cast<const int4*>(bs->pos + c0 + i0);
+      const longlong2* rp = reinterpret_cast<const longlong2*>(bs->crow + c0 + i0);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int4 p4 = pp[k];
+        pos[4 * k] = p4.x;
+        pos[4 * k + 1] = p4.y;
+        pos[4 * k + 2] = p4.z;
+        pos[4 * k + 3] = p4.w;
       }
-      const uint16_t v = f32_to_bf16_rne(out);
-      if (which == 0) {
-        a.q_out[(static_cast<size_t>(a.tok0 + c) * a.H + h) * 128 + feat] = v;
-      } else {
-        cache[row + static_cast<long long>(h) * a.Lcap * 128 + feat] = v;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const longlong2 r2 = rp[k];
+        row[2 * k] = r2.x;
+        row[2 * k + 1] = r2.y;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) other[i] = __shfl_xor_sync(0xffffffffu, acc[i0 + i], 1);
+      uint16_t v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float own = acc[i0 + i];
+        float out = own;
+        if (which < 2) {
+          const double ang = static_cast<double>(pos[i]) * inv;
+          const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+          float sn, cs;
+          __sincosf(static_cast<float>(red), &sn, &cs);   // |red| <= pi
+          out = (r & 1) ? other[i] * sn + own * cs : own * cs - other[i] * sn;
+        }
+        v[i] = f32_to_bf16_rne(out);
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int c = c0 + i0 + i;
+        const long long o = which == 0 ? static_cast<long long>(a.tok0 + c) * a.H * 128 : row[i];
+        if (c < nvalid && row[i] >= 0) dst[o] = v[i];
       }
     }
   } else if constexpr (kMode == kSwiGLU) {
@@ -380,20 +409,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tmem_ld32(tacc + hh * kHalf, acc);
           tc::tmem_wait_ld();
           if (split) {
+            // The parts in CTA order, kPar CTAs' loads in flight at a time.
             float sum[kHalf];
 #pragma unroll
             for (int c = 0; c < kHalf; ++c) sum[c] = 0.f;
-            for (int cc = c_first; cc <= c_last; ++cc) {
-              const int sl = x.tile == stage_lo(cc, a) / a.nst ? 0 : 1;
-              const float* pc = a.part + ((static_cast<size_t>(cc) * 2 + sl) * kTileRows + r) * kN + hh * kHalf;
+            for (int cc0 = c_first; cc0 <= c_last; cc0 += kPar) {
+              float4 pv[kPar][kHalf / 4];
 #pragma unroll
-              for (int c = 0; c < kHalf; c += 4) {
-                const float4 v = cc == cta ? make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3])
-                                           : __ldcg(reinterpret_cast<const float4*>(pc + c));
-                sum[c] += v.x;
-                sum[c + 1] += v.y;
-                sum[c + 2] += v.z;
-                sum[c + 3] += v.w;
+              for (int u = 0; u < kPar; ++u) {
+                const int cc = cc0 + u;
+                if (cc <= c_last && cc != cta) {
+                  const int sl = x.tile == stage_lo(cc, a) / a.nst ? 0 : 1;
+                  const float4* pc = reinterpret_cast<const float4*>(
+                      a.part + ((static_cast<size_t>(cc) * 2 + sl) * kTileRows + r) * kN + hh * kHalf);
+#pragma unroll
+                  for (int e = 0; e < kHalf / 4; ++e) pv[u][e] = __ldcg(pc + e);
+                }
+              }
+#pragma unroll
+              for (int u = 0; u < kPar; ++u) {
+                const int cc = cc0 + u;
+                if (cc <= c_last) {
+#pragma unroll
+                  for (int e = 0; e < kHalf / 4; ++e) {
+                    const float4 v = cc == cta ? make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3])
+                                               : pv[u][e];
+                    sum[4 * e] += v.x;
+                    sum[4 * e + 1] += v.y;
+                    sum[4 * e + 2] += v.z;
+                    sum[4 * e + 3] += v.w;
+                  }
+                }
               }
             }
 #pragma unroll
