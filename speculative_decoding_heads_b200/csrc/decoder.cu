@@ -47,7 +47,6 @@ constexpr float kRmsEps = 1e-6f;
 // The shape of one pass of kN tokens.
 template <int kN_>
 struct Cfg {
-  static constexpr int kN = kN_;                             // tokens per pass (MMA N)
   static constexpr int kKPS = kN_ >= 128 ? 1 : 2;            // column blocks per ring stage
   static constexpr int kXBlock = kN_ * 128;                  // activations of one column block
   static constexpr int kSB = kKPS * (kWBlock + kXBlock);     // bytes per stage: 48, 32, 48 KB
@@ -88,6 +87,8 @@ struct Bars {
   uint64_t full[kNS], empty[kNS];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t mma_done;
+  uint64_t tail[4];        // per lane quarter: the final unit's chunk split is decided
+  int tail_n[4];           // per lane quarter: index of the final unit (-1: no help wanted)
   uint32_t tmem_base;
   int abort;
   // QKV: for each token c of the pass, its rotary position and its cache row
@@ -226,6 +227,54 @@ __device__ __forceinline__ void epilogue_half(const GemmArgs& a, const BarsT* bs
   }
 }
 
+// One 32-column chunk of a finished tile row: the accumulator from tensor
+// memory, for a shared tile plus the other CTAs' parts (summed in CTA order,
+// kPar CTAs' loads in flight at a time), then the epilogue.
+template <int kMode, int kN, class BarsT>
+__device__ __forceinline__ void finish_chunk(const GemmArgs& a, const BarsT* bs, int tile, int r, uint32_t tacc,
+                                             int hh, bool split, int c_first, int c_last, int cta) {
+  float acc[kHalf];
+  tc::tmem_ld32(tacc + hh * kHalf, acc);
+  tc::tmem_wait_ld();
+  if (split) {
+    float sum[kHalf];
+#pragma unroll
+    for (int c = 0; c < kHalf; ++c) sum[c] = 0.f;
+    for (int cc0 = c_first; cc0 <= c_last; cc0 += kPar) {
+      float4 pv[kPar][kHalf / 4];
+#pragma unroll
+      for (int u = 0; u < kPar; ++u) {
+        const int cc = cc0 + u;
+        if (cc <= c_last && cc != cta) {
+          const int sl = tile == stage_lo(cc, a) / a.nst ? 0 : 1;
+          const float4* pc = reinterpret_cast<const float4*>(
+              a.part + ((static_cast<size_t>(cc) * 2 + sl) * kTileRows + r) * kN + hh * kHalf);
+#pragma unroll
+          for (int e = 0; e < kHalf / 4; ++e) pv[u][e] = __ldcg(pc + e);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPar; ++u) {
+        const int cc = cc0 + u;
+        if (cc <= c_last) {
+#pragma unroll
+          for (int e = 0; e < kHalf / 4; ++e) {
+            const float4 v = cc == cta ? make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3])
+                                       : pv[u][e];
+            sum[4 * e] += v.x;
+            sum[4 * e + 1] += v.y;
+            sum[4 * e + 2] += v.z;
+            sum[4 * e + 3] += v.w;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < kHalf; ++c) acc[c] = sum[c];
+  }
+  epilogue_half<kMode, kN>(a, bs, tile, r, hh * kHalf, acc);
+}
+
 template <int kMode, int kN>
 __global__ void __launch_bounds__(kThreads, 1)
     wgemm_kernel(const __grid_constant__ CUtensorMap w_map, const __grid_constant__ CUtensorMap x_map,
@@ -253,6 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bs->acc_empty[b], 4);
     }
     mbar_init(&bs->mma_done, 1);
+    for (int qq = 0; qq < 4; ++qq) mbar_init(&bs->tail[qq], 1);
     bs->abort = 0;
     fence_barrier_init();
   }
@@ -367,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = 32 * q + lane;
     wait_prior_grids();   // the residual stream and the outputs of the kernels before
     int n = 0;
+    bool signalled = false;
     Unit x;
     for (int st = st_lo; next_unit(a, st, st_hi, x); ++n) {
       const int buf = n & 1;
@@ -402,55 +453,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         mine_last = __shfl_sync(0xffffffffu, last, 0) != 0;
         if (mine_last) __threadfence();
       }
+      // This CTA's final unit ends the kernel for it: when it finishes the
+      // tile, warp q of warps 0-3 (idle by now) takes the odd chunks.
+      const bool final_unit = st >= st_hi;
+      const bool help = final_unit && mine_last && kN / kHalf >= 2;
+      if (final_unit) {
+        if (lane == 0) {
+          bs->tail_n[q] = help ? n : -1;
+          tc::mbar_arrive(&bs->tail[q]);
+        }
+        signalled = true;
+      }
       if (mine_last) {
 #pragma unroll 1
-        for (int hh = 0; hh < kN / kHalf; ++hh) {
-          float acc[kHalf];
-          tc::tmem_ld32(tacc + hh * kHalf, acc);
-          tc::tmem_wait_ld();
-          if (split) {
-            // The parts in CTA order, kPar CTAs' loads in flight at a time.
-            float sum[kHalf];
-#pragma unroll
-            for (int c = 0; c < kHalf; ++c) sum[c] = 0.f;
-            for (int cc0 = c_first; cc0 <= c_last; cc0 += kPar) {
-              float4 pv[kPar][kHalf / 4];
-#pragma unroll
-              for (int u = 0; u < kPar; ++u) {
-                const int cc = cc0 + u;
-                if (cc <= c_last && cc != cta) {
-                  const int sl = x.tile == stage_lo(cc, a) / a.nst ? 0 : 1;
-                  const float4* pc = reinterpret_cast<const float4*>(
-                      a.part + ((static_cast<size_t>(cc) * 2 + sl) * kTileRows + r) * kN + hh * kHalf);
-#pragma unroll
-                  for (int e = 0; e < kHalf / 4; ++e) pv[u][e] = __ldcg(pc + e);
-                }
-              }
-#pragma unroll
-              for (int u = 0; u < kPar; ++u) {
-                const int cc = cc0 + u;
-                if (cc <= c_last) {
-#pragma unroll
-                  for (int e = 0; e < kHalf / 4; ++e) {
-                    const float4 v = cc == cta ? make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3])
-                                               : pv[u][e];
-                    sum[4 * e] += v.x;
-                    sum[4 * e + 1] += v.y;
-                    sum[4 * e + 2] += v.z;
-                    sum[4 * e + 3] += v.w;
-                  }
-                }
-              }
-            }
-#pragma unroll
-            for (int c = 0; c < kHalf; ++c) acc[c] = sum[c];
-          }
-          epilogue_half<kMode, kN>(a, bs, x.tile, r, hh * kHalf, acc);
-        }
+        for (int hh = 0; hh < kN / kHalf; hh += help ? 2 : 1)
+          finish_chunk<kMode, kN>(a, bs, x.tile, r, tacc, hh, split, c_first, c_last, cta);
       }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&bs->acc_empty[buf]);
+    }
+    if (!signalled && lane == 0) {   // no final unit reached (an abort): release the helper
+      bs->tail_n[q] = -1;
+      tc::mbar_arrive(&bs->tail[q]);
+    }
+  }
+  if (warp < 4) {
+    // Warps 0-3, done with their roles: warp q takes the odd chunks of the
+    // final unit of lane quarter q when the epilogue warp asks for help.
+    __syncwarp();
+    const int q = warp;
+    if (!mbar_wait(&bs->tail[q], 0)) {
+      set_device_status(a.status, MEDUSA_ERR_TIMEOUT, kDetailDecoderWait);
+      bs->abort = 1;
+    } else if (bs->tail_n[q] >= 0) {
+      const int nf = bs->tail_n[q];
+      wait_prior_grids();
+      tc::fence_after_sync();
+      const int tile = (st_hi - 1) / a.nst;
+      const int t0 = tile * a.nst;
+      const int c_first = stage_owner(t0, a), c_last = stage_owner(t0 + a.nst - 1, a);
+      const uint32_t tacc = tmem + (static_cast<uint32_t>(32 * q) << 16) + (nf & 1) * kN;
+#pragma unroll 1
+      for (int hh = 1; hh < kN / kHalf; hh += 2)
+        finish_chunk<kMode, kN>(a, bs, tile, 32 * q + lane, tacc, hh, c_first != c_last, c_first, c_last, cta);
     }
   }
   tc::fence_before_sync();
