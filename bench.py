@@ -673,7 +673,7 @@ def kernel_revision():
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(REPO, "speculative_decoding_heads_b200", "csrc")
-    for f in ("heads.cu", "common.cuh"):
+    for f in ("heads.cu", "heads_common.cuh", "common.cuh"):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:12]
 

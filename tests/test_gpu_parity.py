@@ -513,6 +513,55 @@ def test_step_host_matches_device_step(mb, dev):
     _status_clean(mb)
 
 
+def test_step_host_single_stream(mb, dev):
+    # With no copy stream every copy goes on the step's stream ahead of the
+    # step; the results equal the two-stream form's.
+    import ctypes
+    w = SMALL["v13b_small"]
+    sub_h, _, _ = pick_sub_h(w)
+    tree = _tree(mb, w)
+    t = dev.materialise(w, sub_h=sub_h)
+    dev.tree_outputs(t, w.B, tree.T, tree.P, tree.D)
+    args = mb.make_step_args(tree, t, mb.MEDUSA_GREEDY)
+    ws = mb.workspace(mb.medusa_step_workspace_size(args))
+    lens0 = t["seq_lens"].clone()
+    kc0, vc0 = t["k_cache"].clone(), t["v_cache"].clone()
+    pin = lambda x: x.cpu().pin_memory()
+    L = lens0.cpu()
+    host_in = {"h": pin(t["h"]), "root_tokens": pin(t["root_tokens"]), "seq_lens": pin(lens0),
+               "q": pin(t["q"]), "base_logits": pin(t["base_logits"]),
+               "k_tree": pin(torch.stack([kc0[:, b, :, int(L[b]):int(L[b]) + w.T] for b in range(w.B)], 1)),
+               "v_tree": pin(torch.stack([vc0[:, b, :, int(L[b]):int(L[b]) + w.T] for b in range(w.B)], 1))}
+    outs = []
+    for single in (False, True):
+        t["seq_lens"].copy_(lens0)
+        t["k_cache"].copy_(kc0)
+        t["v_cache"].copy_(vc0)
+        host_out = {k: torch.full_like(t[k], -7, device="cpu").pin_memory()
+                    for k in ("best_path", "accept_len", "accepted_tokens", "next_token", "seq_lens")}
+        stream = torch.cuda.Stream()
+        if single:
+            io = mb.StepHostIO()
+            for k, x in host_in.items():
+                setattr(io, k, x.data_ptr())
+            for k, x in host_out.items():
+                setattr(io, "seq_lens_out" if k == "seq_lens" else k, x.data_ptr())
+            io.copy_stream = None
+            st = mb._lib.medusa_step_host(ctypes.byref(args), ctypes.byref(io), ws.data_ptr(), ws.numel(),
+                                          stream.cuda_stream)
+            assert st == mb.MEDUSA_OK, mb._lib.medusa_last_error()
+        else:
+            mb.medusa_step_host(args, ws, host_in, host_out, stream)
+        stream.synchronize()
+        outs.append((host_out, t["k_cache"].clone(), t["attn_out"].clone()))
+    for k in outs[0][0]:
+        assert torch.equal(outs[0][0][k], outs[1][0][k]), k
+    assert (outs[1][0]["accept_len"] >= 0).all()
+    assert torch.equal(outs[0][1], outs[1][1])
+    assert torch.equal(outs[0][2], outs[1][2])
+    _status_clean(mb)
+
+
 def test_step_host_refuses_device_buffers_and_overflow(mb, dev):
     # io must hold host memory; a host length that would put the tree rows
     # past Lcap is refused; both before anything is enqueued.
