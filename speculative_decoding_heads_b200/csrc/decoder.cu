@@ -13,9 +13,9 @@
 // tokens): the weights stream from HBM once per pass, as the A operand of
 // M = 128, N = kN, K = 16 tcgen05 products (TMA boxes of 128 rows x 64
 // columns, 128-byte swizzle, no multicast), the tokens' activations are the
-// B operand, and the fp32 accumulators live in tensor memory.  A pass holds
-// 64, 128 or 256 tokens (the smallest that takes all of them, else 256); a
-// ring stage holds 2 column blocks of 64 at 64 tokens and 1 above.  The
+// B operand, and the fp32 accumulators live in tensor memory.  Passes hold
+// 256 tokens, and the last one the smallest of 64, 128 and 256 that takes the
+// rest; a ring stage holds 2 column blocks of 64 at 64 tokens and 1 above.  The
 // ring stages of a product are split evenly over the CTAs (stream-K); a tile
 // of 128 rows cut by a range boundary is summed, per quarter of its rows, by
 // the last CTA to finish it, in CTA order.  The epilogue is fused per
@@ -588,8 +588,8 @@ bool encode_w(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void*
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tokens per pass for a forward over ntok tokens: the smallest of 64, 128
-// and 256 that takes all of them, else 256.
+// Tokens in a pass over ntok remaining tokens: the smallest of 64, 128 and
+// 256 that takes all of them, else 256.
 int tokens_per_pass(int ntok) { return ntok <= 64 ? 64 : (ntok <= 128 ? 128 : kMaxN); }
 
 // Scratch of the matrix products: tile counters, then [G, 2, 128, kN] partials.
@@ -624,18 +624,26 @@ medusa_status_t gemm_n(const void* Wt, const uint16_t* X, GemmArgs a, void* ws, 
     return fail(MEDUSA_ERR_UNSUPPORTED, "medusa_tree_decode: tensor map rejected");
   auto fn = wgemm_kernel<kMode, kN>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-  for (a.tok0 = 0; e == cudaSuccess && a.tok0 < a.ntok; a.tok0 += kN)
+  if (e == cudaSuccess)
     e = launch_kernel(fn, dim3(a.G), dim3(kThreads), static_cast<size_t>(C::kSmem), stream, true, wm, xm, a);
   return e == cudaSuccess ? MEDUSA_OK : cuda_fail("medusa_tree_decode: matrix-product launch", e);
 }
 
+// Passes of 256 tokens, then one pass for the rest in the smallest of 64,
+// 128 and 256 tokens that holds it (a pass costs roughly in proportion to its
+// width from 128 tokens up, so a narrow last pass saves most of a wide one).
 template <int kMode>
 medusa_status_t gemm(const void* Wt, const uint16_t* X, GemmArgs a, void* ws, cudaStream_t stream) {
-  switch (tokens_per_pass(a.ntok)) {
-    case 64: return gemm_n<kMode, 64>(Wt, X, a, ws, stream);
-    case 128: return gemm_n<kMode, 128>(Wt, X, a, ws, stream);
-    default: return gemm_n<kMode, kMaxN>(Wt, X, a, ws, stream);
+  for (int tok0 = 0; tok0 < a.ntok;) {
+    const int n = tokens_per_pass(a.ntok - tok0);
+    a.tok0 = tok0;
+    const medusa_status_t st = n == 64    ? gemm_n<kMode, 64>(Wt, X, a, ws, stream)
+                               : n == 128 ? gemm_n<kMode, 128>(Wt, X, a, ws, stream)
+                                          : gemm_n<kMode, kMaxN>(Wt, X, a, ws, stream);
+    if (st != MEDUSA_OK) return st;
+    tok0 += n;
   }
+  return MEDUSA_OK;
 }
 
 }  // namespace

@@ -196,11 +196,18 @@ def test_tree_attention_many_slices(mb, dev, shape):
 
 
 @pytest.mark.parametrize("variant", ["T200_two_row_groups", "T256_max", "T100_L0", "hd64_bf16_generic",
-                                     "hd256_f32", "chain_L0", "exact_capacity"])
+                                     "hd256_f32", "chain_L0", "exact_capacity", "T129_tail", "T130_tail",
+                                     "T130_tail_L0"])
 def test_tree_attention_edges(mb, dev, variant):
     base = SMALL["v7b_small"]
     from synth.workloads import shrink
-    if variant == "T200_two_row_groups":
+    if variant.startswith("T129_tail") or variant.startswith("T130_tail"):
+        # one or two rows past a 128-row group: a 128-row pass and a 64-row pass
+        n = 128 if variant.startswith("T129") else 129
+        w = shrink(base, K=5, topk=10, n_nodes=n, prefix=0 if variant.endswith("L0") else 201, layers=2, H=3)
+        assert w.T == n + 1
+        _attention_case(mb, dev, w)
+    elif variant == "T200_two_row_groups":
         w = shrink(base, K=5, topk=10, n_nodes=199, prefix=70, layers=1, H=2)
         _attention_case(mb, dev, w)
     elif variant == "T256_max":
