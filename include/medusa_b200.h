@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define MEDUSA_ABI_VERSION 5
+#define MEDUSA_ABI_VERSION 6
 #define MEDUSA_MAX_T 256     /* tree tokens including the root */
 #define MEDUSA_MAX_K 16      /* heads (so tree depth <= 16) */
 #define MEDUSA_MAX_TOPK 32   /* candidates per head */
@@ -434,6 +434,38 @@ medusa_status_t medusa_tree_decode(const medusa_tree_t* tree, const medusa_decod
                                    const int32_t* tree_tokens, void* k_cache, void* v_cache, int Lcap,
                                    const int32_t* seq_lens, float* logits, float* hidden, void* workspace,
                                    size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Greedy generation                                                         */
+/* ------------------------------------------------------------------------ */
+
+size_t medusa_generate_workspace_size(const medusa_tree_t* tree, const medusa_decoder_t* model);
+
+/* Greedy Medusa decoding of one sequence ("Medusa API参考", MedusaModelABC
+ * medusa_generate; "Medusa — 让大模型自己同时猜好几个 token", 实践案例 case 1
+ * and 学到什么): the prompt (HOST, n_prompt tokens) goes through the base
+ * model in chains of at most 17 tokens, writing cache rows 0 .. n_prompt-1;
+ * the base model's arg-max after it is the first root.  Each step then runs
+ * the K heads (W1 [K, D, D], b1 [K, D], Wout [K, V, D], bf16, device) on the
+ * final-norm hidden state of the last accepted token, builds the candidate
+ * tree rooted at the base model's next token, runs the base model over the
+ * tree tokens (medusa_tree_decode), accepts greedily, compacts the accepted
+ * K/V rows and emits root + accepted tokens.  Caches [layers, 1, H, Lcap,
+ * 128] bf16 on the device; their content is overwritten from row 0.
+ * out_tokens (HOST, n_new entries) receives the first n_new emitted tokens,
+ * out_accept (HOST, max_steps entries) each step's accept length, *n_steps
+ * the number of steps.  The host waits for every step (it reads the accept
+ * length).  Workspace zero-filled before its first use (counters reset
+ * themselves).  INVALID_ARG when the prompt plus one tree does not fit in
+ * Lcap, a prompt token is outside [0, V), or the cache or max_steps ran out
+ * before n_new tokens (the tokens so far are written). */
+medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, const medusa_decoder_t* model,
+                                       const void* W1, const void* b1, const void* Wout,
+                                       const int32_t* prompt, int n_prompt, int n_new,
+                                       void* k_cache, void* v_cache, int Lcap,
+                                       int32_t* out_tokens, int32_t* out_accept, int max_steps,
+                                       int32_t* n_steps, void* workspace, size_t workspace_bytes,
+                                       cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* The whole step                                                            */

@@ -26,7 +26,7 @@ if not os.path.exists(LIB_PATH):
         "`python -m speculative_decoding_heads_b200._build` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
-ABI_VERSION = 5   # layout of medusa_step_args_t (StepArgs below) and of every signature
+ABI_VERSION = 6   # layout of medusa_step_args_t (StepArgs below) and of every signature
 _lib.medusa_abi_version.restype = ctypes.c_int
 if _lib.medusa_abi_version() != ABI_VERSION:
     raise ImportError(f"{LIB_PATH} has ABI version {_lib.medusa_abi_version()}, this binding needs "
@@ -58,6 +58,7 @@ EXPORTED = [
     "medusa_accept_kv",
     "medusa_decoder_pack_rows", "medusa_tree_decode_workspace_size", "medusa_tree_decode",
     "medusa_step_workspace_size", "medusa_step", "medusa_step_host",
+    "medusa_generate_workspace_size", "medusa_generate_greedy",
 ]
 
 _vp = ctypes.c_void_p
@@ -147,6 +148,9 @@ _sig("medusa_decoder_pack_rows", _i32, [_i32, _i32, _pi32])
 _sig("medusa_tree_decode_workspace_size", _sz, [_vp, ctypes.POINTER(DecoderModel), _i32])
 _sig("medusa_tree_decode", _i32, [_vp, ctypes.POINTER(DecoderModel), _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp,
                                    _sz, _vp])
+_sig("medusa_generate_workspace_size", _sz, [_vp, ctypes.POINTER(DecoderModel)])
+_sig("medusa_generate_greedy", _i32, [_vp, ctypes.POINTER(DecoderModel), _vp, _vp, _vp, _pi32, _i32, _i32, _vp, _vp,
+                                      _i32, _pi32, _pi32, _i32, _pi32, _vp, _sz, _vp])
 _sig("medusa_step_workspace_size", _sz, [ctypes.POINTER(StepArgs)])
 _sig("medusa_step", _i32, [ctypes.POINTER(StepArgs), _vp, _sz, _vp])
 _sig("medusa_step_host", _i32, [ctypes.POINTER(StepArgs), ctypes.POINTER(StepHostIO), _vp, _sz, _vp])
@@ -550,6 +554,42 @@ def medusa_tree_decode(tree: Tree, model: Decoder, tree_tokens, k_cache, v_cache
     nbytes = _nbytes("ws", ws)
     _check(_lib.medusa_tree_decode(tree.handle, ctypes.byref(model.c), B, _p(tree_tokens), _p(k_cache), _p(v_cache),
                                    Lcap, _p(seq_lens), _p(logits), _p(hidden), _p(ws), nbytes, _stream(stream)))
+
+
+def medusa_generate_workspace_size(tree: Tree, model: Decoder) -> int:
+    return int(_lib.medusa_generate_workspace_size(tree.handle, ctypes.byref(model.c)))
+
+
+def medusa_generate_greedy(tree: Tree, model: Decoder, W1, b1, Wout, prompt, n_new: int, k_cache, v_cache,
+                           ws=None, max_steps=None, stream=None):
+    """Greedy Medusa decoding of one sequence (``medusa_generate_greedy``): prompt (host ints),
+    heads W1 [K, D, D], b1 [K, D], Wout [K, V, D] bf16 with K = tree.K, caches [layers, 1, H, Lcap,
+    128] bf16 (overwritten from row 0).  Returns (the first n_new emitted tokens, the accept length
+    of every step)."""
+    K, D, V = tree.K, model.D, model.V
+    _spec("W1", W1, (K, D, D), torch.bfloat16)
+    _spec("b1", b1, (K, D), torch.bfloat16)
+    _spec("Wout", Wout, (K, V, D), torch.bfloat16)
+    _require(k_cache.dim() == 5, "caches must be [layers, 1, H, Lcap, 128]")
+    Lcap = k_cache.shape[3]
+    shape = (len(model.tensors), 1, D // 128, Lcap, 128)
+    _spec("k_cache", k_cache, shape, torch.bfloat16)
+    _spec("v_cache", v_cache, shape, torch.bfloat16)
+    prompt = [int(x) for x in prompt]
+    _require(len(prompt) >= 1 and n_new >= 1, "the prompt and n_new must be non-empty")
+    max_steps = int(max_steps if max_steps is not None else n_new)
+    if ws is None:
+        ws = workspace(medusa_generate_workspace_size(tree, model))
+    nbytes = _nbytes("ws", ws)
+    pr = (ctypes.c_int32 * len(prompt))(*prompt)
+    out = (ctypes.c_int32 * n_new)()
+    acc = (ctypes.c_int32 * max_steps)()
+    n = ctypes.c_int32(0)
+    st = _lib.medusa_generate_greedy(tree.handle, ctypes.byref(model.c), _p(W1), _p(b1), _p(Wout), pr, len(prompt),
+                                     int(n_new), _p(k_cache), _p(v_cache), Lcap, out, acc, max_steps,
+                                     ctypes.byref(n), _p(ws), nbytes, _stream(stream))
+    _check(st)
+    return list(out), list(acc[:n.value])
 
 
 def make_step_args(tree: Tree, t: dict, mode: int, temperature=0.0, eps=0.09, alpha=0.3,

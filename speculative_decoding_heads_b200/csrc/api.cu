@@ -360,7 +360,7 @@ extern "C" medusa_status_t medusa_decoder_pack_rows(int which, int n, int32_t* o
   return MEDUSA_OK;
 }
 
-static medusa_status_t check_decoder(const medusa_tree_t* tree, const medusa_decoder_t* m, int B, const char* fn) {
+medusa_status_t medusa::check_decoder(const medusa_tree_t* tree, const medusa_decoder_t* m, int B, const char* fn) {
   medusa_status_t st = check_tree(tree, fn);
   if (st != MEDUSA_OK) return st;
   if (!m || !m->layer || !m->embed || !m->final_norm || !m->lm_head)

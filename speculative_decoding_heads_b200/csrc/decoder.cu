@@ -648,6 +648,13 @@ medusa_status_t gemm(const void* Wt, const uint16_t* X, GemmArgs a, void* ws, cu
 
 }  // namespace
 
+uint16_t* decoder_final_rows(void* ws, int ntok, int D, int F, int V) {
+  // the layout of launch_tree_decode: the products' scratch, x, then xn (which
+  // holds the final RMSNorm's output once the forward is done)
+  const size_t o = gemm_scratch_bytes(D, F, V, ntok) + align_up(static_cast<size_t>(ntok) * D * 4, 256);
+  return reinterpret_cast<uint16_t*>(static_cast<unsigned char*>(ws) + o);
+}
+
 size_t decoder_workspace_bytes(int ntok, int D, int F, int V) {
   // The products' scratch; then x fp32, xn bf16, q bf16, attention fp32 and bf16, act bf16.
   size_t o = gemm_scratch_bytes(D, F, V, ntok);

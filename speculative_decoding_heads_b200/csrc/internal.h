@@ -65,6 +65,9 @@ medusa_status_t check_heads(const void* h, const void* W1, const void* b1, const
 // Every host-side check of medusa_step (api.cu); nothing is enqueued.
 medusa_status_t check_step(const medusa_step_args_t* args, const void* ws, size_t ws_bytes);
 
+// Host-side checks of the base model and the tree for medusa_tree_decode (api.cu).
+medusa_status_t check_decoder(const medusa_tree_t* tree, const medusa_decoder_t* m, int B, const char* fn);
+
 // Kernel launchers (heads.cu, tree_kernels.cu, attention.cu, posterior.cu, accept.cu).
 size_t heads_workspace_bytes(int B, int d, int V, int K, int topk);
 medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, const void* Wout,
@@ -134,6 +137,8 @@ medusa_status_t launch_topk_merge(const float* vals, const int32_t* ids, const i
 
 // The tree-token forward of the base model (decoder.cu).
 size_t decoder_workspace_bytes(int ntok, int D, int F, int V);
+// The final RMSNorm's bf16 output rows [ntok, D] inside a forward's workspace.
+uint16_t* decoder_final_rows(void* ws, int ntok, int D, int F, int V);
 medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, int B, const int32_t* tree_tokens,
                                    void* k_cache, void* v_cache, int Lcap, const int32_t* seq_lens,
                                    float* logits, float* hidden, void* ws, cudaStream_t stream);
