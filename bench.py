@@ -638,11 +638,20 @@ def time_tree_decode(a, w, t, tree, mb, stream, peak, world):
                                      t["accept_len"], t["accepted_tokens"], t["next_token"], t["_pws"])
         mb.medusa_accept_kv(tree, t["k_cache"], t["v_cache"], t["seq_lens"], t["best_path"], t["accept_len"])
 
+    # plain decoding's step for comparison: the base model's forward over one token per sequence
+    root_tree = mb.Tree([], 1, 1)
+    one_tok = t["tree_tokens"][:, :1].contiguous()
+    one_logits = torch.empty((w.B, V), device="cuda")
+    one_ws = mb.workspace(mb.medusa_tree_decode_workspace_size(root_tree, model, w.B))
+
+    def one_token():
+        mb.medusa_tree_decode(root_tree, model, one_tok, t["k_cache"], t["v_cache"], lens, one_logits, one_ws)
+
     t["_hws"] = mb.workspace(mb.medusa_heads_workspace_size(w.B, w.d, w.V, w.K, w.topk))
     t["_pws"] = mb.workspace(mb.medusa_posterior_workspace_size(tree, w.B))
     res = {}
     with torch.cuda.stream(stream):
-        for name, fn in (("forward", fwd), ("full_step", full_step)):
+        for name, fn in (("forward", fwd), ("full_step", full_step), ("one_token", one_token)):
             for _ in range(max(3, a.warmup)):
                 fn()
             torch.cuda.synchronize()
@@ -662,10 +671,14 @@ def time_tree_decode(a, w, t, tree, mb, stream, peak, world):
     fwd_us = res["forward"]["median"]
     return {"layers": w.layers, "D": D, "F": F, "V": V, "tokens": ntok, "weights_bytes": wbytes, "kv_bytes": kv_bytes,
             "forward_us": res["forward"], "full_step_us": res["full_step"],
+            "one_token_forward_us": res["one_token"],
+            # accepted tokens per step (the root included) above which a Medusa step beats plain decoding
+            "break_even_tokens_per_step": res["full_step"]["median"] / res["one_token"]["median"],
             "forward_gbs": (wbytes + kv_bytes) / (fwd_us * 1e-6) / 1e9,
             "forward_frac": (wbytes + kv_bytes) / (fwd_us * 1e-6) / 1e9 / peak,
             "note": "random bf16 weights of the base model's shape; the full step's acceptance is meaningless "
-                    "with random weights, so tokens per step are not reported"}
+                    "with random weights, so tokens per step are not reported; one_token_forward is plain "
+                    "decoding's step (one token per sequence at the same cache length)"}
 
 
 def kernel_revision():
