@@ -132,11 +132,12 @@ __device__ __forceinline__ void tma_load_1d(void* dst_smem, const void* src, uin
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// fp32 -> bf16, round to nearest even: one conversion instruction, no branch
+// (a data-dependent branch per value serialised the epilogues' unrolled loops).
 __device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
-  uint32_t b = __float_as_uint(f);
-  if ((b & 0x7f800000u) == 0x7f800000u) return static_cast<uint16_t>((b >> 16) | ((b & 0xffffu) ? 0x40u : 0u));
-  b += 0x7fffu + ((b >> 16) & 1u);
-  return static_cast<uint16_t>(b >> 16);
+  uint16_t r;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(f));
+  return r;
 }
 
 // ---- acquire / release on global counters ---------------------------------
