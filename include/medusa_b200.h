@@ -515,9 +515,11 @@ size_t medusa_step_workspace_size(const medusa_step_args_t* args);
 /* The computations of medusa_heads_topk, medusa_build_tree,
  * medusa_tree_attention, medusa_evaluate_posterior and medusa_accept_kv, in
  * that order, on stream, with the same outputs.  The candidate tree is built
- * by the heads kernel's last CTA (one launch for S1-S4 per group of up to
- * four sequences), and the posterior and the compaction share one launch
- * (S6-S7): three launches per step at B <= 4.  Capturable in a CUDA graph
+ * by the heads' last CTA: S1-S4 take one launch at batch 1 (and per group of
+ * up to four sequences for fp32), two per pass of up to 16 sequences on the
+ * tensor cores (bf16, B >= 2).  Tree attention takes one launch (two for
+ * trees of 129-192 tokens), and the posterior and the compaction share one (S6-S7):
+ * three launches per step at batch 1.  Capturable in a CUDA graph
  * (no allocation, no synchronisation).  Validation errors are returned
  * before anything is enqueued. */
 medusa_status_t medusa_step(const medusa_step_args_t* args, void* workspace,
