@@ -30,11 +30,19 @@ __global__ void set_len_kernel(int32_t* seq_lens, int L) { seq_lens[0] = L; }
 // accepted node (retrieve[best, a]) or `fixed_row`; with root set, also the
 // arg-max of that row's logits (lower id on ties).  One CTA of 256 threads.
 __global__ void next_input_kernel(const uint16_t* rows, const float* logits, int D, int V, int fixed_row,
-                                  const int32_t* retrieve, int dp1, const int32_t* best, const int32_t* alen,
-                                  uint16_t* h, int32_t* root) {
+                                  const int32_t* retrieve, int P, int dp1, const int32_t* best, const int32_t* alen,
+                                  uint16_t* h, int32_t* root, int* status) {
   __shared__ float sv[8];
   __shared__ int si[8];
-  const int row = retrieve ? retrieve[best[0] * dp1 + alen[0]] : fixed_row;
+  int row = fixed_row;
+  if (retrieve) {
+    const int bp = best[0], a = alen[0];
+    row = (bp >= 0 && bp < P && a >= 0 && a < dp1) ? retrieve[bp * dp1 + a] : -1;
+    if (row < 0) {   // the step's outputs are not a path: leave h alone
+      if (threadIdx.x == 0) set_device_status(status, MEDUSA_ERR_DEVICE_CHECK, kDetailPosteriorArgs);
+      return;
+    }
+  }
   for (int i = threadIdx.x; i < D; i += blockDim.x) h[i] = rows[static_cast<size_t>(row) * D + i];
   if (!root) return;
   float bv = -INFINITY;
@@ -186,7 +194,7 @@ extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, con
     last_n = n;
   }
   next_input_kernel<<<1, 256, 0, stream>>>(decoder_final_rows(ws_dec, last_n, D, model->F, V), logits, D, V,
-                                           last_n - 1, nullptr, 0, nullptr, nullptr, h, root);
+                                           last_n - 1, nullptr, 0, 0, nullptr, nullptr, h, root, device_status_ptr());
   set_len_kernel<<<1, 1, 0, stream>>>(seq_len, L);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("medusa_generate_greedy: launch", e);
@@ -214,7 +222,8 @@ extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, con
                                  ws_post, stream, false);
     if (st != MEDUSA_OK) return st;
     next_input_kernel<<<1, 256, 0, stream>>>(decoder_final_rows(ws_dec, tree->T, D, model->F, V), logits, D, V, 0,
-                                             tree->dev.retrieve, dp1, best, alen, h, nullptr);
+                                             tree->dev.retrieve, tree->P, dp1, best, alen, h, nullptr,
+                                             device_status_ptr());
     e = cudaMemcpyAsync(host.data(), alen, 4, cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaMemcpyAsync(host.data() + 1, acc, static_cast<size_t>(dp1) * 4, cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
