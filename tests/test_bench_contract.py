@@ -50,3 +50,28 @@ def test_reference_line_config_names_the_workload(line):
     assert cfg["workload"] == "tiny_f32"
     assert "model" not in cfg
     assert "fit in L2" in cfg["l2"]        # 4 MB of inputs: said plainly, not claimed to exceed L2
+
+
+def test_launch_plan_matches_the_counted_graph_nodes():
+    # The launch counts the benchmark's plan gives where the captured step graph cannot be
+    # queried; the kernel nodes counted on a B200 were 3 (c1, c2, c0), 4 (c3, c4 N16-N64) and
+    # 5 (c4 N128: a 128-row and a 64-row attention launch).
+    sys.path.insert(0, REPO)
+    import bench
+    from synth import workloads as W
+    for name, n in [("vicuna7b_bs1_L1024", 3), ("vicuna7b_bs1_L4096_typical", 3), ("tiny_f32", 3),
+                    ("vicuna13b_bs8_ragged", 4), ("vicuna33b_bs4_L8192_N16", 4), ("vicuna33b_bs4_L8192_N64", 4),
+                    ("vicuna33b_bs4_L8192_N128", 5)]:
+        w = W.get(name)
+        assert bench.expected_launches(w, w.T) == n, name
+    w = W.shrink(W.get("vicuna13b_bs8_ragged"), name="b17", B=17)
+    assert bench.expected_launches(w, w.T) == 2 * 2 + 1 + 1   # two tensor-core passes
+
+
+def test_kernel_short_name():
+    sys.path.insert(0, REPO)
+    import bench
+    assert bench._kernel_short_name("_ZN6medusa12_GLOBAL__N_115heads_tc_kernelILi1ELi16EEEvNS0_4ArgsE") == \
+        "heads_tc_kernel"
+    assert bench._kernel_short_name("_ZN6medusa16posterior_kernelILi0EEEvNS_8PostArgsE") == "posterior_kernel"
+    assert bench._kernel_short_name("plain_name") == "plain_name"
