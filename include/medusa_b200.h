@@ -71,7 +71,7 @@
 extern "C" {
 #endif
 
-#define MEDUSA_ABI_VERSION 6
+#define MEDUSA_ABI_VERSION 7
 #define MEDUSA_MAX_T 256     /* tree tokens including the root */
 #define MEDUSA_MAX_K 16      /* heads (so tree depth <= 16) */
 #define MEDUSA_MAX_TOPK 32   /* candidates per head */
@@ -459,6 +459,22 @@ size_t medusa_generate_workspace_size(const medusa_tree_t* tree, const medusa_de
  * themselves).  INVALID_ARG when the prompt plus one tree does not fit in
  * Lcap, a prompt token is outside [0, V), or the cache or max_steps ran out
  * before n_new tokens (the tokens so far are written). */
+/* medusa_generate_greedy's loop with acceptance in `mode` (MEDUSA_GREEDY,
+ * MEDUSA_TYPICAL or MEDUSA_NUCLEUS, with temperature, eps, alpha and top_p as
+ * medusa_evaluate_posterior; "Medusa API参考", MedusaModelABC medusa_generate:
+ * sampling and top_p).  uniforms (HOST, max_steps entries in [0, 1), or NULL)
+ * gives step s's draw of the next token (see medusa_evaluate_posterior); the
+ * first root, after the prompt, is the base model's arg-max.  Errors as
+ * medusa_generate_greedy, plus medusa_evaluate_posterior's argument checks
+ * and uniforms outside [0, 1). */
+medusa_status_t medusa_generate(const medusa_tree_t* tree, const medusa_decoder_t* model,
+                                const void* W1, const void* b1, const void* Wout, medusa_mode_t mode,
+                                float temperature, float eps, float alpha, float top_p,
+                                const float* uniforms, const int32_t* prompt, int n_prompt, int n_new,
+                                void* k_cache, void* v_cache, int Lcap, int32_t* out_tokens,
+                                int32_t* out_accept, int max_steps, int32_t* n_steps, void* workspace,
+                                size_t workspace_bytes, cudaStream_t stream);
+
 medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, const medusa_decoder_t* model,
                                        const void* W1, const void* b1, const void* Wout,
                                        const int32_t* prompt, int n_prompt, int n_new,

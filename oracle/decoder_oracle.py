@@ -143,13 +143,18 @@ def greedy_decode(model, prompt, n_new: int, Lcap: int):
     return out
 
 
-def medusa_generate_greedy(model, heads, choices, K: int, topk: int, prompt, n_new: int, Lcap: int):
-    """Greedy Medusa decoding of one sequence, built from the step's oracle functions.
+def medusa_generate(model, heads, choices, K: int, topk: int, prompt, n_new: int, Lcap: int, mode: str = "greedy",
+                    temperature: float = 0.0, eps: float = 0.09, alpha: float = 0.3, top_p: float = 0.8,
+                    uniforms=None, trace=None):
+    """Medusa decoding of one sequence, built from the step's oracle functions.
 
-    After the prompt's forward, each step: the heads on the last accepted token's final hidden
-    state (after the final RMSNorm), their top-k, the candidate tree rooted at the base model's own
-    next token, the base model's forward over the tree at the cache length (S5 inside it), greedy
-    acceptance, and the KV compaction.  The step emits the root and the a accepted tokens.
+    After the prompt's forward, the base model's arg-max is the first root.  Each step: the heads
+    on the last accepted token's final hidden state (after the final RMSNorm), their top-k, the
+    candidate tree rooted at the base model's next token, the base model's forward over the tree at
+    the cache length (S5 inside it), acceptance in ``mode`` (greedy, typical or nucleus, as
+    ``evaluate_posterior``; with ``uniforms[s]`` the next token of step s is drawn), and the KV
+    compaction.  The step emits the root and the a accepted tokens.  ``trace``, when a list, gets
+    (logits [T, V], candidates [P, D+1], best path, accept length, head logits [K, V]) of every step.
     Returns (tokens [n_new], accept length of every step)."""
     tr = O.tree_tables(choices, K, topk)
     kcs, vcs = _empty_caches(model, Lcap)
@@ -165,8 +170,11 @@ def medusa_generate_greedy(model, heads, choices, K: int, topk: int, prompt, n_n
         ids, _ = O.topk_desc(z, topk)
         toks, cand, _ = O.build_tree(tr, [root], ids, [L])
         logits, x, kcs, vcs = _forward(model, tr, toks[0], kcs, vcs, L)
-        post = O.evaluate_posterior(tr, logits[None], cand, "greedy")
+        u = None if uniforms is None else np.asarray([uniforms[len(accepts)]], dtype=np.float64)
+        post = O.evaluate_posterior(tr, logits[None], cand, mode, temperature, eps, alpha, top_p, u)
         a, best = int(post["accept_len"][0]), int(post["best_path"][0])
+        if trace is not None:
+            trace.append((logits, cand[0], best, a, z[0]))
         k_new, v_new, _ = O.accept_kv(tr, np.stack(kcs)[:, None], np.stack(vcs)[:, None], [L], [best], [a])
         kcs = [k_new[l, 0] for l in range(len(kcs))]
         vcs = [v_new[l, 0] for l in range(len(vcs))]
@@ -177,3 +185,9 @@ def medusa_generate_greedy(model, heads, choices, K: int, topk: int, prompt, n_n
         L += a + 1
         accepts.append(a)
     return out[:n_new], accepts
+
+
+def medusa_generate_greedy(model, heads, choices, K: int, topk: int, prompt, n_new: int, Lcap: int):
+    """Greedy Medusa decoding of one sequence (``medusa_generate`` in greedy mode).
+    Returns (tokens [n_new], accept length of every step)."""
+    return medusa_generate(model, heads, choices, K, topk, prompt, n_new, Lcap)

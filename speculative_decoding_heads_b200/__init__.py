@@ -26,7 +26,7 @@ if not os.path.exists(LIB_PATH):
         "`python -m speculative_decoding_heads_b200._build` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
-ABI_VERSION = 6   # layout of medusa_step_args_t (StepArgs below) and of every signature
+ABI_VERSION = 7   # layout of medusa_step_args_t (StepArgs below) and of every signature
 _lib.medusa_abi_version.restype = ctypes.c_int
 if _lib.medusa_abi_version() != ABI_VERSION:
     raise ImportError(f"{LIB_PATH} has ABI version {_lib.medusa_abi_version()}, this binding needs "
@@ -58,7 +58,7 @@ EXPORTED = [
     "medusa_accept_kv",
     "medusa_decoder_pack_rows", "medusa_tree_decode_workspace_size", "medusa_tree_decode",
     "medusa_step_workspace_size", "medusa_step", "medusa_step_host",
-    "medusa_generate_workspace_size", "medusa_generate_greedy",
+    "medusa_generate_workspace_size", "medusa_generate_greedy", "medusa_generate",
 ]
 
 _vp = ctypes.c_void_p
@@ -151,6 +151,9 @@ _sig("medusa_tree_decode", _i32, [_vp, ctypes.POINTER(DecoderModel), _i32, _vp, 
 _sig("medusa_generate_workspace_size", _sz, [_vp, ctypes.POINTER(DecoderModel)])
 _sig("medusa_generate_greedy", _i32, [_vp, ctypes.POINTER(DecoderModel), _vp, _vp, _vp, _pi32, _i32, _i32, _vp, _vp,
                                       _i32, _pi32, _pi32, _i32, _pi32, _vp, _sz, _vp])
+_sig("medusa_generate", _i32, [_vp, ctypes.POINTER(DecoderModel), _vp, _vp, _vp, _i32, _f32, _f32, _f32, _f32,
+                               ctypes.POINTER(ctypes.c_float), _pi32, _i32, _i32, _vp, _vp, _i32, _pi32, _pi32, _i32,
+                               _pi32, _vp, _sz, _vp])
 _sig("medusa_step_workspace_size", _sz, [ctypes.POINTER(StepArgs)])
 _sig("medusa_step", _i32, [ctypes.POINTER(StepArgs), _vp, _sz, _vp])
 _sig("medusa_step_host", _i32, [ctypes.POINTER(StepArgs), ctypes.POINTER(StepHostIO), _vp, _sz, _vp])
@@ -562,7 +565,16 @@ def medusa_generate_workspace_size(tree: Tree, model: Decoder) -> int:
 
 def medusa_generate_greedy(tree: Tree, model: Decoder, W1, b1, Wout, prompt, n_new: int, k_cache, v_cache,
                            ws=None, max_steps=None, stream=None):
-    """Greedy Medusa decoding of one sequence (``medusa_generate_greedy``): prompt (host ints),
+    """``medusa_generate`` in greedy mode."""
+    return medusa_generate(tree, model, W1, b1, Wout, prompt, n_new, k_cache, v_cache, MEDUSA_GREEDY, ws=ws,
+                           max_steps=max_steps, stream=stream)
+
+
+def medusa_generate(tree: Tree, model: Decoder, W1, b1, Wout, prompt, n_new: int, k_cache, v_cache,
+                    mode: int = MEDUSA_GREEDY, temperature=0.0, eps=0.09, alpha=0.3, top_p=0.8, uniforms=None,
+                    ws=None, max_steps=None, stream=None):
+    """Medusa decoding of one sequence (``medusa_generate``), acceptance in ``mode`` with the next
+    token of step s drawn with ``uniforms[s]`` (host floats, at least max_steps of them) if given: prompt (host ints),
     heads W1 [K, D, D], b1 [K, D], Wout [K, V, D] bf16 with K = tree.K, caches [layers, 1, H, Lcap,
     128] bf16 (overwritten from row 0).  Returns (the first n_new emitted tokens, the accept length
     of every step)."""
@@ -585,9 +597,15 @@ def medusa_generate_greedy(tree: Tree, model: Decoder, W1, b1, Wout, prompt, n_n
     out = (ctypes.c_int32 * n_new)()
     acc = (ctypes.c_int32 * max_steps)()
     n = ctypes.c_int32(0)
-    st = _lib.medusa_generate_greedy(tree.handle, ctypes.byref(model.c), _p(W1), _p(b1), _p(Wout), pr, len(prompt),
-                                     int(n_new), _p(k_cache), _p(v_cache), Lcap, out, acc, max_steps,
-                                     ctypes.byref(n), _p(ws), nbytes, _stream(stream))
+    uni = None
+    if uniforms is not None:
+        uniforms = [float(x) for x in uniforms]
+        _require(len(uniforms) >= max_steps, "uniforms needs one value per step (max_steps of them)")
+        uni = (ctypes.c_float * len(uniforms))(*uniforms)
+    st = _lib.medusa_generate(tree.handle, ctypes.byref(model.c), _p(W1), _p(b1), _p(Wout), int(mode),
+                              float(temperature), float(eps), float(alpha), float(top_p), uni, pr, len(prompt),
+                              int(n_new), _p(k_cache), _p(v_cache), Lcap, out, acc, max_steps,
+                              ctypes.byref(n), _p(ws), nbytes, _stream(stream))
     _check(st)
     return list(out), list(acc[:n.value])
 

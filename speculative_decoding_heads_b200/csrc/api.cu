@@ -273,7 +273,7 @@ extern "C" size_t medusa_posterior_workspace_size(const medusa_tree_t* tree, int
   return posterior_workspace_bytes(t, B);
 }
 
-static medusa_status_t check_posterior(const medusa_tree_t* tree, int B, int V, const float* logits,
+medusa_status_t medusa::check_posterior(const medusa_tree_t* tree, int B, int V, const float* logits,
                                        const int32_t* candidates, medusa_mode_t mode, float temperature,
                                        float eps, float alpha, float top_p, const int32_t* best_path,
                                        const int32_t* accept_len, const int32_t* accepted_tokens,

@@ -1,4 +1,5 @@
-// Greedy Medusa generation of one sequence on the GPU: the loop of
+// Medusa generation of one sequence on the GPU (greedy, typical or nucleus
+// acceptance, as medusa_evaluate_posterior): the loop of
 // "Medusa API参考：核心函数与类详解" (MedusaModelABC, medusa_generate: each step
 // proposes with the heads, verifies the tree with one base-model forward and
 // keeps the accepted prefix) and "Medusa — 让大模型自己同时猜好几个 token"
@@ -12,7 +13,8 @@
 //   the candidate tree rooted at the base model's next token (one launch);
 //   the base model's forward over the tree tokens at the cache length, which
 //   writes the tree's K/V rows into the cache;
-//   greedy acceptance with the compaction of the accepted rows (one launch);
+//   acceptance with the compaction of the accepted rows (one launch; the
+//   next token drawn with the step's uniform when the caller gives them);
 //   h for the next step: the final-norm row of the last accepted node.
 // The host reads the accept length and the accepted tokens after each step.
 #include <vector>
@@ -102,7 +104,7 @@ GenLayout gen_layout(const medusa_tree_t* tree, const medusa_decoder_t* m) {
   l.vals = take(static_cast<size_t>(tree->K) * tree->topk * 4);
   l.logits = take(static_cast<size_t>(T) * m->V * 4);
   l.h = take(static_cast<size_t>(m->D) * 2);
-  l.small = take(static_cast<size_t>(8 + tree->D + 1) * 4);   // root, seq_len, best, alen, accepted tokens
+  l.small = take(static_cast<size_t>(8 + tree->D + 1) * 4);   // root, seq_len, best, alen, uniform, -, accepted tokens
   l.total = o;
   return l;
 }
@@ -132,13 +134,14 @@ extern "C" size_t medusa_generate_workspace_size(const medusa_tree_t* tree, cons
   return gen_layout(tree, model).total;
 }
 
-extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, const medusa_decoder_t* model,
-                                                  const void* W1, const void* b1, const void* Wout,
-                                                  const int32_t* prompt, int n_prompt, int n_new, void* k_cache,
-                                                  void* v_cache, int Lcap, int32_t* out_tokens,
-                                                  int32_t* out_accept, int max_steps, int32_t* n_steps,
-                                                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  const char* fn = "medusa_generate_greedy";
+extern "C" medusa_status_t medusa_generate(const medusa_tree_t* tree, const medusa_decoder_t* model,
+                                           const void* W1, const void* b1, const void* Wout, medusa_mode_t mode,
+                                           float temperature, float eps, float alpha, float top_p,
+                                           const float* uniforms, const int32_t* prompt, int n_prompt, int n_new,
+                                           void* k_cache, void* v_cache, int Lcap, int32_t* out_tokens,
+                                           int32_t* out_accept, int max_steps, int32_t* n_steps, void* workspace,
+                                           size_t workspace_bytes, cudaStream_t stream) {
+  const char* fn = "medusa_generate";
   medusa_status_t st = check_decoder(tree, model, 1, fn);
   if (st != MEDUSA_OK) return st;
   if (!W1 || !b1 || !Wout || !prompt || !k_cache || !v_cache || !out_tokens || !out_accept || !n_steps || !workspace)
@@ -158,6 +161,16 @@ extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, con
                    reinterpret_cast<const int32_t*>(w + l.ids), reinterpret_cast<const float*>(w + l.vals),
                    w + l.heads, heads_workspace_bytes(1, model->D, model->V, tree->K, tree->topk));
   if (st != MEDUSA_OK) return st;
+  st = check_posterior(tree, 1, model->V, reinterpret_cast<const float*>(w + l.logits),
+                       reinterpret_cast<const int32_t*>(w + l.cand), mode, temperature, eps, alpha, top_p,
+                       reinterpret_cast<const int32_t*>(w + l.small), reinterpret_cast<const int32_t*>(w + l.small),
+                       reinterpret_cast<const int32_t*>(w + l.small), reinterpret_cast<const int32_t*>(w + l.small),
+                       w + l.post, posterior_workspace_bytes(tree->dev, 1));
+  if (st != MEDUSA_OK) return st;
+  if (uniforms)
+    for (int i = 0; i < max_steps; ++i)
+      if (!(uniforms[i] >= 0.f && uniforms[i] < 1.f))
+        return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": uniforms outside [0, 1)");
 
   void* ws_dec = w + l.dec;
   void* ws_heads = w + l.heads;
@@ -171,6 +184,7 @@ extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, con
   uint16_t* h = reinterpret_cast<uint16_t*>(w + l.h);
   int32_t* small = reinterpret_cast<int32_t*>(w + l.small);
   int32_t *root = small, *seq_len = small + 1, *best = small + 2, *alen = small + 3, *acc = small + 8;
+  float* u_dev = reinterpret_cast<float*>(small + 4);   // this step's uniform
   const int D = model->D, V = model->V, H = D / 128;
   cudaError_t e;
 
@@ -185,7 +199,7 @@ extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, con
       if (st != MEDUSA_OK) return st;
     }
     e = cudaMemcpyAsync(tokens, prompt + at, static_cast<size_t>(n) * 4, cudaMemcpyHostToDevice, stream);
-    if (e != cudaSuccess) return cuda_fail("medusa_generate_greedy: prompt copy", e);
+    if (e != cudaSuccess) return cuda_fail("medusa_generate: prompt copy", e);
     set_len_kernel<<<1, 1, 0, stream>>>(seq_len, L);
     st = launch_tree_decode(g.t->dev, model, 1, tokens, k_cache, v_cache, Lcap, seq_len, logits, nullptr, ws_dec,
                             stream);
@@ -197,7 +211,7 @@ extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, con
                                            last_n - 1, nullptr, 0, 0, nullptr, nullptr, h, root, device_status_ptr());
   set_len_kernel<<<1, 1, 0, stream>>>(seq_len, L);
   e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail("medusa_generate_greedy: launch", e);
+  if (e != cudaSuccess) return cuda_fail("medusa_generate: launch", e);
 
   TreeBuild tb{};
   tb.t = tree->dev;
@@ -216,10 +230,15 @@ extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, con
     st = launch_tree_decode(tree->dev, model, 1, tokens, k_cache, v_cache, Lcap, seq_len, logits, nullptr, ws_dec,
                             stream);
     if (st != MEDUSA_OK) return st;
-    // greedy acceptance; the next token goes where the next step's root is read
-    st = launch_posterior_accept(tree->dev, 1, V, logits, cand, MEDUSA_GREEDY, 0.f, 0.09f, 0.3f, 0.8f, nullptr, best,
-                                 alen, acc, root, model->layers, H, 128, MEDUSA_BF16, k_cache, v_cache, Lcap, seq_len,
-                                 ws_post, stream, false);
+    // acceptance; the next token (drawn with this step's uniform, if any) goes where the next
+    // step's root is read
+    if (uniforms) {
+      e = cudaMemcpyAsync(u_dev, uniforms + steps, 4, cudaMemcpyHostToDevice, stream);
+      if (e != cudaSuccess) return cuda_fail("medusa_generate: uniform copy", e);
+    }
+    st = launch_posterior_accept(tree->dev, 1, V, logits, cand, mode, temperature, eps, alpha, top_p,
+                                 uniforms ? u_dev : nullptr, best, alen, acc, root, model->layers, H, 128, MEDUSA_BF16,
+                                 k_cache, v_cache, Lcap, seq_len, ws_post, stream, false);
     if (st != MEDUSA_OK) return st;
     next_input_kernel<<<1, 256, 0, stream>>>(decoder_final_rows(ws_dec, tree->T, D, model->F, V), logits, D, V, 0,
                                              tree->dev.retrieve, tree->P, dp1, best, alen, h, nullptr,
@@ -227,7 +246,7 @@ extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, con
     e = cudaMemcpyAsync(host.data(), alen, 4, cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaMemcpyAsync(host.data() + 1, acc, static_cast<size_t>(dp1) * 4, cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-    if (e != cudaSuccess) return cuda_fail("medusa_generate_greedy: step", e);
+    if (e != cudaSuccess) return cuda_fail("medusa_generate: step", e);
     const int a = host[0];
     if (a < 0 || a >= dp1) return fail(MEDUSA_ERR_DEVICE_CHECK, std::string(fn) + ": accept length out of range");
     for (int j = 0; j <= a && produced < n_new; ++j) out_tokens[produced++] = host[1 + j];
@@ -238,4 +257,15 @@ extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, con
   if (produced < n_new)
     return fail(MEDUSA_ERR_INVALID_ARG, std::string(fn) + ": stopped before n_new tokens (Lcap or max_steps)");
   return MEDUSA_OK;
+}
+
+extern "C" medusa_status_t medusa_generate_greedy(const medusa_tree_t* tree, const medusa_decoder_t* model,
+                                                  const void* W1, const void* b1, const void* Wout,
+                                                  const int32_t* prompt, int n_prompt, int n_new, void* k_cache,
+                                                  void* v_cache, int Lcap, int32_t* out_tokens,
+                                                  int32_t* out_accept, int max_steps, int32_t* n_steps,
+                                                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return medusa_generate(tree, model, W1, b1, Wout, MEDUSA_GREEDY, 0.f, 0.09f, 0.3f, 0.8f, nullptr, prompt, n_prompt,
+                         n_new, k_cache, v_cache, Lcap, out_tokens, out_accept, max_steps, n_steps, workspace,
+                         workspace_bytes, stream);
 }

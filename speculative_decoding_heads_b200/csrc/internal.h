@@ -68,6 +68,13 @@ medusa_status_t check_step(const medusa_step_args_t* args, const void* ws, size_
 // Host-side checks of the base model and the tree for medusa_tree_decode (api.cu).
 medusa_status_t check_decoder(const medusa_tree_t* tree, const medusa_decoder_t* m, int B, const char* fn);
 
+// Host-side checks of medusa_evaluate_posterior (api.cu).
+medusa_status_t check_posterior(const medusa_tree_t* tree, int B, int V, const float* logits,
+                                const int32_t* candidates, medusa_mode_t mode, float temperature, float eps,
+                                float alpha, float top_p, const int32_t* best_path, const int32_t* accept_len,
+                                const int32_t* accepted_tokens, const int32_t* next_token, const void* ws,
+                                size_t ws_bytes);
+
 // Kernel launchers (heads.cu, tree_kernels.cu, attention.cu, posterior.cu, accept.cu).
 size_t heads_workspace_bytes(int B, int d, int V, int K, int topk);
 medusa_status_t launch_heads(const void* h, const void* W1, const void* b1, const void* Wout,

@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(mb):
 
 
 def test_abi_version(mb):
-    assert mb.abi_version() == 6
+    assert mb.abi_version() == 7
 
 
 def _compare_tables(mb, choices, K, topk):

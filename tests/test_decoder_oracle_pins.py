@@ -176,3 +176,52 @@ def test_greedy_medusa_generation_is_lossless(seed, V, K, topk, n_nodes, kind):
     assert len(accepts) <= n_new and all(0 <= a <= K for a in accepts)
     if kind == "copy":
         assert sum(accepts) > 0, "no proposal was ever accepted: the case would not exercise acceptance"
+
+
+@pytest.mark.parametrize("mode", ["typical", "nucleus"])
+def test_sampled_generation_at_low_temperature_is_greedy(mode):
+    """At a temperature far below the logit gaps the tempered distribution is one-hot: typical
+    acceptance keeps exactly the arg-max child (its probability ~1 is above min(eps, alpha)), the
+    nucleus holds the arg-max alone, and a draw with u in [0.1, 0.9] returns the arg-max.  So
+    sampled Medusa generation reduces to greedy generation, token for token and step for step."""
+    rng = np.random.default_rng(11)
+    V, K, topk = 6, 3, 2
+    model = _model(rng, V)
+    heads = _copy_heads(model, K)
+    prompt = rng.integers(0, V, size=5)
+    choices = O.ranksum_choices(K, topk, 10)
+    ref, ref_acc = D.medusa_generate_greedy(model, heads, choices, K, topk, prompt, 20, Lcap=96)
+    u = 0.1 + 0.8 * rng.random(40)
+    trace = []
+    got, acc = D.medusa_generate(model, heads, choices, K, topk, prompt, 20, 96, mode=mode, temperature=1e-3,
+                                 uniforms=u, trace=trace)
+    assert got == ref and acc == ref_acc and sum(acc) > 0
+    assert [step[3] for step in trace] == acc
+
+
+def test_sampled_generation_draws_from_the_tempered_distribution():
+    """With a high temperature the drawn roots leave the greedy path: every emitted root is the
+    inverse-CDF draw of its step's uniform from the tempered distribution at the previous step's
+    last accepted node."""
+    rng = np.random.default_rng(12)
+    V, K, topk = 6, 2, 2
+    model = _model(rng, V)
+    heads = _heads(rng, K, V)
+    prompt = rng.integers(0, V, size=4)
+    choices = O.ranksum_choices(K, topk, 4)
+    tr = O.tree_tables(choices, K, topk)
+    u = rng.random(30)
+    trace = []
+    got, acc = D.medusa_generate(model, heads, choices, K, topk, prompt, 16, 96, mode="typical",
+                                 temperature=1.5, uniforms=u, trace=trace)
+    greedy, _ = D.medusa_generate_greedy(model, heads, choices, K, topk, prompt, 16, Lcap=96)
+    assert got != greedy
+    pos = 0
+    for s, (logits, cand, best, a, _) in enumerate(trace[:-1]):
+        pos += a + 1
+        if pos >= len(got):
+            break
+        node = tr["retrieve"][best, a]
+        z = logits[node] / 1.5
+        w = np.exp(z - z.max())
+        assert got[pos] == O.sample_index(w, u[s])   # the next step's root

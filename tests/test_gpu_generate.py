@@ -10,6 +10,17 @@ Small LLaMA-shaped base models (hd 128, two heads, two layers) with bf16 weights
   error bound, since the device rounds its intermediates to bf16.
 - **Acceptance.** Heads that repeat the base model's current prediction get proposals accepted, so
   the compaction and the positions of later steps are exercised.
+- **Sampled acceptance (medusa_generate).**
+  - Typical and nucleus acceptance at a temperature far below the logit gaps reduce to greedy
+    decoding on the device.
+  - Typical acceptance at temperature 0.7 matches the oracle's sampled generation. Its seeds keep,
+    on the oracle's trajectory:
+    - every head top-k gap clear;
+    - every typical decision |p - threshold| above 25% of max(p, threshold);
+    - every draw 10% of the mass inside its token's interval.
+
+    Those margins are well above what the device's bf16 intermediates can move (4e-2 of the logits'
+    RMS at most, divided by the temperature).
 """
 
 import numpy as np
@@ -144,3 +155,79 @@ def test_generate_refuses_bad_arguments(mb):
     with pytest.raises(ValueError):       # heads of the wrong count
         mb.medusa_generate_greedy(tree, dec, hd["W1"][:2], hd["b1"], hd["Wout"], [1, 2], 4, kc, kc.clone())
     assert mb.device_status(clear=True) == (0, 0)
+
+
+def test_sampled_generation_at_low_temperature_is_greedy(mb):
+    V, n_prompt, K, topk, n_nodes, n_new = 12, 6, 3, 2, 10, 20
+    choices = O.ranksum_choices(K, topk, n_nodes)
+    Lcap = n_prompt + n_new + len(choices) + 3
+    rng, model, prompt, ref = _clear_seed(V, n_prompt, n_new, Lcap, need_repeat=True)
+    dec, hd, tree = _device(mb, model, _heads(rng, model, K, "copy"), choices, K, topk)
+    greedy, g_acc = _generate(mb, dec, hd, tree, prompt, n_new, Lcap)
+    assert greedy == ref and sum(g_acc) > 0
+    u = (0.1 + 0.8 * rng.random(n_new)).tolist()
+    for mode in (mb.MEDUSA_TYPICAL, mb.MEDUSA_NUCLEUS):
+        kc = torch.zeros((NL, 1, H, Lcap, 128), dtype=torch.bfloat16, device="cuda")
+        toks, acc = mb.medusa_generate(tree, dec, hd["W1"], hd["b1"], hd["Wout"], prompt, n_new, kc, kc.clone(),
+                                       mode=mode, temperature=1e-3, uniforms=u, max_steps=n_new)
+        assert mb.device_status(clear=True) == (0, 0)
+        assert toks == greedy and acc == g_acc, mode
+
+
+def _topk_clear(z, k, rel):
+    """The k+1 largest values of every row are rel * RMS apart (the top-k set and its order hold)."""
+    for row in np.atleast_2d(z):
+        top = np.sort(row)[::-1][:k + 1]
+        if np.min(top[:-1] - top[1:]) < rel * np.sqrt(np.mean(row ** 2)):
+            return False
+    return True
+
+
+def _sampled_seed(V, K, topk, n_nodes, n_prompt, n_new, temp, tries=300):
+    """A model, prompt and uniforms whose typical-acceptance trajectory (oracle) keeps the
+    margins the module docstring lists."""
+    choices = O.ranksum_choices(K, topk, n_nodes)
+    tr = O.tree_tables(choices, K, topk)
+    Lcap = n_prompt + n_new + tr["T"] + 2
+    for seed in range(tries):
+        rng = np.random.default_rng(5000 + seed)
+        model = _model(rng, V)
+        prompt = rng.integers(0, V, size=n_prompt).tolist()
+        kcs, vcs = Dm._empty_caches(model, Lcap)
+        logits0 = Dm._forward(model, Dm.chain_tree(n_prompt), np.asarray(prompt), kcs, vcs, 0)[0][-1]
+        if not _topk_clear(logits0, topk, 2 * MAX_TOL):   # the first root and the first heads' top-k
+            continue
+        heads = _heads(rng, model, K, "copy")
+        u = 0.05 + 0.9 * rng.random(n_new)
+        trace = []
+        got, acc = Dm.medusa_generate(model, heads, choices, K, topk, prompt, n_new, Lcap, mode="typical",
+                                      temperature=temp, uniforms=u, trace=trace)
+        ok = True
+        for s, (logits, cand, best, a, z) in enumerate(trace):
+            st = O.node_statistics(logits, temp, 0.09, 0.3)
+            ret = tr["retrieve"]
+            ok = ok and _topk_clear(z, topk, 2 * MAX_TOL)
+            for p in range(tr["P"]):
+                for j in range(1, tr["D"] + 1):
+                    if ret[p, j] < 0:
+                        break
+                    pr, th = st["prob"][ret[p, j - 1], int(cand[p, j])], st["threshold"][ret[p, j - 1]]
+                    ok = ok and abs(pr - th) >= 0.25 * max(pr, th)
+            ok = ok and O.sample_margin_ok(st["prob"][ret[best, a]], float(u[s]), rel=0.1)
+            if not ok:
+                break
+        if ok and sum(acc) > 0:
+            return model, choices, heads, prompt, u, got, acc, Lcap
+    raise RuntimeError("no seed with clear sampled decisions")
+
+
+def test_typical_generation_matches_the_oracle(mb):
+    V, K, topk, n_nodes, n_prompt, n_new, temp = 8, 2, 2, 4, 5, 10, 0.7
+    model, choices, heads, prompt, u, ref, ref_acc, Lcap = _sampled_seed(V, K, topk, n_nodes, n_prompt, n_new, temp)
+    dec, hd, tree = _device(mb, model, heads, choices, K, topk)
+    kc = torch.zeros((NL, 1, H, Lcap, 128), dtype=torch.bfloat16, device="cuda")
+    toks, acc = mb.medusa_generate(tree, dec, hd["W1"], hd["b1"], hd["Wout"], prompt, n_new, kc, kc.clone(),
+                                   mode=mb.MEDUSA_TYPICAL, temperature=temp, uniforms=u.tolist(), max_steps=n_new)
+    assert mb.device_status(clear=True) == (0, 0)
+    assert toks == ref
+    assert acc == ref_acc[:len(acc)]
