@@ -64,7 +64,7 @@ struct GemmArgs {
   int tiles, nst, W, G;   // tiles of 128 rows, stages per tile, all stages, CTAs
   int kps;                // column blocks per ring stage
   int tok0, ntok;         // this pass: tokens tok0 .. tok0 + kN - 1 (clipped to ntok)
-  float* part;            // [G, 2, 128, kN]
+  float* part;            // [G, 2, kN, 128]: each CTA's parts of its first and last tile
   unsigned* tile_cnt;     // [tiles * 4]
   int* status;
   // QKV
@@ -210,13 +210,12 @@ __device__ __forceinline__ void epilogue_half(const GemmArgs& a, const BarsT* bs
   } else if constexpr (kMode == kResid) {
     const int f = tile * kTileRows + r;
     if (f >= a.rows) return;
+    // One finishing CTA per element: x + product, added in L2 (a single
+    // fp32 addition, as a load, add and store would give), with no load.
     float* xr = a.x + static_cast<size_t>(a.tok0 + c0) * a.rows + f;
-    float old[kHalf];
-#pragma unroll
-    for (int i = 0; i < kHalf; ++i) old[i] = c0 + i < nvalid ? xr[static_cast<size_t>(i) * a.rows] : 0.f;
 #pragma unroll
     for (int i = 0; i < kHalf; ++i)
-      if (c0 + i < nvalid) xr[static_cast<size_t>(i) * a.rows] = old[i] + acc[i];
+      if (c0 + i < nvalid) atomicAdd(xr + static_cast<size_t>(i) * a.rows, acc[i]);
   } else {
     const int f = tile * kTileRows + r;
     if (f >= a.rows) return;
@@ -227,6 +226,13 @@ __device__ __forceinline__ void epilogue_half(const GemmArgs& a, const BarsT* bs
   }
 }
 
+// The partial sums of a shared tile: CTA cc's slot sl (its first or its last
+// tile) holds [kN tokens][128 rows] fp32, token-major, so that a warp's 32
+// rows of one token are one 128-byte line.  This returns token c's row 0.
+__device__ __forceinline__ float* part_at(const GemmArgs& a, int cc, int sl, int c, int kN) {
+  return a.part + ((static_cast<size_t>(cc) * 2 + sl) * kN + c) * kTileRows;
+}
+
 // One 32-column chunk of a finished tile row: the accumulator from tensor
 // memory, for a shared tile plus the other CTAs' parts (summed in CTA order,
 // kPar CTAs' loads in flight at a time), then the epilogue.
@@ -234,43 +240,37 @@ template <int kMode, int kN, class BarsT>
 __device__ __forceinline__ void finish_chunk(const GemmArgs& a, const BarsT* bs, int tile, int r, uint32_t tacc,
                                              int hh, bool split, int c_first, int c_last, int cta) {
   float acc[kHalf];
-  tc::tmem_ld32(tacc + hh * kHalf, acc);
-  tc::tmem_wait_ld();
-  if (split) {
-    float sum[kHalf];
+  if (!split) {
+    tc::tmem_ld32(tacc + hh * kHalf, acc);
+    tc::tmem_wait_ld();
+  } else {
+    // This CTA's own part is read again from tensor memory at its place in
+    // the order, so that it holds no registers across the loads.
 #pragma unroll
-    for (int c = 0; c < kHalf; ++c) sum[c] = 0.f;
+    for (int c = 0; c < kHalf; ++c) acc[c] = 0.f;
+#pragma unroll 1
     for (int cc0 = c_first; cc0 <= c_last; cc0 += kPar) {
-      float4 pv[kPar][kHalf / 4];
+      float pv[kPar][kHalf];
 #pragma unroll
       for (int u = 0; u < kPar; ++u) {
         const int cc = cc0 + u;
-        if (cc <= c_last && cc != cta) {
+        if (cc == cta) {
+          tc::tmem_ld32(tacc + hh * kHalf, pv[u]);
+        } else if (cc <= c_last) {
           const int sl = tile == stage_lo(cc, a) / a.nst ? 0 : 1;
-          const float4* pc = reinterpret_cast<const float4*>(
-              a.part + ((static_cast<size_t>(cc) * 2 + sl) * kTileRows + r) * kN + hh * kHalf);
+          const float* pc = part_at(a, cc, sl, hh * kHalf, kN) + r;
 #pragma unroll
-          for (int e = 0; e < kHalf / 4; ++e) pv[u][e] = __ldcg(pc + e);
+          for (int i = 0; i < kHalf; ++i) pv[u][i] = __ldcg(pc + i * kTileRows);
         }
       }
+      tc::tmem_wait_ld();
 #pragma unroll
-      for (int u = 0; u < kPar; ++u) {
-        const int cc = cc0 + u;
-        if (cc <= c_last) {
+      for (int u = 0; u < kPar; ++u)
+        if (cc0 + u <= c_last) {
 #pragma unroll
-          for (int e = 0; e < kHalf / 4; ++e) {
-            const float4 v = cc == cta ? make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3])
-                                       : pv[u][e];
-            sum[4 * e] += v.x;
-            sum[4 * e + 1] += v.y;
-            sum[4 * e + 2] += v.z;
-            sum[4 * e + 3] += v.w;
-          }
+          for (int i = 0; i < kHalf; ++i) acc[i] += pv[u][i];
         }
-      }
     }
-#pragma unroll
-    for (int c = 0; c < kHalf; ++c) acc[c] = sum[c];
   }
   epilogue_half<kMode, kN>(a, bs, tile, r, hh * kHalf, acc);
 }
@@ -432,17 +432,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // A tile shared with other CTAs: store this part; the last to finish
         // sums the parts in CTA order.
         const int slot = x.tile == st_lo / a.nst ? 0 : 1;
-        float* mine = a.part + ((static_cast<size_t>(cta) * 2 + slot) * kTileRows + r) * kN;
+        float* mine = part_at(a, cta, slot, 0, kN) + r;
 #pragma unroll 1
         for (int hh = 0; hh < kN / kHalf; ++hh) {
           float acc[kHalf];
           tc::tmem_ld32(tacc + hh * kHalf, acc);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < kHalf; c += 4)
-            *reinterpret_cast<float4*>(mine + hh * kHalf + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+          for (int c = 0; c < kHalf; ++c) mine[(hh * kHalf + c) * kTileRows] = acc[c];
         }
-        __threadfence();
+        fence_acq_rel_gpu();
         __syncwarp();
         int last = 0;
         if (lane == 0) {
@@ -451,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last) *cnt = 0u;
         }
         mine_last = __shfl_sync(0xffffffffu, last, 0) != 0;
-        if (mine_last) __threadfence();
+        if (mine_last) fence_acq_rel_gpu();
       }
       // This CTA's final unit ends the kernel for it: when it finishes the
       // tile, warp q of warps 0-3 (idle by now) takes the odd chunks.
@@ -592,7 +591,7 @@ bool encode_w(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void*
 // 256 that takes all of them, else 256.
 int tokens_per_pass(int ntok) { return ntok <= 64 ? 64 : (ntok <= 128 ? 128 : kMaxN); }
 
-// Scratch of the matrix products: tile counters, then [G, 2, 128, kN] partials.
+// Scratch of the matrix products: tile counters, then [G, 2, kN, 128] partials.
 size_t gemm_scratch_bytes(int D, int F, int V, int ntok) {
   int rows = 3 * D;
   if (2 * F > rows) rows = 2 * F;
