@@ -211,6 +211,28 @@ size_t attention_workspace_bytes(const TreeDev& t, int layers, int B, int H, int
   return 0;
 }
 
+// Tree rows handled in groups of 128 (tree_attn_tc128): where a group would
+// hold more than 64 of them; the rest (at most 64) go to one 64-row group.
+int rows_in_128_groups(int T) { return T <= 64 ? 0 : (T % 128 == 0 || T % 128 > 64 ? T : T / 128 * 128); }
+
+medusa_status_t launch_attention_bf16_out(const TreeDev& t, int B, int H, const void* q, const void* k_cache,
+                                          const void* v_cache, int Lcap, const int32_t* seq_lens, float scale,
+                                          uint16_t* out, cudaStream_t stream) {
+  int* status = device_status_ptr();
+  const float sl = scale * kLog2e;
+  AttnOut dec;
+  dec.bf16 = out;
+  dec.wait_first = true;
+  const int full = rows_in_128_groups(t.T);
+  if (full > 0) {
+    const medusa_status_t st = launch_attention_tc128(t, 1, B, H, q, k_cache, v_cache, Lcap, seq_lens, sl, nullptr,
+                                                      status, stream, true, 0, full, dec);
+    if (st != MEDUSA_OK || full == t.T) return st;
+  }
+  return launch_attention_tc64(t, 1, B, H, q, k_cache, v_cache, Lcap, seq_lens, sl, nullptr, status, stream, true,
+                               full, t.T, 0, 1, nullptr, dec);
+}
+
 medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int hd, medusa_dtype_t dtype,
                                  const void* q, const void* k_cache, const void* v_cache, int Lcap,
                                  const int32_t* seq_lens, float scale, void* out, void* ws,
@@ -220,11 +242,9 @@ medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int
   int* status = device_status_ptr();
   cudaError_t e;
   if (dtype == MEDUSA_BF16 && hd == kHd) {
-    // Rows in groups of 128 where a group would hold more than 64 of them,
-    // the rest (at most 64) in one 64-row group.
     float* o = static_cast<float*>(out);
     const float sl = scale * kLog2e;
-    const int full = t.T <= 64 ? 0 : (t.T % 128 == 0 || t.T % 128 > 64 ? t.T : t.T / 128 * 128);
+    const int full = rows_in_128_groups(t.T);
     if (full > 0) {
       const medusa_status_t st =
           launch_attention_tc128(t, layers, B, H, q, k_cache, v_cache, Lcap, seq_lens, sl, o, status, stream, pdl, 0,

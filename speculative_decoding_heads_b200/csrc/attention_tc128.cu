@@ -91,6 +91,8 @@ struct Params {
   const int32_t* seq_lens;
   float scale_log2;
   float* out;
+  uint16_t* out_bf16;      // if set, the output goes here as bf16 instead of `out`
+  int wait_first;          // wait for the preceding kernel before the first load
   int* status;
   int kv_one_box;   // 1: one 32 KB TMA box per tile (4-D map), 0: two 16 KB boxes
 };
@@ -163,6 +165,7 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
   tc::prefetch_tensormap(q_map);
   tc::prefetch_tensormap(k_map);
   tc::prefetch_tensormap(v_map);
+  if (p.wait_first) wait_prior_grids();   // q and the tree's K/V rows come from it
   int kkk = 0, kkv = 0;
   Slice sk = seek(kkk, p, bar->lens), sv = seek(kkv, p, bar->lens);
   int ek = 0, gv = 0;     // K-ring entries and V tiles issued
@@ -462,8 +465,20 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&bar->o_read);
-        if (r < p.row_hi) {
-          float* dst = p.out + ((static_cast<size_t>(s.lb) * T + r) * p.H + s.e) * kHd + 64 * hf;
+        const size_t ooff = ((static_cast<size_t>(s.lb) * T + r) * p.H + s.e) * kHd + 64 * hf;
+        if (r < p.row_hi && p.out_bf16) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + ooff);
+#pragma unroll
+          for (int c = 0; c < 64; c += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              w[u] = static_cast<uint32_t>(f32_to_bf16_rne(o[c + 2 * u] * inv)) |
+                     (static_cast<uint32_t>(f32_to_bf16_rne(o[c + 2 * u + 1] * inv)) << 16);
+            dst[c / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else if (r < p.row_hi) {
+          float* dst = p.out + ooff;
 #pragma unroll
           for (int c = 0; c < 64; c += 4)
             *reinterpret_cast<float4*>(dst + c) = make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
@@ -542,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 medusa_status_t launch_attention_tc128(const TreeDev& t, int layers, int B, int H, const void* q,
                                        const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
                                        float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl,
-                                       int row_lo, int row_hi) {
+                                       int row_lo, int row_hi, const AttnOut& dec) {
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!enc) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: cuTensorMapEncodeTiled unavailable");
   if (t.T > 2 * kRows || t.W > 4) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: more than 256 tree tokens");
@@ -605,6 +620,8 @@ medusa_status_t launch_attention_tc128(const TreeDev& t, int layers, int B, int 
   prm.seq_lens = seq_lens;
   prm.scale_log2 = scale_log2;
   prm.out = out;
+  prm.out_bf16 = dec.bf16;
+  prm.wait_first = dec.wait_first ? 1 : 0;
   prm.status = status;
   prm.kv_one_box = one_box;
   const int grid = static_cast<int>(items < sm_count() ? items : sm_count());

@@ -104,6 +104,8 @@ struct Params {
   const int32_t* seq_lens;
   float scale_log2;
   float* out;
+  uint16_t* out_bf16;      // if set, the output goes here as bf16 instead of `out`
+  int wait_first;          // wait for the preceding kernel before the first load
   int* status;
   int kv_one_box;   // 1: one 32 KB TMA box per tile (4-D map), 0: two 16 KB boxes
   int split_r, split_G;   // this launch is window split_r of split_G along the prefix (0, 1: all of it)
@@ -200,6 +202,7 @@ __device__ void run_producer(const CUtensorMap* q_map, const CUtensorMap* k_map,
   tc::prefetch_tensormap(q_map);
   tc::prefetch_tensormap(k_map);
   tc::prefetch_tensormap(v_map);
+  if (p.wait_first) wait_prior_grids();   // q and the tree's K/V rows come from it
   int kkq = 0, kkk = 0, kkv = 0;
   Slice sq = seek<kSplit>(kkq, p, bar->lens), sk = seek<kSplit>(kkk, p, bar->lens), sv = seek<kSplit>(kkv, p, bar->lens);
   int nq = 0, gk = 0, gv = 0, tk = 0, tv = 0;     // loads issued; step within slice
@@ -520,7 +523,8 @@ __device__ void run_softmax(const Params& p, unsigned char* smem, uint32_t tmem,
 }
 
 // ---- epilogue (warps 2, 3, 8, 9) ------------------------------------------------
-// out[query] = (O(high-part lanes) + O(remainder lanes)) / row sum, in fp32.
+// out[query] = (O(high-part lanes) + O(remainder lanes)) / row sum, in fp32
+// (or rounded to bf16 into out_bf16).
 template <bool kSplit>
 __device__ void run_epilogue(const Params& p, uint32_t tmem, Bars* bar, int warp, int lane) {
   const int q = warp & 3, h = lane >> 4, i = lane & 15;
@@ -536,15 +540,26 @@ __device__ void run_epilogue(const Params& p, uint32_t tmem, Bars* bar, int warp
     const int r = p.row_lo + kRows * s.grp + 16 * q + i;   // tree token
     const float inv = 1.f / bar->lsum[k & 1][16 * q + i];
     const uint32_t oa = tmem + la + col_o(k & 1);
-    float* orow = p.out + ((static_cast<size_t>(s.lb) * T + r) * p.H + s.e) * kHd + 64 * h;
+    const size_t ooff = ((static_cast<size_t>(s.lb) * T + r) * p.H + s.e) * kHd + 64 * h;
 #pragma unroll 1
     for (int cp = 0; cp < 2; ++cp) {
       float a[32], b[32];                        // columns 64h + 32cp + (0..31)
       tc::tmem_ld32x2<64>(oa + 32 * cp, a);
       tc::tmem_ld32x2<64>(oa + kLaneHalf + 32 * cp, b);
       tc::tmem_wait_ld();
-      if (r < p.row_hi) {
-        float* dst = orow + 32 * cp;
+      if (r < p.row_hi && p.out_bf16) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + ooff + 32 * cp);
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            w[u] = static_cast<uint32_t>(f32_to_bf16_rne((a[c + 2 * u] + b[c + 2 * u]) * inv)) |
+                   (static_cast<uint32_t>(f32_to_bf16_rne((a[c + 2 * u + 1] + b[c + 2 * u + 1]) * inv)) << 16);
+          dst[c / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      } else if (r < p.row_hi) {
+        float* dst = p.out + ooff + 32 * cp;
 #pragma unroll
         for (int c = 0; c < 32; c += 4)
           *reinterpret_cast<float4*>(dst + c) = make_float4((a[c] + b[c]) * inv, (a[c + 1] + b[c + 1]) * inv,
@@ -647,7 +662,8 @@ void* tensor_map_encoder() {
 medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H, const void* q,
                                       const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
                                       float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl,
-                                      int row_lo, int row_hi, int split_r, int split_G, float* lse) {
+                                      int row_lo, int row_hi, int split_r, int split_G, float* lse,
+                                      const AttnOut& dec) {
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!enc) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: cuTensorMapEncodeTiled unavailable");
   if (t.T > 4 * kRows || t.W > 4) return fail(MEDUSA_ERR_UNSUPPORTED, "tree attention: more than 256 tree tokens");
@@ -710,6 +726,8 @@ medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H
   prm.seq_lens = seq_lens;
   prm.scale_log2 = scale_log2;
   prm.out = out;
+  prm.out_bf16 = dec.bf16;
+  prm.wait_first = dec.wait_first ? 1 : 0;
   prm.status = status;
   prm.kv_one_box = one_box;
   prm.split_r = split_r;

@@ -73,6 +73,7 @@ struct GemmArgs {
   uint16_t* v_cache;
   const int32_t* seq_lens;
   const int32_t* depth;   // [T]
+  const float2* rope;     // [ntok, 64]: (cos, sin) of each token's angle per frequency
   int T, H, Lcap;
   // RESID
   float* x;               // [ntok, rows]
@@ -91,9 +92,8 @@ struct Bars {
   int tail_n[4];           // per lane quarter: index of the final unit (-1: no help wanted)
   uint32_t tmem_base;
   int abort;
-  // QKV: for each token c of the pass, its rotary position and its cache row
-  // offset ((b H) Lcap + L + node) 128 (-1: no valid cache row)
-  alignas(16) int pos[kN];
+  // QKV: for each token c of the pass, its cache row offset
+  // ((b H) Lcap + L + node) 128 (-1: no valid cache row)
   alignas(16) long long crow[kN];
 };
 
@@ -147,26 +147,23 @@ __device__ __forceinline__ void epilogue_half(const GemmArgs& a, const BarsT* bs
     const int j = r >> 1;                                   // pair index (frequency)
     const int feat = j + (r & 1) * 64;                      // feature within the head
     // rotation frequency base^(-2j/128) with base 10000, angle reduced in double
-    const double inv = exp2(-static_cast<double>(2 * j) / 128.0 * 13.287712379549449);
     uint16_t* cache = which == 1 ? a.k_cache : a.v_cache;
-    // 16 tokens at a time: their table entries (vector loads) and partner
-    // values first, so that the 16 rotations are independent and no store
-    // sits between loads; then the stores, each under its own predicate.
+    // 16 tokens at a time: their cache rows (vector loads), rotations
+    // (cos, sin of the token's angle for frequency j, from the forward's
+    // table) and partner values first, so that the 16 rotations are
+    // independent and no store sits between loads; then the stores, each
+    // under its own predicate.
     uint16_t* const dst = which == 0 ? a.q_out + h * 128 + feat : cache + static_cast<long long>(h) * a.Lcap * 128 + feat;
 #pragma unroll
     for (int i0 = 0; i0 < kHalf; i0 += 16) {
-      int pos[16];
       long long row[16];
       float other[16];
-      const int4* pp = reinterpret_cast<const int4*>(bs->pos + c0 + i0);
+      float2 rot[16];
       const longlong2* rp = reinterpret_cast<const longlong2*>(bs->crow + c0 + i0);
+      if (which < 2) {
+        const float2* tp = a.rope + static_cast<size_t>(a.tok0 + c0 + i0) * 64 + j;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int4 p4 = pp[k];
-        pos[4 * k] = p4.x;
-        pos[4 * k + 1] = p4.y;
-        pos[4 * k + 2] = p4.z;
-        pos[4 * k + 3] = p4.w;
+        for (int i = 0; i < 16; ++i) rot[i] = c0 + i0 + i < nvalid ? tp[i * 64] : make_float2(1.f, 0.f);
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -182,10 +179,7 @@ __device__ __forceinline__ void epilogue_half(const GemmArgs& a, const BarsT* bs
         const float own = acc[i0 + i];
         float out = own;
         if (which < 2) {
-          const double ang = static_cast<double>(pos[i]) * inv;
-          const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
-          float sn, cs;
-          __sincosf(static_cast<float>(red), &sn, &cs);   // |red| <= pi
+          const float cs = rot[i].x, sn = rot[i].y;
           out = (r & 1) ? other[i] * sn + own * cs : own * cs - other[i] * sn;
         }
         v[i] = f32_to_bf16_rne(out);
@@ -198,14 +192,20 @@ __device__ __forceinline__ void epilogue_half(const GemmArgs& a, const BarsT* bs
       }
     }
   } else if constexpr (kMode == kSwiGLU) {
+    // Lanes 2j' (gate) and 2j' + 1 (up) of feature j share the 32 tokens:
+    // the even lane finishes tokens 0-15, the odd lane tokens 16-31, each
+    // with the other's value for its token.
     const int j = tile * 64 + (r >> 1);   // output feature
-    const bool writer = !(r & 1) && 2 * j < a.rows;
-    uint16_t* dst = a.act + static_cast<size_t>(a.tok0 + c0) * (a.rows / 2) + j;
+    const int odd = r & 1;
+    const int hi = odd * (kHalf / 2);
+    uint16_t* dst = a.act + static_cast<size_t>(a.tok0 + c0 + hi) * (a.rows / 2) + j;
 #pragma unroll
-    for (int i = 0; i < kHalf; ++i) {
-      const float own = acc[i];
-      const float up = __shfl_xor_sync(0xffffffffu, own, 1);
-      if (c0 + i < nvalid && writer) dst[static_cast<size_t>(i) * (a.rows / 2)] = f32_to_bf16_rne(silu(own) * up);
+    for (int i = 0; i < kHalf / 2; ++i) {
+      const float mine = acc[i + hi];                                       // gate (even) or up (odd)
+      const float theirs = __shfl_xor_sync(0xffffffffu, odd ? acc[i] : acc[i + kHalf / 2], 1);
+      const float gate = odd ? theirs : mine, up = odd ? mine : theirs;
+      if (c0 + hi + i < nvalid && 2 * j < a.rows)
+        dst[static_cast<size_t>(i) * (a.rows / 2)] = f32_to_bf16_rne(silu(gate) * up);
     }
   } else if constexpr (kMode == kResid) {
     const int f = tile * kTileRows + r;
@@ -313,19 +313,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (kMode == kQKV) {
     for (int c = tid; c < kN; c += kThreads) {
       const int n = a.tok0 + c;
-      int p = 0;
       long long row = -1;
       if (n < a.ntok) {
         const int b = n / a.T, node = n - b * a.T;
         const int L = a.seq_lens[b];
-        if (L < 0 || L + a.T > a.Lcap) {   // the tree's rows would not fit in the cache
+        if (L < 0 || L + a.T > a.Lcap)   // the tree's rows would not fit in the cache
           set_device_status(a.status, MEDUSA_ERR_DEVICE_CHECK, kDetailDecoderSeqLen);
-        } else {
-          p = L + a.depth[node];
+        else
           row = (static_cast<long long>(b) * a.H * a.Lcap + L + node) * 128;
-        }
       }
-      bs->pos[c] = p;
       bs->crow[c] = row;
     }
   }
@@ -508,10 +504,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- small kernels ------------------------------------------------------------
 
-// x[n] = embed[tokens[n]] (bf16 -> fp32), n over the B*T tree tokens.
-__global__ void embed_kernel(const int32_t* tokens, const uint16_t* embed, int D, int V, float* x, int* status) {
+// x[n] = embed[tokens[n]] (bf16 -> fp32), n over the B*T tree tokens; and the
+// token's rotation table: rope[n][j] = (cos, sin)(p base^(-2j/128)), base
+// 10000, at its position p = L_b + depth, the angle reduced in double.
+__global__ void embed_kernel(const int32_t* tokens, const uint16_t* embed, int D, int V, float* x,
+                             const int32_t* seq_lens, const int32_t* depth, int T, float2* rope, int* status) {
   allow_dependents();
   const int n = blockIdx.x;
+  if (threadIdx.x < 64) {
+    const int j = threadIdx.x, b = n / T;
+    const int p = seq_lens[b] + depth[n - b * T];   // a bad length is reported by the QKV products
+    const double ang = static_cast<double>(p) * exp2(-static_cast<double>(2 * j) / 128.0 * 13.287712379549449);
+    double sn, cs;
+    sincos(ang, &sn, &cs);
+    rope[static_cast<size_t>(n) * 64 + j] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  }
   const int tok = tokens[n];
   if (tok < 0 || tok >= V) {
     if (threadIdx.x == 0) set_device_status(status, MEDUSA_ERR_DEVICE_CHECK, kDetailDecoderToken);
@@ -566,14 +573,6 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* x, c
       yr[k] = o;
     }
   }
-}
-
-__global__ void to_bf16_kernel(const float* x, size_t n, uint16_t* y) {
-  wait_prior_grids();
-  allow_dependents();
-  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x)
-    y[i] = f32_to_bf16_rne(x[i]);
 }
 
 bool encode_w(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, uint64_t kdim,
@@ -655,14 +654,14 @@ uint16_t* decoder_final_rows(void* ws, int ntok, int D, int F, int V) {
 }
 
 size_t decoder_workspace_bytes(int ntok, int D, int F, int V) {
-  // The products' scratch; then x fp32, xn bf16, q bf16, attention fp32 and bf16, act bf16.
+  // The products' scratch; then x fp32, xn bf16, q bf16, attention output bf16, act bf16.
   size_t o = gemm_scratch_bytes(D, F, V, ntok);
   o += align_up(static_cast<size_t>(ntok) * D * 4, 256);       // x
   o += align_up(static_cast<size_t>(ntok) * D * 2, 256);       // xn
   o += align_up(static_cast<size_t>(ntok) * D * 2, 256);       // q (bf16, [ntok, H, 128])
-  o += align_up(static_cast<size_t>(ntok) * D * 4, 256);       // attention output fp32
   o += align_up(static_cast<size_t>(ntok) * D * 2, 256);       // attention output bf16
   o += align_up(static_cast<size_t>(ntok) * F * 2, 256);       // act
+  o += align_up(static_cast<size_t>(ntok) * 64 * 8, 256);      // rotation table
   return o;
 }
 
@@ -680,16 +679,17 @@ medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, 
   o += align_up(static_cast<size_t>(ntok) * D * 2, 256);
   uint16_t* qb = reinterpret_cast<uint16_t*>(w + o);
   o += align_up(static_cast<size_t>(ntok) * D * 2, 256);
-  float* att = reinterpret_cast<float*>(w + o);
-  o += align_up(static_cast<size_t>(ntok) * D * 4, 256);
   uint16_t* attb = reinterpret_cast<uint16_t*>(w + o);
   o += align_up(static_cast<size_t>(ntok) * D * 2, 256);
   uint16_t* act = reinterpret_cast<uint16_t*>(w + o);
+  o += align_up(static_cast<size_t>(ntok) * F * 2, 256);
+  float2* rope = reinterpret_cast<float2*>(w + o);
   int* status = device_status_ptr();
   const size_t slab = static_cast<size_t>(B) * H * Lcap * 128;   // one layer of one cache, elements
   const float scale = 1.0f / sqrtf(128.0f);
 
-  embed_kernel<<<ntok, 256, 0, stream>>>(tree_tokens, static_cast<const uint16_t*>(m->embed), D, V, x, status);
+  embed_kernel<<<ntok, 256, 0, stream>>>(tree_tokens, static_cast<const uint16_t*>(m->embed), D, V, x, seq_lens,
+                                         t.depth, t.T, rope, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("medusa_tree_decode: embedding launch", e);
   for (int l = 0; l < m->layers; ++l) {
@@ -708,16 +708,14 @@ medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, 
     g.v_cache = vc;
     g.seq_lens = seq_lens;
     g.depth = t.depth;
+    g.rope = rope;
     g.T = t.T;
     g.H = H;
     g.Lcap = Lcap;
     medusa_status_t st = gemm<kQKV>(ly.wqkv, xn, g, gws, stream);
     if (st != MEDUSA_OK) return st;
-    st = launch_attention(t, 1, B, H, 128, MEDUSA_BF16, qb, kc, vc, Lcap, seq_lens, scale, att, nullptr, stream);
+    st = launch_attention_bf16_out(t, B, H, qb, kc, vc, Lcap, seq_lens, scale, attb, stream);
     if (st != MEDUSA_OK) return st;
-    e = launch_kernel(to_bf16_kernel, dim3(2 * sm_count()), dim3(256), 0, stream, true, static_cast<const float*>(att),
-                      static_cast<size_t>(ntok) * D, attb);
-    if (e != cudaSuccess) return cuda_fail("medusa_tree_decode: conversion launch", e);
     g = GemmArgs{};
     g.ntok = ntok;
     g.rows = D;

@@ -104,6 +104,11 @@ medusa_status_t launch_attention(const TreeDev& t, int layers, int B, int H, int
                                  medusa_dtype_t dtype, const void* q, const void* k_cache,
                                  const void* v_cache, int Lcap, const int32_t* seq_lens,
                                  float scale, void* out, void* ws, cudaStream_t stream, bool pdl = false);
+// bf16, hd 128 only: the base forward's attention, its output bf16 [B, T, H, 128],
+// launched to overlap the preceding kernel (AttnOut).
+medusa_status_t launch_attention_bf16_out(const TreeDev& t, int B, int H, const void* q, const void* k_cache,
+                                          const void* v_cache, int Lcap, const int32_t* seq_lens, float scale,
+                                          uint16_t* out, cudaStream_t stream);
 
 size_t posterior_workspace_bytes(const TreeDev& t, int B);
 medusa_status_t launch_posterior(const TreeDev& t, int B, int V, const float* logits,
@@ -153,6 +158,14 @@ medusa_status_t launch_tree_decode(const TreeDev& t, const medusa_decoder_t* m, 
 // cuTensorMapEncodeTiled (PFN_cuTensorMapEncodeTiled_v12000), or null.
 void* tensor_map_encoder();
 
+// Inside the base forward: the output as bf16 (the next product's operand)
+// instead of fp32, and a launch that overlaps the preceding kernel, whose
+// outputs (q, the tree's K/V rows) the kernel waits for before its first load.
+struct AttnOut {
+  uint16_t* bf16 = nullptr;
+  bool wait_first = false;
+};
+
 // split_r / split_G: attend only to window split_r of split_G of each slice's
 // cached prefix (the tree's own rows with the last window); lse, if not null,
 // receives ln sum exp(scale q.k) over the window per (layer, seq, node, head).
@@ -160,12 +173,12 @@ medusa_status_t launch_attention_tc64(const TreeDev& t, int layers, int B, int H
                                       const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
                                       float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl,
                                       int row_lo, int row_hi, int split_r = 0, int split_G = 1,
-                                      float* lse = nullptr);
+                                      float* lse = nullptr, const AttnOut& dec = AttnOut{});
 
 medusa_status_t launch_attention_tc128(const TreeDev& t, int layers, int B, int H, const void* q,
                                        const void* k_cache, const void* v_cache, int Lcap, const int32_t* seq_lens,
                                        float scale_log2, float* out, int* status, cudaStream_t stream, bool pdl,
-                                       int row_lo, int row_hi);
+                                       int row_lo, int row_hi, const AttnOut& dec = AttnOut{});
 
 // cudaLaunchKernelEx with programmatic stream serialisation when `pdl` is set.
 template <typename... Params, typename... Args>

@@ -58,21 +58,23 @@ def _close(got, ref, what):
     return e_rms, e_max
 
 
-@pytest.mark.parametrize("B,lens,choices", [
-    (2, [37, 70], ("ranksum", 3, 2, 14)),        # T 15: one pass of 64 tokens
-    (4, [5, 130, 64, 0], ("ranksum", 4, 3, 20)),  # T 21: 84 tokens, one pass of 128; an empty prefix
-    (1, [300], ("ranksum", 5, 10, 63)),           # T 64: the 7B tree, one full pass
-    (3, [10, 200, 77], ("ranksum", 5, 10, 63)),   # 192 tokens: one pass of 256
-    (5, [3, 90, 0, 41, 260], ("ranksum", 5, 10, 63)),   # 320 tokens: passes of 256 and 64 rows
+@pytest.mark.parametrize("B,lens,choices,lcap", [
+    (2, [37, 70], ("ranksum", 3, 2, 14), 0),        # T 15: one pass of 64 tokens
+    (4, [5, 130, 64, 0], ("ranksum", 4, 3, 20), 0),  # T 21: 84 tokens, one pass of 128; an empty prefix
+    (1, [300], ("ranksum", 5, 10, 63), 0),           # T 64: the 7B tree, one full pass
+    (3, [10, 200, 77], ("ranksum", 5, 10, 63), 0),   # 192 tokens: one pass of 256
+    (5, [3, 90, 0, 41, 260], ("ranksum", 5, 10, 63), 0),   # 320 tokens: passes of 256 and 64 rows
+    (3, [0, 1, 700], ("ranksum", 3, 2, 14), 800),    # a larger cache, with near-empty prefixes
+    (1, [900], ("ranksum", 5, 10, 63), 1000),        # the 7B tree over a longer prefix
 ])
-def test_tree_decode_matches_oracle(mb, B, lens, choices):
+def test_tree_decode_matches_oracle(mb, B, lens, choices, lcap):
     rng = np.random.default_rng(B * 100 + len(choices))
     D, F, V, nl, H = 256, 384, 1000, 2, 2
     _, K, topk, n = choices
     ch = O.ranksum_choices(K, topk, n)
     tr = O.tree_tables(ch, K, topk)
     T = tr["T"]
-    Lcap = max(lens) + T + 3
+    Lcap = max(max(lens) + T + 3, lcap)
     embed, layers, final_norm, lm_head = _model(rng, D, F, V, nl)
     tokens = rng.integers(0, V, size=(B, T))
     kc = _bf(rng.normal(size=(nl, B, H, Lcap, 128)))
