@@ -154,10 +154,6 @@ __device__ __forceinline__ unsigned atom_add_release_gpu(unsigned* p, unsigned v
   return old;
 }
 
-// Orders this thread's earlier memory accesses before its later ones for
-// every observer on the GPU (lighter than the sequentially consistent fence).
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-
 __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
   unsigned old;
   asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");

@@ -128,6 +128,10 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ba
   return false;
 }
 
+// Orders this thread's earlier memory accesses before its later ones for
+// every observer on the GPU (lighter than the sequentially consistent fence).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 // SiLU for a value that is rounded to bf16 next: the fast exponential and
 // division (a few ulp of fp32) are far inside bf16's rounding.
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
