@@ -20,8 +20,9 @@
 // of 128 rows cut by a range boundary is summed, per quarter of its rows, by
 // the last CTA to finish it, in CTA order.  The epilogue is fused per
 // product:
-//   QKV     rotary embedding of q and k at position L_b + depth, q to its
-//           buffer, k and v into the cache rows L_b + node
+//   QKV     rotary embedding of q and k at position L_b + depth ((cos, sin)
+//           from a table the embedding kernel builds once per forward), q to
+//           its buffer, k and v into the cache rows L_b + node
 //   RESID   x += product (the fp32 residual stream)
 //   SWIGLU  act = SiLU(gate) * up, bf16
 //   LOGITS  fp32 logits
@@ -150,7 +151,6 @@ __device__ __forceinline__ void epilogue_half(const GemmArgs& a, const BarsT* bs
     const int which = tile / a.H, h = tile - which * a.H;   // 0 q, 1 k, 2 v; head h
     const int j = r >> 1;                                   // pair index (frequency)
     const int feat = j + (r & 1) * 64;                      // feature within the head
-    // rotation frequency base^(-2j/128) with base 10000, angle reduced in double
     uint16_t* cache = which == 1 ? a.k_cache : a.v_cache;
     // 16 tokens at a time: their cache rows (vector loads), rotations
     // (cos, sin of the token's angle for frequency j, from the forward's
