@@ -172,3 +172,92 @@ def test_merge_combine_and_rescale_refuse(mb):
         mb.medusa_attention_rescale(lses, 0, torch.zeros(11, 8))
     with pytest.raises(ValueError):
         mb.medusa_attention_rescale(lses.double(), 0, torch.zeros(10, 8))
+
+
+# The base forward and the generation loop check their arguments against the
+# model's sizes before anything reaches the C ABI, so a stand-in model with
+# the sizes (D 128: one head; F 256; V 16; two layers) is enough here.
+_DEC_D, _DEC_V, _DEC_LAYERS, _DEC_LCAP = 128, 16, 2, 40
+
+
+@pytest.fixture(scope="module")
+def dec_model(mb):
+    from types import SimpleNamespace
+    return SimpleNamespace(D=_DEC_D, F=256, V=_DEC_V, tensors=[{}] * _DEC_LAYERS, c=mb.DecoderModel())
+
+
+def _decode_args(tree, Bd=2, **over):
+    cache = (_DEC_LAYERS, Bd, _DEC_D // 128, _DEC_LCAP, 128)
+    a = dict(toks=torch.zeros(Bd, tree.T, dtype=i32), kc=torch.zeros(cache, dtype=bf), vc=torch.zeros(cache, dtype=bf),
+             lens=torch.zeros(Bd, dtype=i32), logits=torch.zeros(Bd * tree.T, _DEC_V), hidden=None,
+             ws=torch.zeros(4096, dtype=torch.uint8))
+    a.update(over)
+    return a
+
+
+DECODE_CASES = {
+    "tree tokens of another tree": lambda t: dict(toks=torch.zeros(2, t.T + 1, dtype=i32)),
+    "tree tokens int64": lambda t: dict(toks=torch.zeros(2, t.T, dtype=torch.int64)),
+    "cache of another layer count": lambda t: dict(kc=torch.zeros(_DEC_LAYERS + 1, 2, 1, _DEC_LCAP, 128, dtype=bf)),
+    "cache fp32": lambda t: dict(vc=torch.zeros(_DEC_LAYERS, 2, 1, _DEC_LCAP, 128)),
+    "v cache shorter than k cache": lambda t: dict(vc=torch.zeros(_DEC_LAYERS, 2, 1, _DEC_LCAP - 1, 128, dtype=bf)),
+    "cache not contiguous": lambda t: dict(kc=torch.zeros(_DEC_LAYERS, 2, 1, 128, _DEC_LCAP, dtype=bf).transpose(3, 4)),
+    "lengths for another batch": lambda t: dict(lens=torch.zeros(3, dtype=i32)),
+    "logits too short": lambda t: dict(logits=torch.zeros(2 * t.T - 1, _DEC_V)),
+    "hidden of the wrong width": lambda t: dict(hidden=torch.zeros(2 * t.T, _DEC_D + 1)),
+}
+
+
+def _decode(mb, tree, model, a):
+    mb.medusa_tree_decode(tree, model, a["toks"], a["kc"], a["vc"], a["lens"], a["logits"], a["ws"], hidden=a["hidden"])
+
+
+@pytest.mark.parametrize("case", sorted(DECODE_CASES))
+def test_tree_decode_refuses(mb, tree, dec_model, case):
+    # each case fails its own check, before the one on where tensors live
+    with pytest.raises(ValueError) as e:
+        _decode(mb, tree, dec_model, _decode_args(tree, **DECODE_CASES[case](tree)))
+    assert "CUDA tensors" not in str(e.value)
+
+
+def test_tree_decode_well_formed_reaches_the_device_check(mb, tree, dec_model):
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        _decode(mb, tree, dec_model, _decode_args(tree, hidden=torch.zeros(2 * tree.T, _DEC_D)))
+
+
+def _gen_args(tree, **over):
+    cache = (_DEC_LAYERS, 1, _DEC_D // 128, _DEC_LCAP, 128)
+    a = dict(W1=torch.zeros(tree.K, _DEC_D, _DEC_D, dtype=bf), b1=torch.zeros(tree.K, _DEC_D, dtype=bf),
+             Wout=torch.zeros(tree.K, _DEC_V, _DEC_D, dtype=bf), prompt=[1, 2, 3], n_new=4,
+             kc=torch.zeros(cache, dtype=bf), vc=torch.zeros(cache, dtype=bf), uniforms=None,
+             ws=torch.zeros(4096, dtype=torch.uint8))
+    a.update(over)
+    return a
+
+
+GENERATE_CASES = {
+    "W1 for another head count": lambda t: dict(W1=torch.zeros(t.K + 1, _DEC_D, _DEC_D, dtype=bf)),
+    "b1 fp32": lambda t: dict(b1=torch.zeros(t.K, _DEC_D)),
+    "Wout over another vocabulary": lambda t: dict(Wout=torch.zeros(t.K, _DEC_V + 1, _DEC_D, dtype=bf)),
+    "caches for two sequences": lambda t: dict(kc=torch.zeros(_DEC_LAYERS, 2, 1, _DEC_LCAP, 128, dtype=bf)),
+    "empty prompt": lambda t: dict(prompt=[]),
+    "nothing to generate": lambda t: dict(n_new=0),
+    "fewer uniforms than steps": lambda t: dict(uniforms=[0.5] * 3),
+}
+
+
+def _generate(mb, tree, model, a):
+    mb.medusa_generate(tree, model, a["W1"], a["b1"], a["Wout"], a["prompt"], a["n_new"], a["kc"], a["vc"],
+                       mb.MEDUSA_TYPICAL, temperature=0.7, uniforms=a["uniforms"], ws=a["ws"])
+
+
+@pytest.mark.parametrize("case", sorted(GENERATE_CASES))
+def test_generate_refuses(mb, tree, dec_model, case):
+    with pytest.raises(ValueError) as e:
+        _generate(mb, tree, dec_model, _gen_args(tree, **GENERATE_CASES[case](tree)))
+    assert "CUDA tensors" not in str(e.value)
+
+
+def test_generate_well_formed_reaches_the_device_check(mb, tree, dec_model):
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        _generate(mb, tree, dec_model, _gen_args(tree, uniforms=[0.5] * 4))
