@@ -627,6 +627,8 @@ def make_step_args(tree: Tree, t: dict, mode: int, temperature=0.0, eps=0.09, al
                         ("best_path", (B,)), ("accept_len", (B,)), ("next_token", (B,)),
                         ("accepted_tokens", (B, tree.D + 1))):
         _spec(name, t[name], shape, torch.int32)
+    if t.get("uniforms") is not None:
+        _spec("uniforms", t["uniforms"], (B,), torch.float32)
     a = StepArgs()
     a.tree = tree.handle
     a.B, a.d = t["h"].shape
@@ -647,7 +649,6 @@ def make_step_args(tree: Tree, t: dict, mode: int, temperature=0.0, eps=0.09, al
     a._shape = {"B": B, "d": a.d, "V": V, "T": T, "D": tree.D, "layers": layers, "H": H, "hd": hd,
                 "dtype": t["h"].dtype}
     if t.get("uniforms") is not None:
-        _spec("uniforms", t["uniforms"], (B,), torch.float32)
         a.uniforms = _p(t["uniforms"]).value
     return a
 

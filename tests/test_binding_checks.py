@@ -261,3 +261,82 @@ def test_generate_refuses(mb, tree, dec_model, case):
 def test_generate_well_formed_reaches_the_device_check(mb, tree, dec_model):
     with pytest.raises(ValueError, match="CUDA tensors"):
         _generate(mb, tree, dec_model, _gen_args(tree, uniforms=[0.5] * 4))
+
+
+# The step's arguments (make_step_args): every field against the tree and
+# the head/attention shapes (layers 2, H 1, hd 128, Lcap 40).
+def _step(tree, **over):
+    L_, H_, hd_, Lc = 2, 1, 128, 40
+    T, P, D = tree.T, tree.P, tree.D
+    a = dict(h=torch.zeros(B, d, dtype=bf), W1=torch.zeros(tree.K, d, d, dtype=bf), b1=torch.zeros(tree.K, d, dtype=bf),
+             Wout=torch.zeros(tree.K, V, d, dtype=bf), root_tokens=torch.zeros(B, dtype=i32),
+             q=torch.zeros(L_, B, T, H_, hd_, dtype=bf), k_cache=torch.zeros(L_, B, H_, Lc, hd_, dtype=bf),
+             v_cache=torch.zeros(L_, B, H_, Lc, hd_, dtype=bf), seq_lens=torch.zeros(B, dtype=i32),
+             base_logits=torch.zeros(B, T, V), topk_ids=torch.zeros(B, tree.K, tree.topk, dtype=i32),
+             topk_vals=torch.zeros(B, tree.K, tree.topk), tree_tokens=torch.zeros(B, T, dtype=i32),
+             candidates=torch.zeros(B, P, D + 1, dtype=i32), position_ids=torch.zeros(B, T, dtype=i32),
+             attn_out=torch.zeros(L_, B, T, H_, hd_), best_path=torch.zeros(B, dtype=i32),
+             accept_len=torch.zeros(B, dtype=i32), accepted_tokens=torch.zeros(B, D + 1, dtype=i32),
+             next_token=torch.zeros(B, dtype=i32), uniforms=None)
+    a.update(over)
+    return a
+
+
+STEP_CASES = {
+    "Wout for another head count": lambda t: dict(Wout=torch.zeros(t.K + 1, V, d, dtype=bf)),
+    "q fp32 with bf16 h": lambda t: dict(q=torch.zeros(2, B, t.T, 1, 128)),
+    "base logits over another vocabulary": lambda t: dict(base_logits=torch.zeros(B, t.T, V + 1)),
+    "root tokens int64": lambda t: dict(root_tokens=torch.zeros(B, dtype=torch.int64)),
+    "candidates for another path count": lambda t: dict(candidates=torch.zeros(B, t.P + 1, t.D + 1, dtype=i32)),
+    "accepted tokens too short": lambda t: dict(accepted_tokens=torch.zeros(B, t.D, dtype=i32)),
+    "position ids for another tree": lambda t: dict(position_ids=torch.zeros(B, t.T + 1, dtype=i32)),
+    "uniforms for another batch": lambda t: dict(uniforms=torch.zeros(B + 1)),
+}
+
+
+@pytest.mark.parametrize("case", sorted(STEP_CASES))
+def test_step_args_refuse(mb, tree, case):
+    with pytest.raises(ValueError) as e:
+        mb.make_step_args(tree, _step(tree, **STEP_CASES[case](tree)), mb.MEDUSA_GREEDY)
+    assert "CUDA tensors" not in str(e.value)
+
+
+def test_step_args_well_formed_reach_the_device_check(mb, tree):
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        mb.make_step_args(tree, _step(tree, uniforms=torch.zeros(B)), mb.MEDUSA_TYPICAL)
+
+
+# The host-buffer step checks its host buffers against the step's shapes
+# before anything is enqueued.
+def _host_step_args(mb, tree):
+    a = mb.StepArgs()
+    a._shape = {"B": B, "d": d, "V": V, "T": tree.T, "D": tree.D, "layers": 2, "H": 1, "hd": 128, "dtype": bf}
+    return a
+
+
+HOST_CASES = {
+    "an unknown input": lambda t: ({"k_cache": torch.zeros(1)}, {}),
+    "q of another tree": lambda t: ({"q": torch.zeros(2, B, t.T + 1, 1, 128, dtype=bf)}, {}),
+    "tree rows fp32": lambda t: ({"k_tree": torch.zeros(2, B, 1, t.T, 128)}, {}),
+    "base logits over another vocabulary": lambda t: ({"base_logits": torch.zeros(B, t.T, V - 1)}, {}),
+    "accepted tokens too short": lambda t: ({}, {"accepted_tokens": torch.zeros(B, t.D, dtype=i32)}),
+    "lengths out as int64": lambda t: ({}, {"seq_lens": torch.zeros(B, dtype=torch.int64)}),
+}
+
+
+@pytest.mark.parametrize("case", sorted(HOST_CASES))
+def test_host_step_refuses(mb, tree, case):
+    host_in, host_out = HOST_CASES[case](tree)
+    with pytest.raises(ValueError):
+        mb.medusa_step_host(_host_step_args(mb, tree), torch.zeros(16, dtype=torch.uint8), host_in, host_out)
+
+
+def test_host_step_well_formed_passes_the_buffer_checks(mb, tree):
+    # well-formed host buffers get past every buffer check (here, without a GPU, the failure comes later
+    # and is not one of those checks)
+    host_in = {"h": torch.zeros(B, d, dtype=bf), "q": torch.zeros(2, B, tree.T, 1, 128, dtype=bf),
+               "base_logits": torch.zeros(B, tree.T, V)}
+    host_out = {"accepted_tokens": torch.zeros(B, tree.D + 1, dtype=i32), "seq_lens": torch.zeros(B, dtype=i32)}
+    with pytest.raises(Exception) as e:
+        mb.medusa_step_host(_host_step_args(mb, tree), torch.zeros(16, dtype=torch.uint8), host_in, host_out)
+    assert not isinstance(e.value, ValueError), e.value
