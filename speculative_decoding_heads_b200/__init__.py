@@ -508,8 +508,26 @@ class Decoder:
     once when the model is set up) into the layout the kernels read."""
 
     def __init__(self, embed, layers, final_norm, lm_head):
+        # Every tensor's shape against D, F and V before anything is packed: the kernels read
+        # D x F (and so on) elements from each pointer.
+        _require(isinstance(embed, torch.Tensor) and embed.dim() == 2, "embed must be [V, D]")
         V, D = embed.shape
+        _require(D > 0 and D % 128 == 0, f"D = {D}: the model's width must be a multiple of the head size 128")
+        _require(len(layers) >= 1, "the model needs at least one layer")
+        _require(isinstance(layers[0].get("W_gate"), torch.Tensor) and layers[0]["W_gate"].dim() == 2,
+                 "W_gate must be [F, D]")
         F = layers[0]["W_gate"].shape[0]
+        for name, t, shape in (("lm_head", lm_head, (V, D)), ("final_norm", final_norm, (D,))):
+            _require(isinstance(t, torch.Tensor) and tuple(t.shape) == shape,
+                     f"{name} must have shape {shape}")
+        want = {"attn_norm": (D,), "mlp_norm": (D,), "Wq": (D, D), "Wk": (D, D), "Wv": (D, D), "Wo": (D, D),
+                "W_gate": (F, D), "W_up": (F, D), "W_down": (D, F)}
+        for i, ly in enumerate(layers):
+            for name, shape in want.items():
+                t = ly.get(name)
+                _require(isinstance(t, torch.Tensor) and tuple(t.shape) == shape,
+                         f"layer {i}: {name} must have shape {shape}"
+                         + (f", got {tuple(t.shape)}" if isinstance(t, torch.Tensor) else ""))
         dev = embed.device
         iq = torch.tensor(medusa_decoder_pack_rows(0, D), dtype=torch.long, device=dev)
         igu = torch.tensor(medusa_decoder_pack_rows(1, 2 * F), dtype=torch.long, device=dev)

@@ -340,3 +340,45 @@ def test_host_step_well_formed_passes_the_buffer_checks(mb, tree):
     with pytest.raises(Exception) as e:
         mb.medusa_step_host(_host_step_args(mb, tree), torch.zeros(16, dtype=torch.uint8), host_in, host_out)
     assert not isinstance(e.value, ValueError), e.value
+
+
+# The base model's weights are checked against D, F and V before they are
+# packed (D 128, F 256, V 16, two layers).
+def _dec_weights(**over):
+    Dm, Fm, Vm = 128, 256, 16
+    layer = dict(attn_norm=torch.ones(Dm), mlp_norm=torch.ones(Dm), Wq=torch.zeros(Dm, Dm), Wk=torch.zeros(Dm, Dm),
+                 Wv=torch.zeros(Dm, Dm), Wo=torch.zeros(Dm, Dm), W_gate=torch.zeros(Fm, Dm), W_up=torch.zeros(Fm, Dm),
+                 W_down=torch.zeros(Dm, Fm))
+    a = dict(embed=torch.zeros(Vm, Dm), layers=[dict(layer), dict(layer)], final_norm=torch.ones(Dm),
+             lm_head=torch.zeros(Vm, Dm))
+    for k, v in over.items():
+        if k.startswith("layer1_"):
+            a["layers"][1][k[len("layer1_"):]] = v
+        else:
+            a[k] = v
+    return a
+
+
+DECODER_CASES = {
+    "width not a multiple of 128": dict(embed=torch.zeros(16, 96)),
+    "LM head over another vocabulary": dict(lm_head=torch.zeros(17, 128)),
+    "final norm too short": dict(final_norm=torch.ones(127)),
+    "second layer's down projection too narrow": dict(layer1_W_down=torch.zeros(128, 128)),
+    "second layer's up projection of another width": dict(layer1_W_up=torch.zeros(128, 128)),
+    "second layer without an output projection": dict(layer1_Wo=None),
+    "second layer's attention norm too long": dict(layer1_attn_norm=torch.ones(129)),
+}
+
+
+@pytest.mark.parametrize("case", sorted(DECODER_CASES))
+def test_decoder_refuses_inconsistent_weights(mb, case):
+    a = _dec_weights(**DECODER_CASES[case])
+    with pytest.raises(ValueError) as e:
+        mb.Decoder(a["embed"], a["layers"], a["final_norm"], a["lm_head"])
+    assert "CUDA tensors" not in str(e.value)
+
+
+def test_decoder_well_formed_reaches_the_device_check(mb):
+    a = _dec_weights()
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        mb.Decoder(a["embed"], a["layers"], a["final_norm"], a["lm_head"])
