@@ -36,14 +36,27 @@ def _rope_ref(x, pos, base=D.ROPE_BASE):
     return np.concatenate([z.real, z.imag], axis=-1)
 
 
-def _causal_forward(tokens, embed, layers, k_caches, v_caches, L, H):
-    """A plain causal decoder over a token sequence at positions L.. with a prefix cache."""
+def _rms_ref(x, w):
+    """RMSNorm by torch's own routine (eps 1e-6, as the pages' Vicuna bases use)."""
+    t = torch.from_numpy(np.asarray(x, dtype=np.float64))
+    return torch.nn.functional.rms_norm(t, (t.shape[-1],), weight=torch.from_numpy(np.asarray(w, np.float64)),
+                                        eps=1e-6).numpy()
+
+
+def _silu_ref(x):
+    return torch.nn.functional.silu(torch.from_numpy(np.asarray(x, dtype=np.float64))).numpy()
+
+
+def _causal_forward(tokens, embed, layers, k_caches, v_caches, L, H, final_norm=None, lm_head=None):
+    """A plain causal decoder over a token sequence at positions L.. with a prefix cache, written
+    without the oracle's helpers (torch's RMSNorm, SiLU and attention; RoPE as complex
+    multiplication).  Returns the residual stream, and the logits when the head is given."""
     x = embed[np.asarray(tokens)].astype(np.float64)
     n, Dm = x.shape
     hd = Dm // H
     pos = L + np.arange(n)
     for li, ly in enumerate(layers):
-        h = D.rms_norm(x, ly["attn_norm"])
+        h = _rms_ref(x, ly["attn_norm"])
         q = _rope_ref((h @ ly["Wq"].T).reshape(n, H, hd).transpose(1, 0, 2), pos)
         k = _rope_ref((h @ ly["Wk"].T).reshape(n, H, hd).transpose(1, 0, 2), pos)
         v = (h @ ly["Wv"].T).reshape(n, H, hd).transpose(1, 0, 2)
@@ -54,9 +67,11 @@ def _causal_forward(tokens, embed, layers, k_caches, v_caches, L, H):
             torch.from_numpy(q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None],
             attn_mask=mask[None, None])[0].numpy()
         x = x + att.transpose(1, 0, 2).reshape(n, Dm) @ ly["Wo"].T
-        hm = D.rms_norm(x, ly["mlp_norm"])
-        x = x + (O.silu(hm @ ly["W_gate"].T) * (hm @ ly["W_up"].T)) @ ly["W_down"].T
-    return x
+        hm = _rms_ref(x, ly["mlp_norm"])
+        x = x + (_silu_ref(hm @ ly["W_gate"].T) * (hm @ ly["W_up"].T)) @ ly["W_down"].T
+    if lm_head is None:
+        return x
+    return x, _rms_ref(x, final_norm) @ np.asarray(lm_head).T
 
 
 @pytest.mark.parametrize("choices,K,topk,L", [(WORKED, 2, 2, 9), (O.ranksum_choices(4, 3, 20), 4, 3, 17),
@@ -71,12 +86,13 @@ def test_tree_forward_equals_causal_forward_along_every_path(choices, K, topk, L
     tokens = rng.integers(0, Vv, size=T)
     kcs = [rng.normal(size=(H, L + T + 3, hd)) for _ in range(nl)]
     vcs = [rng.normal(size=(H, L + T + 3, hd)) for _ in range(nl)]
-    logits, hid, kc_out, _ = D.tree_forward(tr, tokens, embed, layers, np.ones(Dm), rng.normal(size=(Vv, Dm)),
-                                            kcs, vcs, L, H)
+    final_norm, lm_head = 1.0 + 0.1 * rng.normal(size=Dm), rng.normal(size=(Vv, Dm))
+    logits, hid, kc_out, _ = D.tree_forward(tr, tokens, embed, layers, final_norm, lm_head, kcs, vcs, L, H)
     for p in range(tr["P"]):
         path = [n for n in tr["retrieve"][p] if n >= 0]
-        ref = _causal_forward(tokens[path], embed, layers, kcs, vcs, L, H)
+        ref, ref_logits = _causal_forward(tokens[path], embed, layers, kcs, vcs, L, H, final_norm, lm_head)
         assert np.allclose(hid[path], ref, atol=1e-10, rtol=1e-10), p
+        assert np.allclose(logits[path], ref_logits, atol=1e-9, rtol=1e-9), p
     # the prefix rows of the caches are untouched; the tree rows now hold the tree's keys
     for li in range(nl):
         assert np.array_equal(kc_out[li][:, :L], kcs[li][:, :L])
@@ -225,3 +241,75 @@ def test_sampled_generation_draws_from_the_tempered_distribution():
         z = logits[node] / 1.5
         w = np.exp(z - z.max())
         assert got[pos] == O.sample_index(w, u[s])   # the next step's root
+
+
+# ---- planted mistakes in the decoder oracle: each must fail the path pin ----
+def _flawed_layer(flaw):
+    """The oracle's decoder layer with one plausible mistake planted."""
+    def layer(tree, x, ly, k_cache, v_cache, L_b, H):
+        x = np.asarray(x, dtype=np.float64)
+        T, Dm = x.shape
+        hd = Dm // H
+        depth = np.asarray(tree["depth"])
+        pos = depth if flaw == "positions without the prefix length" else L_b + depth
+        kc, vc = np.array(k_cache, dtype=np.float64), np.array(v_cache, dtype=np.float64)
+        h = D.rms_norm(x, ly["attn_norm"])
+        q = (h @ ly["Wq"].T).reshape(T, H, hd).transpose(1, 0, 2)
+        k = (h @ ly["Wk"].T).reshape(T, H, hd).transpose(1, 0, 2)
+        v = (h @ ly["Wv"].T).reshape(T, H, hd).transpose(1, 0, 2)
+        q = D.rope(q, pos)
+        if flaw != "rotation of q only":
+            k = D.rope(k, pos)
+        rows = L_b + (depth if flaw == "tree keys at rows L + depth" else np.arange(T))
+        kc[:, rows, :] = k
+        vc[:, rows, :] = v
+        att = np.stack([O.tree_attention_slice(tree, q[e], kc[e], vc[e], L_b, O.attention_scale(hd))
+                        for e in range(H)], axis=1)
+        proj = att.reshape(T, Dm) @ ly["Wo"].T
+        x = proj if flaw == "no residual around attention" else x + proj
+        hm = h if flaw == "feed-forward on the attention's normalised input" else D.rms_norm(x, ly["mlp_norm"])
+        x = x + D.swiglu_mlp(hm, ly["W_gate"], ly["W_up"], ly["W_down"])
+        return x, kc, vc
+    return layer
+
+
+def _forward_without_final_norm(tree, tokens, embed, layers, final_norm, lm_head, k_caches, v_caches, L_b, H):
+    x = np.asarray(embed, dtype=np.float64)[np.asarray(tokens)]
+    for li, ly in enumerate(layers):
+        x, _, _ = D.decoder_layer(tree, x, ly, k_caches[li], v_caches[li], L_b, H)
+    return x @ np.asarray(lm_head).T, x, None, None
+
+
+def _rope_adjacent_pairs(x, pos, base=D.ROPE_BASE):
+    """RoPE pairing dimensions (2i, 2i + 1) instead of (i, i + hd/2)."""
+    x = np.asarray(x, dtype=np.float64)
+    hd = x.shape[-1]
+    inv = base ** (-np.arange(hd // 2) * 2.0 / hd)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * inv[None, :]
+    a, b = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2], y[..., 1::2] = a * np.cos(ang) - b * np.sin(ang), a * np.sin(ang) + b * np.cos(ang)
+    return y
+
+
+DECODER_MUTANTS = {
+    **{f: ("decoder_layer", _flawed_layer(f)) for f in (
+        "positions without the prefix length", "rotation of q only", "tree keys at rows L + depth",
+        "no residual around attention", "feed-forward on the attention's normalised input")},
+    "no final norm before the LM head": ("tree_forward", _forward_without_final_norm),
+    "rotation pairs adjacent dimensions": ("rope", _rope_adjacent_pairs),
+}
+
+
+def test_unflawed_copy_passes_the_path_pin(monkeypatch):
+    # the harness itself: the layer copy above, with no flaw planted, satisfies the pin
+    monkeypatch.setattr(D, "decoder_layer", _flawed_layer(None))
+    test_tree_forward_equals_causal_forward_along_every_path(WORKED, 2, 2, 9)
+
+
+@pytest.mark.parametrize("name", sorted(DECODER_MUTANTS))
+def test_decoder_mutants_are_caught(monkeypatch, name):
+    attr, fn = DECODER_MUTANTS[name]
+    monkeypatch.setattr(D, attr, fn)
+    with pytest.raises(AssertionError):
+        test_tree_forward_equals_causal_forward_along_every_path(WORKED, 2, 2, 9)
